@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the fused causal GQA attention, forward + backward, on B200.
+
+One step = the whole hot path over one batch of the workload: the forward
+kernel, then the three backward stages (preprocess, main, dQ finalize), all
+through the C ABI on one stream.  The metric is attention TFLOP/s with causal
+FLOPs counted as half of dense (fwd 2*B*Hq*S^2*D, bwd 5*B*Hq*S^2*D).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+        python bench.py --impl reference ...   (the fp64 CPU oracle, host cores)
+Under torchrun (N > 1) every rank runs its own batch of the workload (weak
+scaling; no collective on the data path).  Timing: CUDA events around each
+step on the launching stream, L2 flushed (256 MiB write) before every step,
+outside the events; the reported time is the max over ranks.  Rank 0 prints one
+JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+P_NOM_TFLOPS = 2250.0  # B200 dense bf16, NVIDIA's published figure
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "attention fwd / bwd TFLOP/s (bf16, causal) and % of B200 tensor peak"
+KERNEL_SOURCES = ("attn_fwd.cuh", "attn_bwd.cuh", "sm100_ptx.cuh", "axis_attn.cu")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "causal_attention_fwd_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel, {})
+    if e.get("workload") == workload and e.get("source_hash") == kernel_source_hash():
+        return e.get("dram_bytes_per_launch")
+    return None
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons of one GPU via NVML."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            handle = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    handle = h
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nvml, self.h = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, do not guess
+            self.err = repr(e)
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                t = time.time()
+                mhz = n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)
+                rs = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                pw = n.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((t, mhz, rs, pw))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.th = threading.Thread(target=self._run, daemon=True)
+            self.th.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.th.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples[-5:]
+        mhz = statistics.median(s[1] for s in inside) if inside else None
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = [k for k, v in self.REASONS.items() if bits & v and k != "gpu_idle"]
+        return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside),
+                "power_w_max": max((s[3] for s in inside), default=None)}
+
+
+# ----------------------------------------------------------- reference arm
+def cpu_sample(w, budget_s: float, max_heads: int | None = None):
+    """The oracle, as it stands, on whole query heads of the workload (each with
+    its kv head), until `budget_s` of CPU time has passed.  Returns TFLOP/s
+    counted like the GPU metric, the threads used and a description."""
+    import oracle
+    from causal_attention_fwd_b200.synthetic import workload_inputs
+
+    q, k, v, do = workload_inputs(w)
+    G = w.Hq // w.Hkv
+    per_head = (w.fwd_flops + w.bwd_flops) / (w.B * w.Hq)
+    done, t_total, heads = 0, 0.0, []
+    n = 0
+    while n == 0 or (t_total < budget_s and (max_heads is None or n < max_heads)):
+        b, h = n % w.B, (n // w.B) % w.Hq
+        sl = lambda t, hh: t[b:b + 1, :, hh:hh + 1].contiguous()  # noqa: E731
+        qs, ks, vs, dos = sl(q, h), sl(k, h // G), sl(v, h // G), sl(do, h)
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qs, ks, vs, w.scale, w.causal)
+        oracle.attn_bwd(qs, ks, vs, dos, w.scale, w.causal)
+        t_total += time.perf_counter() - t0
+        done += 1
+        heads.append((b, h))
+        n += 1
+    tflops = done * per_head / t_total / 1e12
+    desc = (f"{done} whole query head(s) of the workload, each fwd+bwd with its kv head "
+            f"(B=1 Hq=1 Hkv=1 S={w.S} D={w.D}); {t_total:.1f} s")
+    return tflops, oracle.max_threads(), desc, t_total
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return 0
+    from causal_attention_fwd_b200.synthetic import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    import oracle
+
+    oracle.build()
+    times, vals = [], []
+    desc, cores = "", oracle.max_threads()
+    for s in range(args.warmup + args.steps):
+        v, cores, desc, t = cpu_sample(w, 0.0, max_heads=1)  # one head per step
+        if s >= args.warmup:
+            times.append(t)
+            vals.append(v)
+    per_head = (w.fwd_flops + w.bwd_flops) / (w.B * w.Hq)
+    value = per_head * len(times) / sum(times) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,sigma^2), bf16-rounded)",
+        "config": {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "causal": w.causal, "sample_per_step": "one whole query head (fwd+bwd)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "one whole query head of the workload per step, fwd+bwd, fp64"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llm1b")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import ctypes
+
+    import torch
+    import torch.distributed as dist
+
+    import causal_attention_fwd_b200 as aa
+    from causal_attention_fwd_b200.synthetic import WORKLOAD_SEED, WORKLOADS, workload_inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = WORKLOADS[args.workload]
+    B, Hq, Hkv, S, D = w.B, w.Hq, w.Hkv, w.S, w.D
+    q_h, k_h, v_h, do_h = workload_inputs(w, seed=WORKLOAD_SEED[w.name] + 100 * rank)
+    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, S), device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = aa.axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D)
+    ws = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    causal = int(w.causal)
+
+    def check(rc, what):
+        if rc:
+            raise aa.AxisAttnError(rc, what)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        check(aa.axis_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                               B, Hq, Hkv, S, D, w.scale, causal, sp), "fwd")
+        if ev:
+            ev[1].record(stream)
+        check(aa.axis_attn_bwd_prepare(o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, Hq, Hkv, S, D,
+                                       ws.data_ptr(), ws_bytes, sp), "bwd_prepare")
+        if ev:
+            ev[2].record(stream)
+        check(aa.axis_attn_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(),
+                                    dv.data_ptr(), B, Hq, Hkv, S, D, w.scale, causal, ws.data_ptr(),
+                                    ws_bytes, sp), "bwd_main")
+        if ev:
+            ev[3].record(stream)
+        check(aa.axis_attn_bwd_finalize(dq.data_ptr(), B, Hq, Hkv, S, D, ws.data_ptr(), ws_bytes, sp),
+              "bwd_finalize")
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    aa.check_status(stream)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.05)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for s in range(args.steps):
+        flush.fill_(s & 0xFF)  # L2 flush, outside the events
+        step(evs[s])
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    aa.check_status(stream)
+
+    per = torch.tensor([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs], dtype=torch.float64)
+    totals = per.sum(0)  # ms per stage over all steps
+    step_total = torch.tensor([sum(e[0].elapsed_time(e[4]) for e in evs)], dtype=torch.float64)
+    if world > 1:
+        t = torch.cat([step_total, totals]).to(dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t = t.cpu()
+        step_total, totals = t[:1], t[1:]
+    total_ms = float(step_total[0])
+    K = args.steps
+    flops_step = w.fwd_flops + w.bwd_flops
+    value = world * flops_step * K / (total_ms * 1e-3) / 1e12
+    names = ["attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_kernel", "attn_bwd_dq_convert_kernel"]
+    avg_ms = [float(totals[i]) / K for i in range(4)]
+    fwd_tf = w.fwd_flops / (avg_ms[0] * 1e-3) / 1e12
+    bwd_ms = sum(avg_ms[1:])
+    bwd_tf = w.bwd_flops / (bwd_ms * 1e-3) / 1e12
+    pk, pk_src = peaks()
+    p_meas = pk["bf16_tflops"]
+
+    # dominant kernel and its roofline
+    dom = max(range(4), key=lambda i: avg_ms[i])
+    dom_flops = w.fwd_flops if dom == 0 else w.bwd_flops
+    roof = None
+    if dom in (0, 2):
+        achieved = dom_flops / (avg_ms[dom] * 1e-3) / 1e12
+        roof = {"kernel": names[dom], "bound": "tensor", "achieved": achieved, "peak": p_meas,
+                "peak_source": f"{pk_src} bf16_tflops (burst)", "unit": "TFLOP/s",
+                "frac": achieved / p_meas, "frac_of_nominal_2250": achieved / P_NOM_TFLOPS,
+                "traffic": profiled_traffic(names[dom], w.name),
+                "flops_per_launch": dom_flops, "avg_launch_ms": avg_ms[dom]}
+
+    # ---- end to end through the public API, host buffers, copies inside the timed region
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = lambda t: t.pin_memory()  # noqa: E731
+        hq, hk, hv, hdo = pin(q_h), pin(k_h), pin(v_h), pin(do_h)
+        ho, hl = torch.empty_like(hq).pin_memory(), torch.empty((B, Hq, S), dtype=torch.float32).pin_memory()
+        hdq, hdk, hdv = (torch.empty_like(t).pin_memory() for t in (hq, hk, hv))
+        qq, kk, vv, dd = (torch.empty_like(t) for t in (q, k, v, do))
+
+        def e2e_step():
+            for dst, src in ((qq, hq), (kk, hk), (vv, hv), (dd, hdo)):
+                dst.copy_(src, non_blocking=True)
+            oo, ll = aa.attention_forward(qq, kk, vv, causal=w.causal, scale=w.scale, out=o, lse=lse)
+            g = aa.attention_backward(qq, kk, vv, oo, ll, dd, causal=w.causal, scale=w.scale, workspace=ws,
+                                      grads=(dq, dk, dv))
+            for dst, src in ((ho, oo), (hl, ll), (hdq, g[0]), (hdk, g[1]), (hdv, g[2])):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64)
+        if world > 1:
+            ems = ems.to(dev)
+            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+            ems = ems.cpu()
+        aa.check_status(stream)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
+        e2e = {"value": world * flops_step * args.e2e_steps / (float(ems[0]) * 1e-3) / 1e12,
+               "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": args.e2e_steps}
+
+    clocks = sampler.summary(t_wall0, t_wall1)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        tf, cores, desc, t = cpu_sample(w, args.cpu_budget)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,sigma^2), bf16-rounded; each rank its own batch)",
+            "config": {"workload": f"{w.name}: {w.describe()}", "B": B, "S": S, "Hq": Hq, "Hkv": Hkv,
+                       "D": D, "global_batch": B * world, "parallelism": f"replicas x{world} (no collective)",
+                       "l2": "flushed before every step (256 MiB write, outside the timed events)"},
+            "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+            "fwd_frac_of_nominal_2250": fwd_tf / P_NOM_TFLOPS, "bwd_frac_of_nominal_2250": bwd_tf / P_NOM_TFLOPS,
+            "fwd_frac_of_measured": fwd_tf / p_meas, "bwd_frac_of_measured": bwd_tf / p_meas,
+            "kernel_ms": dict(zip(names, avg_ms)),
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 4 * K, "clocks": clocks,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,24 @@
+"""B200 (sm_100a) fused causal GQA attention, forward and backward.
+
+The compute lives in ``libaxis_attn.so`` (hand-written CUDA, C ABI in
+``include/axis_attn.h``); ``binding`` is its ctypes front end.  Importing the
+package does not load the library; the first call does, and raises if it is
+missing (there is no CPU fallback).
+"""
+from .binding import (  # noqa: F401
+    EXPORTS,
+    AxisAttnError,
+    attention_backward,
+    attention_forward,
+    axis_attn_bwd,
+    axis_attn_bwd_finalize,
+    axis_attn_bwd_main,
+    axis_attn_bwd_prepare,
+    axis_attn_bwd_workspace_bytes,
+    axis_attn_fwd,
+    axis_attn_get_status,
+    axis_attn_strerror,
+    check_status,
+    library_path,
+    load,
+)

@@ -1,0 +1,310 @@
+// axis_attn.cu -- host side of the C ABI declared in include/axis_attn.h:
+// argument validation, TMA tensor maps, workspace layout and kernel launches.
+// All device work is in attn_fwd.cuh and attn_bwd.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/axis_attn.h"
+#include "attn_bwd.cuh"
+#include "attn_fwd.cuh"
+
+namespace axis_attn {
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Device check, cached per device: compute capability 10.0 only.
+int check_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AXIS_ATTN_ERR_CUDA;
+  static int cached[64];  // 0 unknown, 1 ok, 2 unsupported
+  if (dev < 0 || dev >= 64) return AXIS_ATTN_ERR_UNSUPPORTED;
+  if (cached[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return AXIS_ATTN_ERR_CUDA;
+    cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  *dev_out = dev;
+  return cached[dev] == 1 ? AXIS_ATTN_OK : AXIS_ATTN_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int Hq, int Hkv, int S, int D, float scale) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || Hq % Hkv != 0) return AXIS_ATTN_ERR_SHAPE;
+  if (!(std::isfinite(scale) && scale > 0.f)) return AXIS_ATTN_ERR_SHAPE;
+  if (D != 64 && D != 128) return AXIS_ATTN_ERR_UNSUPPORTED;
+  const long long elems = (long long)B * S * (Hq > Hkv ? Hq : Hkv) * D;
+  if (elems >= (1LL << 31)) return AXIS_ATTN_ERR_SHAPE;
+  return AXIS_ATTN_OK;
+}
+
+// 4-D map over a [B, S, H, D] bf16 tensor: dims (D, H, S, B), box (64, 1, rows, 1),
+// 128-byte swizzle, out-of-range rows read as zero.
+bool make_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int D, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct WsLayout {
+  size_t lse2, dr, dqacc, total;
+  int S_pad;
+};
+
+WsLayout ws_layout(int B, int Hq, int S, int D) {
+  WsLayout w;
+  w.S_pad = (S + 127) / 128 * 128;
+  const size_t rows = (size_t)B * Hq * w.S_pad;
+  w.lse2 = 0;
+  w.dr = round256(rows * 4);
+  w.dqacc = w.dr + round256(rows * 4);
+  w.total = w.dqacc + round256((size_t)B * Hq * S * D * 4);
+  return w;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+// `done` is a static of the calling template instantiation, so each kernel has
+// its own flags.
+template <typename K>
+int set_smem(K kernel, uint32_t bytes, int dev, bool (&done)[64]) {
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+      return AXIS_ATTN_ERR_CUDA;
+    done[dev] = true;
+  }
+  return AXIS_ATTN_OK;
+}
+
+template <int HD, bool CAUSAL>
+int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
+               cudaStream_t st, int dev) {
+  auto kern = attn_fwd_kernel<HD, CAUSAL>;
+  static bool done[64];
+  if (int rc = set_smem(kern, FwdCfg<HD>::SMEM, dev, done)) return rc;
+  const unsigned grid = (unsigned)a.n_qblocks * a.B * a.Hq;
+  kern<<<grid, 512, FwdCfg<HD>::SMEM, st>>>(mq, mk, mv, a);
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+template <int HD, bool CAUSAL>
+int launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                    const BwdArgs& a, cudaStream_t st, int dev) {
+  auto kern = attn_bwd_kernel<HD, CAUSAL>;
+  static bool done[64];
+  if (int rc = set_smem(kern, BwdCfg<HD>::SMEM, dev, done)) return rc;
+  const unsigned grid = (unsigned)((a.S + 127) / 128) * a.B * a.Hkv;
+  kern<<<grid, 512, BwdCfg<HD>::SMEM, st>>>(mq, mk, mv, mdo, a);
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace axis_attn
+
+using namespace axis_attn;
+
+extern "C" int axis_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                             int Hkv, int S, int D, float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o || !lse) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return AXIS_ATTN_ERR_ALIGN;
+  if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, B, S, Hq, D, 128) || !make_map(&mk, k, B, S, Hkv, D, 128) ||
+      !make_map(&mv, v, B, S, Hkv, D, 128))
+    return AXIS_ATTN_ERR_CUDA;
+  FwdArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.S = S;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  a.n_qblocks = (S + 255) / 256;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64)
+    return causal ? launch_fwd<64, true>(mq, mk, mv, a, st, dev) : launch_fwd<64, false>(mq, mk, mv, a, st, dev);
+  return causal ? launch_fwd<128, true>(mq, mk, mv, a, st, dev) : launch_fwd<128, false>(mq, mk, mv, a, st, dev);
+}
+
+extern "C" size_t axis_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
+  if (check_shape(B, Hq, Hkv, S, D, 1.f) != AXIS_ATTN_OK) return 0;
+  return ws_layout(B, Hq, S, D).total;
+}
+
+namespace {
+
+int check_ws(void* workspace, size_t workspace_bytes, const WsLayout& w) {
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < w.total)
+    return AXIS_ATTN_ERR_WORKSPACE;
+  return AXIS_ATTN_OK;
+}
+
+struct WsPtrs {
+  float *lse2, *dr, *dqacc;
+};
+
+WsPtrs ws_ptrs(void* workspace, const WsLayout& w) {
+  char* ws = static_cast<char*>(workspace);
+  return {reinterpret_cast<float*>(ws + w.lse2), reinterpret_cast<float*>(ws + w.dr),
+          reinterpret_cast<float*>(ws + w.dqacc)};
+}
+
+}  // namespace
+
+extern "C" int axis_attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, int Hkv,
+                                     int S, int D, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!o || !dO || !lse) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return AXIS_ATTN_ERR_ALIGN;
+  if (int rc = check_shape(B, Hq, Hkv, S, D, 1.f)) return rc;
+  const WsLayout w = ws_layout(B, Hq, S, D);
+  if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  const WsPtrs p = ws_ptrs(workspace, w);
+  const int rows = B * Hq * w.S_pad;
+  const size_t dq_vec4 = (size_t)B * Hq * S * D / 4;
+  const unsigned grid = (unsigned)((rows + 255) / 256);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto* ob = static_cast<const __nv_bfloat16*>(o);
+  const auto* db = static_cast<const __nv_bfloat16*>(dO);
+  if (D == 64)
+    attn_bwd_prep_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, p.lse2, p.dr, reinterpret_cast<float4*>(p.dqacc),
+                                                   dq_vec4, Hq, S, w.S_pad, rows);
+  else
+    attn_bwd_prep_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, p.lse2, p.dr, reinterpret_cast<float4*>(p.dqacc),
+                                                    dq_vec4, Hq, S, w.S_pad, rows);
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+extern "C" int axis_attn_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                                  int B, int Hq, int Hkv, int S, int D, float scale, int causal, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !dO || !dk || !dv) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv))
+    return AXIS_ATTN_ERR_ALIGN;
+  if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
+  const WsLayout w = ws_layout(B, Hq, S, D);
+  if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  const int BM = D == 64 ? BwdCfg<64>::BM : BwdCfg<128>::BM;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, B, S, Hq, D, BM) || !make_map(&mdo, dO, B, S, Hq, D, BM) ||
+      !make_map(&mk, k, B, S, Hkv, D, 128) || !make_map(&mv, v, B, S, Hkv, D, 128))
+    return AXIS_ATTN_ERR_CUDA;
+  const WsPtrs p = ws_ptrs(workspace, w);
+  BwdArgs a;
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.lse2 = p.lse2;
+  a.dr = p.dr;
+  a.dqacc = p.dqacc;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.S = S;
+  a.S_pad = w.S_pad;
+  a.scale = scale;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64)
+    return causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, a, st, dev)
+                  : launch_bwd_main<64, false>(mq, mk, mv, mdo, a, st, dev);
+  return causal ? launch_bwd_main<128, true>(mq, mk, mv, mdo, a, st, dev)
+                : launch_bwd_main<128, false>(mq, mk, mv, mdo, a, st, dev);
+}
+
+extern "C" int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, int D, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!dq) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(dq)) return AXIS_ATTN_ERR_ALIGN;
+  if (int rc = check_shape(B, Hq, Hkv, S, D, 1.f)) return rc;
+  const WsLayout w = ws_layout(B, Hq, S, D);
+  if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  const WsPtrs p = ws_ptrs(workspace, w);
+  const size_t n8 = (size_t)B * S * Hq * D / 8;
+  const unsigned grid = (unsigned)((n8 + 255) / 256 < 4096 ? (n8 + 255) / 256 : 4096);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64)
+    attn_bwd_dq_convert_kernel<64><<<grid, 256, 0, st>>>(p.dqacc, static_cast<__nv_bfloat16*>(dq), Hq, S, n8);
+  else
+    attn_bwd_dq_convert_kernel<128><<<grid, 256, 0, st>>>(p.dqacc, static_cast<__nv_bfloat16*>(dq), Hq, S, n8);
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+extern "C" int axis_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                             const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D,
+                             float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  // Validate everything first so that no stage runs when a later one would fail.
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return AXIS_ATTN_ERR_ALIGN;
+  if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
+  if (int rc = check_ws(workspace, workspace_bytes, ws_layout(B, Hq, S, D))) return rc;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  if (int rc = axis_attn_bwd_prepare(o, dO, lse, B, Hq, Hkv, S, D, workspace, workspace_bytes, stream)) return rc;
+  if (int rc = axis_attn_bwd_main(q, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, workspace,
+                                  workspace_bytes, stream))
+    return rc;
+  return axis_attn_bwd_finalize(dq, B, Hq, Hkv, S, D, workspace, workspace_bytes, stream);
+}
+
+extern "C" int axis_attn_get_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return AXIS_ATTN_ERR_CUDA;
+  unsigned int st = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&st, g_status, sizeof(st)) != cudaSuccess) return AXIS_ATTN_ERR_CUDA;
+  if (st != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return AXIS_ATTN_ERR_CUDA;
+  if (st != 0) return AXIS_ATTN_ERR_TIMEOUT;
+  return cudaGetLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+extern "C" const char* axis_attn_strerror(int code) {
+  switch (code) {
+    case AXIS_ATTN_OK: return "ok";
+    case AXIS_ATTN_ERR_NULL: return "a required pointer is NULL";
+    case AXIS_ATTN_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case AXIS_ATTN_ERR_SHAPE: return "invalid size, head ratio or scale";
+    case AXIS_ATTN_ERR_UNSUPPORTED: return "unsupported head dim (need 64 or 128) or device (need sm_100)";
+    case AXIS_ATTN_ERR_WORKSPACE: return "workspace NULL, not 256-byte aligned, or too small";
+    case AXIS_ATTN_ERR_CUDA: return "CUDA runtime or driver error";
+    case AXIS_ATTN_ERR_TIMEOUT: return "a device-side wait timed out";
+    default: return "unknown status";
+  }
+}

@@ -1,0 +1,131 @@
+/*
+ * axis_attn.h -- C ABI of the B200 (sm_100a) fused causal GQA softmax attention.
+ *
+ * The operation (forward and backward of scaled-dot-product softmax attention,
+ * causal mask optional, GQA head sharing, bf16 storage with fp32 accumulation,
+ * attention probabilities never written to device memory) is the fused flash
+ * attention of the "Axis" page (zyoralabs.com/axis, feature list: "fused flash
+ * attention, forward and backward"; "bf16 storage ... fp32 accumulation"), with
+ * KV groups from the same page's second code sample (n_heads / n_kv_heads) and
+ * the [B, S, H, D] tensor layout of the axiomlm page (PyPI, Quick Start section
+ * 8).  The pages give no formula; the library computes, for batch b, query head
+ * h, kv head kv = h / (Hq / Hkv), and query row i:
+ *
+ *   s_ij = scale * <Q[b,i,h,:], K[b,j,kv,:]>,  visible iff (!causal || j <= i)
+ *   LSE[b,h,i] = ln sum_{visible j} exp(s_ij)         (natural log, fp32)
+ *   P_ij = exp(s_ij - LSE[b,h,i]),  O[b,i,h,:] = sum_j P_ij V[b,j,kv,:]
+ *
+ * and the analytic gradients dQ, dK, dV of sum(dO * O), with dK and dV summed
+ * over the query heads of each kv group.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors: q, o, dO, dq are [B, S, Hq, D]; k, v, dk, dv are [B, S, Hkv, D];
+ *    all bf16, contiguous, row-major.  lse is fp32 [B, Hq, S].
+ *  - Pointers are DEVICE pointers owned by the caller and must be 16-byte
+ *    aligned.  The library allocates no device memory and keeps no pointer
+ *    after a call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *    is the legacy default stream), perform no host synchronisation and may be
+ *    captured in a CUDA graph.
+ *  - Requirements: B, Hq, Hkv, S >= 1; Hq % Hkv == 0; D in {64, 128};
+ *    scale finite and > 0; B*S*max(Hq,Hkv)*D < 2^31; the current device is
+ *    compute capability 10.0 (B200, sm_100a).
+ *  - Errors: a violated requirement returns a non-zero axis_attn_status before
+ *    anything is launched, and the outputs are left untouched.  A launch or
+ *    driver failure returns AXIS_ATTN_ERR_CUDA.  A device-side wait that runs
+ *    past its time limit (which signals a bug, never expected in use) makes the
+ *    kernel stop early, release its resources and set a device status word
+ *    that axis_attn_get_status() reports as AXIS_ATTN_ERR_TIMEOUT.
+ */
+#ifndef AXIS_ATTN_H
+#define AXIS_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    AXIS_ATTN_OK = 0,
+    AXIS_ATTN_ERR_NULL = 1,        /* a required pointer is NULL */
+    AXIS_ATTN_ERR_ALIGN = 2,       /* a pointer is not 16-byte aligned */
+    AXIS_ATTN_ERR_SHAPE = 3,       /* a size, head ratio or scale is invalid */
+    AXIS_ATTN_ERR_UNSUPPORTED = 4, /* D not in {64,128}, or not a CC 10.0 device */
+    AXIS_ATTN_ERR_WORKSPACE = 5,   /* workspace NULL, misaligned or too small */
+    AXIS_ATTN_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed */
+    AXIS_ATTN_ERR_TIMEOUT = 7      /* a device-side wait ran out (see above) */
+} axis_attn_status;
+
+/*
+ * Forward.  Writes o [B,S,Hq,D] (bf16) and lse [B,Hq,S] (fp32, natural log,
+ * scale included: lse = ln sum_j exp(scale * q.k_j) over visible keys).
+ * causal != 0 applies the mask j <= i (one sequence length for queries and
+ * keys, so the diagonal is included and no row is fully masked).
+ */
+int axis_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                  int B, int Hq, int Hkv, int S, int D, float scale, int causal,
+                  void* stream);
+
+/*
+ * Bytes of device workspace axis_attn_bwd() needs for these sizes (0 if the
+ * sizes are invalid).  It holds, per (b, query head), fp32 rows of
+ * log2-scaled LSE and of Dr = rowsum(dO * O), padded to a multiple of 128,
+ * and an fp32 dQ accumulator [B, Hq, S, D].
+ */
+size_t axis_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int S, int D);
+
+/*
+ * Backward.  Given the forward's inputs q, k, v, its outputs o and lse, and the
+ * incoming gradient dO [B,S,Hq,D], writes dq [B,S,Hq,D], dk and dv
+ * [B,S,Hkv,D] (bf16; fully overwritten, not accumulated into).  dk and dv sum
+ * the contributions of all Hq/Hkv query heads of a kv group.  `workspace` is a
+ * caller-owned device buffer of at least axis_attn_bwd_workspace_bytes() bytes,
+ * 256-byte aligned; its contents on entry do not matter and on return are
+ * unspecified.  Two calls that overlap on the device must not share it.
+ * dq is accumulated in fp32 with atomic adds, so its low-order bits may vary
+ * from run to run; dk and dv do not.
+ */
+int axis_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                  const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                  int B, int Hq, int Hkv, int S, int D, float scale, int causal,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The three stages axis_attn_bwd() runs, in order, on one stream, exposed so a
+ * caller can overlap or time them separately.  Arguments mean what they mean
+ * for axis_attn_bwd() and are validated the same way; the workspace carries the
+ * state from one stage to the next, so all three must get the same workspace
+ * and sizes, in this order, with nothing writing the workspace in between.
+ *   prepare:  Dr = rowsum(dO * O) and LSE * log2(e) into the workspace; zeroes
+ *             the fp32 dQ accumulator.  Reads o, dO, lse.
+ *   main:     dk, dv (written) and the dQ accumulator (added into).  Reads q, k,
+ *             v, dO and the workspace.
+ *   finalize: dq = bf16(dQ accumulator).
+ */
+int axis_attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, int Hkv,
+                          int S, int D, void* workspace, size_t workspace_bytes, void* stream);
+int axis_attn_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk,
+                       void* dv, int B, int Hq, int Hkv, int S, int D, float scale, int causal,
+                       void* workspace, size_t workspace_bytes, void* stream);
+int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, int D, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then returns AXIS_ATTN_ERR_TIMEOUT if any kernel of
+ * this library on the current device has reported a timed-out device wait since
+ * the last call (and clears that report), AXIS_ATTN_ERR_CUDA if the CUDA
+ * context holds an error, else AXIS_ATTN_OK.  For tests and debugging: it
+ * blocks the host.
+ */
+int axis_attn_get_status(void* stream);
+
+/* Static, human-readable text for a status code. */
+const char* axis_attn_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AXIS_ATTN_H */

@@ -309,6 +309,13 @@ int oracle_attn_bwd_dkdv_rows(const double* q, const double* k, const double* v,
         if (f < 0) { units[nu] = u; f = nu++; }
         unit_of[r] = f;
     }
+    /* Under the causal mask only query rows i >= j see key j, so each unit
+     * needs the per-row statistics from its smallest sampled key row on. */
+    int* first = (int*)malloc(sizeof(int) * (size_t)(nu > 0 ? nu : 1));
+    for (int t = 0; t < nu; ++t) first[t] = causal ? S : 0;
+    if (causal)
+        for (int r = 0; r < n; ++r)
+            if (rows[3 * r + 2] < first[unit_of[r]]) first[unit_of[r]] = rows[3 * r + 2];
     double* lse = (double*)malloc(sizeof(double) * (size_t)(nu > 0 ? nu : 1) * G * S);
     double* dr = (double*)malloc(sizeof(double) * (size_t)(nu > 0 ? nu : 1) * G * S);
     const long stat_rows = (long)nu * G * S;
@@ -322,6 +329,7 @@ int oracle_attn_bwd_dkdv_rows(const double* q, const double* k, const double* v,
             const int g = (int)((t / S) % G);
             const int un = (int)(t / ((long)S * G));
             const int b = units[un] / Hkv, kv = units[un] % Hkv, h = kv * G + g;
+            if (i < first[un]) { lse[t] = 0.0; dr[t] = 0.0; continue; }
             double l;
             softmax_row(&z, q, k, b, h, i, p, &l);
             out_row(&z, v, b, kv, p, o_row);
@@ -359,6 +367,7 @@ int oracle_attn_bwd_dkdv_rows(const double* q, const double* k, const double* v,
     }
     free(unit_of);
     free(units);
+    free(first);
     free(lse);
     free(dr);
     return 0;

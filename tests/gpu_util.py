@@ -1,0 +1,54 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI,
+compare with the oracle using the tolerances of the benchmark spec.
+
+Tolerances (fp32 accumulation, bf16 inputs and outputs):
+  O   max |GPU - oracle|                          <= 1e-2
+  LSE max |GPU - oracle|                          <= 1e-4
+  dQ, dK, dV  ||GPU - oracle||_2 / ||oracle||_2    <= 1e-2
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import causal_attention_fwd_b200 as aa
+
+TOL_O = 1e-2
+TOL_LSE = 1e-4
+TOL_GRAD = 1e-2
+
+
+def run_gpu(q, k, v, dout, causal: bool, scale: float, check=True):
+    """fwd + bwd on cuda:0 through the C ABI; returns CPU tensors."""
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, dout))
+    o, lse = aa.attention_forward(qd, kd, vd, causal=causal, scale=scale)
+    dq, dk, dv = aa.attention_backward(qd, kd, vd, o, lse, dod, causal=causal, scale=scale)
+    if check:
+        aa.check_status()
+    torch.cuda.synchronize()
+    return tuple(t.cpu() for t in (o, lse, dq, dk, dv))
+
+
+def f64(t) -> np.ndarray:
+    return t.to(torch.float64).numpy() if isinstance(t, torch.Tensor) else np.asarray(t, np.float64)
+
+
+def rel_l2(got, ref) -> float:
+    got, ref = f64(got), f64(ref)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
+
+
+def max_abs(got, ref) -> float:
+    return float(np.abs(f64(got) - f64(ref)).max()) if np.size(ref) else 0.0
+
+
+def assert_close(o, lse, dq, dk, dv, ro, rlse, rdq, rdk, rdv, tag=""):
+    eo, el = max_abs(o, ro), max_abs(lse, rlse)
+    eq, ek, ev = rel_l2(dq, rdq), rel_l2(dk, rdk), rel_l2(dv, rdv)
+    msg = f"{tag}: O {eo:.2e} LSE {el:.2e} dQ {eq:.2e} dK {ek:.2e} dV {ev:.2e}"
+    assert np.isfinite([eo, el, eq, ek, ev]).all(), msg
+    assert eo <= TOL_O and el <= TOL_LSE, msg
+    assert eq <= TOL_GRAD and ek <= TOL_GRAD and ev <= TOL_GRAD, msg
+    return msg

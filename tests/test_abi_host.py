@@ -1,0 +1,125 @@
+"""Host-side checks of the C ABI (CPU only; nothing here launches a kernel).
+
+The library must load, export every function include/axis_attn.h declares,
+size the backward workspace, and reject every invalid argument with its status
+code before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import causal_attention_fwd_b200 as aa
+from causal_attention_fwd_b200 import build as build_mod
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "axis_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return aa.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(axis_attn_\w+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert _declared() == sorted(aa.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    nm = os.popen(f"nm -D --defined-only {aa.library_path()}").read()
+    for name in _declared():
+        assert re.search(rf"\bT {name}\b", nm), name
+
+
+def test_strerror_covers_every_status(lib):
+    texts = {aa.axis_attn_strerror(c) for c in range(8)}
+    assert len(texts) == 8 and "ok" in texts
+    assert aa.axis_attn_strerror(99) == "unknown status"
+
+
+def test_workspace_bytes(lib):
+    # lse2 + dr rows padded to 128, each section rounded to 256 bytes, + fp32 dQ accumulator
+    B, Hq, Hkv, S, D = 2, 12, 4, 1000, 64
+    rows = B * Hq * 1024
+    r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert aa.axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D) == 2 * r256(rows * 4) + r256(B * Hq * S * D * 4)
+    assert aa.axis_attn_bwd_workspace_bytes(1, 3, 2, 128, 64) == 0      # Hq % Hkv != 0
+    assert aa.axis_attn_bwd_workspace_bytes(1, 1, 1, 128, 96) == 0      # unsupported D
+    assert aa.axis_attn_bwd_workspace_bytes(1, 1, 1, 0, 64) == 0        # empty sequence
+
+
+A = 1 << 20  # a fake, 16-byte aligned "device" address; never dereferenced
+
+
+def _fwd(**over):
+    args = dict(q=A, k=A, v=A, o=A, lse=A, B=1, Hq=2, Hkv=1, S=128, D=64, scale=0.125, causal=1,
+                stream=None)
+    args.update(over)
+    return aa.axis_attn_fwd(*args.values())
+
+
+def _bwd(**over):
+    args = dict(q=A, k=A, v=A, o=A, dO=A, lse=A, dq=A, dk=A, dv=A, B=1, Hq=2, Hkv=1, S=128, D=64,
+                scale=0.125, causal=1, workspace=A, workspace_bytes=1 << 30, stream=None)
+    args.update(over)
+    return aa.axis_attn_bwd(*args.values())
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), 1), (dict(lse=None), 1), (dict(v=0), 1),
+    (dict(k=A + 8), 2), (dict(o=A + 2), 2), (dict(lse=A + 4), 2),
+    (dict(B=0), 3), (dict(S=0), 3), (dict(Hq=3, Hkv=2), 3), (dict(Hkv=0), 3),
+    (dict(scale=0.0), 3), (dict(scale=-1.0), 3), (dict(scale=float("nan")), 3),
+    (dict(scale=float("inf")), 3),
+    (dict(B=1 << 16, S=1 << 16), 3),
+    (dict(D=32), 4), (dict(D=96), 4), (dict(D=256), 4),
+])
+def test_fwd_rejects(lib, over, code):
+    assert _fwd(**over) == code
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(dO=None), 1), (dict(dq=None), 1), (dict(dv=None), 1),
+    (dict(dk=A + 8), 2), (dict(dO=A + 1), 2),
+    (dict(S=0), 3), (dict(Hq=4, Hkv=3), 3), (dict(scale=0.0), 3), (dict(D=80), 4),
+    (dict(workspace=None), 5), (dict(workspace=A + 16), 5), (dict(workspace_bytes=1000), 5),
+])
+def test_bwd_rejects(lib, over, code):
+    assert _bwd(**over) == code
+
+
+def test_torch_helpers_raise_without_valid_args(lib):
+    import torch
+
+    q = torch.zeros(1, 128, 2, 32, dtype=torch.bfloat16)  # CPU tensors, D = 32: rejected
+    with pytest.raises(aa.AxisAttnError) as e:
+        aa.attention_forward(q, q[:, :, :1], q[:, :, :1], stream=type("S", (), {"cuda_stream": 0})())
+    assert e.value.code == 4
+
+
+def test_no_cpu_fallback(tmp_path, monkeypatch):
+    """With the library absent, the first call raises instead of computing on the CPU."""
+    import causal_attention_fwd_b200.binding as bnd
+
+    monkeypatch.setattr(bnd, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(bnd, "_lib", None)
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        bnd.axis_attn_bwd_workspace_bytes(1, 1, 1, 128, 64)
+
+
+def test_valid_args_without_gpu_report_cuda_error(lib):
+    """Valid arguments on a machine with no usable GPU: a status, not a crash."""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _fwd() in (4, 6)
