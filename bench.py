@@ -198,6 +198,32 @@ def run_reference(args, rank: int, world: int):
     return 0
 
 
+# ------------------------------------------------------- multi-rank plumbing
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling: independent problems)."""
+    return base_seed + 100 * rank
+
+
+def reduce_max(values, world: int, device=None):
+    """Element-wise max over ranks of a list of floats (the slowest rank sets
+    the time).  Uses the default process group when world > 1."""
+    import torch
+
+    t = torch.tensor(list(values), dtype=torch.float64)
+    if world > 1:
+        import torch.distributed as dist
+
+        t = t.to(device) if device is not None else t
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t = t.cpu()
+    return [float(x) for x in t]
+
+
+def whole_job_tflops(flops_per_step_per_rank: float, steps: int, max_ms: float, world: int) -> float:
+    """Units all ranks processed divided by the slowest rank's device time."""
+    return world * flops_per_step_per_rank * steps / (max_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -234,7 +260,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     w = WORKLOADS[args.workload]
     B, Hq, Hkv, S, D = w.B, w.Hq, w.Hkv, w.S, w.D
-    q_h, k_h, v_h, do_h = workload_inputs(w, seed=WORKLOAD_SEED[w.name] + 100 * rank)
+    q_h, k_h, v_h, do_h = workload_inputs(w, seed=rank_seed(WORKLOAD_SEED[w.name], rank))
     q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, S), device=dev, dtype=torch.float32)
@@ -294,18 +320,14 @@ def main():
     sampler.stop()
     aa.check_status(stream)
 
-    per = torch.tensor([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs], dtype=torch.float64)
-    totals = per.sum(0)  # ms per stage over all steps
-    step_total = torch.tensor([sum(e[0].elapsed_time(e[4]) for e in evs)], dtype=torch.float64)
-    if world > 1:
-        t = torch.cat([step_total, totals]).to(dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t = t.cpu()
-        step_total, totals = t[:1], t[1:]
-    total_ms = float(step_total[0])
+    per = [[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs]
+    stage_ms = [sum(p[i] for p in per) for i in range(4)]  # ms per stage over all steps
+    step_ms = sum(e[0].elapsed_time(e[4]) for e in evs)
+    reduced = reduce_max([step_ms] + stage_ms, world, dev)
+    total_ms, totals = reduced[0], reduced[1:]
     K = args.steps
     flops_step = w.fwd_flops + w.bwd_flops
-    value = world * flops_step * K / (total_ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops_step, K, total_ms, world)
     names = ["attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_kernel", "attn_bwd_dq_convert_kernel"]
     avg_ms = [float(totals[i]) / K for i in range(4)]
     fwd_tf = w.fwd_flops / (avg_ms[0] * 1e-3) / 1e12
@@ -355,15 +377,11 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64)
-        if world > 1:
-            ems = ems.to(dev)
-            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
-            ems = ems.cpu()
+        ems = reduce_max([e0.elapsed_time(e1)], world, dev)
         aa.check_status(stream)
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
         d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
-        e2e = {"value": world * flops_step * args.e2e_steps / (float(ems[0]) * 1e-3) / 1e12,
+        e2e = {"value": whole_job_tflops(flops_step, args.e2e_steps, ems[0], world),
                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": args.e2e_steps}
 

@@ -56,7 +56,8 @@ def test_fuzz_full_outputs(oracle_mod, B, Hq, Hkv, S, D, causal):
     got = run_gpu(q, k, v, do, causal, sc)
     ro, rl = oracle_mod.attn_fwd(q, k, v, sc, causal)
     rdq, rdk, rdv, _ = oracle_mod.attn_bwd(q, k, v, do, sc, causal)
-    assert_close(*got, ro, rl, rdq, rdk, rdv, tag=f"B{B} Hq{Hq} Hkv{Hkv} S{S} D{D} c{int(causal)}")
+    print(assert_close(*got, ro, rl, rdq, rdk, rdv, tag=f"B{B} Hq{Hq} Hkv{Hkv} S{S} D{D} c{int(causal)}",
+                       S=S))
 
 
 @pytest.mark.parametrize("name", ["tiny", "gpt2s_gqa"])
