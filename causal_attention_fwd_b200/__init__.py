@@ -13,6 +13,7 @@ from .binding import (  # noqa: F401
     axis_attn_bwd,
     axis_attn_bwd_finalize,
     axis_attn_bwd_main,
+    axis_attn_bwd_noalloc,
     axis_attn_bwd_prepare,
     axis_attn_bwd_workspace_bytes,
     axis_attn_fwd,

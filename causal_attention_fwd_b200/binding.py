@@ -25,6 +25,7 @@ EXPORTS = (
     "axis_attn_bwd_prepare",
     "axis_attn_bwd_main",
     "axis_attn_bwd_finalize",
+    "axis_attn_bwd_noalloc",
     "axis_attn_get_status",
     "axis_attn_strerror",
 )
@@ -77,6 +78,8 @@ def load():
             lib.axis_attn_bwd_main.restype = i
             lib.axis_attn_bwd_finalize.argtypes = [vp] + [i] * 5 + [vp, sz, vp]
             lib.axis_attn_bwd_finalize.restype = i
+            lib.axis_attn_bwd_noalloc.argtypes = [vp] * 9 + [i] * 5 + [f, i, vp]
+            lib.axis_attn_bwd_noalloc.restype = i
             lib.axis_attn_get_status.argtypes = [vp]
             lib.axis_attn_get_status.restype = i
             lib.axis_attn_strerror.argtypes = [i]
@@ -112,6 +115,14 @@ def axis_attn_bwd_main(q, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, wor
 
 def axis_attn_bwd_finalize(dq, B, Hq, Hkv, S, D, workspace, workspace_bytes, stream) -> int:
     return load().axis_attn_bwd_finalize(dq, B, Hq, Hkv, S, D, workspace, workspace_bytes, stream)
+
+
+def axis_attn_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
+                          stream) -> int:
+    """Backward with the library's built-in 32 MiB scratch instead of a workspace,
+    for callers that cannot allocate device memory (see include/axis_attn.h)."""
+    return load().axis_attn_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
+                                        stream)
 
 
 def axis_attn_get_status(stream) -> int:

@@ -286,6 +286,53 @@ extern "C" int axis_attn_bwd(const void* q, const void* k, const void* v, const 
   return axis_attn_bwd_finalize(dq, B, Hq, Hkv, S, D, workspace, workspace_bytes, stream);
 }
 
+// ----------------------------------------------------------------------------
+// axis_attn_bwd_noalloc: the backward with library-owned scratch, for callers
+// that may not call cudaMalloc (allocator callbacks, pre-reserved memory pools,
+// paths that must not block on the allocator) and have no workspace to pass.
+// The scratch is a fixed device array; the library never allocates or frees.
+
+// The array's name in host code is only a handle for the runtime; the device
+// address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[AXIS_ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace axis_attn {
+namespace {
+
+void* g_noalloc_addr[64];
+std::mutex g_noalloc_mutex;
+
+int noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return AXIS_ATTN_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return AXIS_ATTN_OK;
+}
+
+}  // namespace
+}  // namespace axis_attn
+
+extern "C" int axis_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                     const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S,
+                                     int D, float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return AXIS_ATTN_ERR_ALIGN;
+  if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
+  if (ws_layout(B, Hq, S, D).total > (size_t)AXIS_ATTN_NOALLOC_SCRATCH_BYTES) return AXIS_ATTN_ERR_WORKSPACE;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  void* scratch = nullptr;
+  if (int rc = noalloc_scratch(dev, &scratch)) return rc;
+  return axis_attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, scratch,
+                       (size_t)AXIS_ATTN_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 extern "C" int axis_attn_get_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return AXIS_ATTN_ERR_CUDA;
   unsigned int st = 0, zero = 0;

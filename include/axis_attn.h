@@ -113,6 +113,37 @@ int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, int D, void*
                            size_t workspace_bytes, void* stream);
 
 /*
+ * Backward for callers that cannot allocate device memory: same arguments,
+ * results and errors as axis_attn_bwd(), minus the workspace.  (No counterpart
+ * on the pages: this is a packaging variant of the backward, not a different
+ * computation.)
+ *
+ * Who needs it: code that runs where cudaMalloc is off limits -- inside a
+ * custom allocator or memory-pool callback, in a process whose device memory
+ * is fully reserved up front by a framework, or in a host path that must never
+ * block on the allocator -- and cannot be handed a workspace by its caller.
+ * Instead of a caller-owned workspace, the scratch lives in a fixed array built
+ * into this library (AXIS_ATTN_NOALLOC_SCRATCH_BYTES = 32 MiB, 256-byte aligned)
+ * that every GPU which loads the library holds until the process exits.
+ *
+ * Limit: the sizes must satisfy
+ *   axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D) <= 32 MiB
+ * (e.g. B=2, Hq=12, S=1024, D=64 fits; B=4, Hq=32, S=2048, D=64 does not);
+ * larger sizes return AXIS_ATTN_ERR_WORKSPACE and launch nothing.
+ * The first call on a device looks up that device's address of the array
+ * (cudaGetSymbolAddress); make that first call before capturing a stream.
+ * The array is shared by every call on a device and keeps the last call's
+ * contents; each call re-initialises what it reads (including zeroing its dQ
+ * accumulator), but two calls that overlap on the GPU (different streams, or
+ * concurrent host threads) race on it and must be serialised by the caller.
+ */
+#define AXIS_ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+int axis_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                          const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                          int B, int Hq, int Hkv, int S, int D, float scale, int causal,
+                          void* stream);
+
+/*
  * Synchronises `stream`, then returns AXIS_ATTN_ERR_TIMEOUT if any kernel of
  * this library on the current device has reported a timed-out device wait since
  * the last call (and clears that report), AXIS_ATTN_ERR_CUDA if the CUDA
