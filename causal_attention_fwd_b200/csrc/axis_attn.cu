@@ -112,7 +112,7 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   static bool done[64];
   if (int rc = set_smem(kern, FwdCfg<HD>::SMEM, dev, done)) return rc;
   const unsigned grid = (unsigned)a.n_qblocks * a.B * a.Hq;
-  kern<<<grid, 512, FwdCfg<HD>::SMEM, st>>>(mq, mk, mv, a);
+  kern<<<grid, FWD_THREADS, FwdCfg<HD>::SMEM, st>>>(mq, mk, mv, a);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 

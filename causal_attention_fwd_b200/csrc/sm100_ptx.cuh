@@ -69,14 +69,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same condition (for event loops that poll several
+// barriers).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Progress watchdog for event loops: call `stalled()` once per idle pass; it
+// returns true (after raising the abort flag and the status word) when no
+// progress was reported through `progress()` for AXIS_ATTN_WAIT_LIMIT_NS, or
+// when another role or CTA gave up.
+struct Watchdog {
+  uint64_t t0;
+  __device__ __forceinline__ Watchdog() : t0(0) {}
+  __device__ __forceinline__ void progress() { t0 = 0; }
+  __device__ __forceinline__ bool stalled(volatile int* abort, int site);
+};
+
 // Wait until the phase of `bar` with parity `parity` has completed.  Gives up
 // when `*abort` becomes non-zero (another role of the CTA gave up) or after
 // AXIS_ATTN_WAIT_LIMIT_NS; in the latter case it raises `*abort` and records
 // the failure in g_status.  Returns true when the phase completed.
 // Called by a single thread, or by all lanes of a warp (see wait_warp).
-__device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                               volatile int* abort, int site) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
+                                            int site) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -92,6 +116,32 @@ __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool Watchdog::stalled(volatile int* abort, int site) {
+  if (*abort) return true;
+  const uint64_t now = global_timer_ns();
+  if (t0 == 0) {
+    t0 = now;
+    return false;
+  }
+  if (*reinterpret_cast<volatile unsigned int*>(&g_status) & 1u) {
+    *abort = 1;
+    return true;
+  }
+  if (now - t0 > AXIS_ATTN_WAIT_LIMIT_NS) {
+    *abort = 1;
+    atomicOr(&g_status, 1u | ((unsigned)(site & 0xff) << 8));
+    return true;
+  }
+  return false;
+}
+
+// Fast path inline (one try_wait); the timed loop only runs on a miss.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                  int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort, site);
 }
 
 // Warp-uniform bounded wait: every lane polls, and the warp proceeds only if
@@ -280,6 +330,36 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
 }
 
 // ------------------------------------------------------------- arithmetic
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed pairs of fp32 (sm_100 executes f32x2 FMA/ADD/MUL as one instruction).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
