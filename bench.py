@@ -297,9 +297,11 @@ def main():
         if ev:
             ev[4].record(stream)
 
-    for _ in range(args.warmup):
+    for n in range(args.warmup):
         flush.fill_(1)
         step()
+        if n == 0:
+            aa.check_status(stream)  # fail fast on a device-side timeout
     aa.check_status(stream)
 
     sampler = ClockSampler(local)

@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     axis_attn_bwd_workspace_bytes,
     axis_attn_fwd,
     axis_attn_get_status,
+    axis_attn_last_status_word,
     axis_attn_strerror,
     check_status,
     library_path,

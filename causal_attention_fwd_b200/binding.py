@@ -27,6 +27,7 @@ EXPORTS = (
     "axis_attn_bwd_finalize",
     "axis_attn_bwd_noalloc",
     "axis_attn_get_status",
+    "axis_attn_last_status_word",
     "axis_attn_strerror",
 )
 
@@ -82,6 +83,8 @@ def load():
             lib.axis_attn_bwd_noalloc.restype = i
             lib.axis_attn_get_status.argtypes = [vp]
             lib.axis_attn_get_status.restype = i
+            lib.axis_attn_last_status_word.argtypes = []
+            lib.axis_attn_last_status_word.restype = ctypes.c_uint
             lib.axis_attn_strerror.argtypes = [i]
             lib.axis_attn_strerror.restype = ctypes.c_char_p
             _lib = lib
@@ -127,6 +130,10 @@ def axis_attn_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, sca
 
 def axis_attn_get_status(stream) -> int:
     return load().axis_attn_get_status(stream)
+
+
+def axis_attn_last_status_word() -> int:
+    return int(load().axis_attn_last_status_word())
 
 
 def axis_attn_strerror(code: int) -> str:
@@ -195,4 +202,5 @@ def check_status(stream=None):
     """Synchronise and raise if a kernel reported a timed-out device wait."""
     rc = axis_attn_get_status(_stream(stream))
     if rc:
-        raise AxisAttnError(rc, "axis_attn_get_status")
+        w = axis_attn_last_status_word()
+        raise AxisAttnError(rc, f"axis_attn_get_status (status word {w:#x}, wait site {(w >> 8) & 0xff})")

@@ -33,9 +33,9 @@ namespace axis_attn {
 struct BwdArgs {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  const float* lse2;  // [B*Hq][S_pad]  LSE * log2(e); +inf on padding rows
-  const float* dr;    // [B*Hq][S_pad]  rowsum(dO * O); 0 on padding rows
-  float* dqacc;       // [B*Hq][S][HD]  fp32, pre-scaled by `scale`
+  const float* nlse2;  // [B*Hq][S_pad]  -LSE * log2(e); -inf on padding rows
+  const float* ndr;    // [B*Hq][S_pad]  -rowsum(dO * O); 0 on padding rows
+  float* dqacc;        // [B*Hq][S][HD]  fp32, pre-scaled by `scale`
   int B, Hq, Hkv, S, S_pad;
   float scale, scale_log2;
 };
@@ -43,46 +43,96 @@ struct BwdArgs {
 template <int HD>
 struct BwdCfg {
   static constexpr int BM = HD == 64 ? 128 : 64;   // query rows per step
-  static constexpr bool QLANE = HD == 64;          // dQ lanes = query rows
+  static constexpr bool QLANE = HD == 64;          // dQ lanes = query rows (else features)
   static constexpr int NSLAB = HD / 64;
   static constexpr uint32_t KSLAB = 128 * 128;     // 128 key rows x 128 bytes
   static constexpr uint32_t KTILE = NSLAB * KSLAB;
   static constexpr uint32_t QSLAB = BM * 128;      // BM query rows x 128 bytes
   static constexpr uint32_t QTILE = NSLAB * QSLAB;
-  static constexpr uint32_t DS_BYTES = (BM / 64) * 128 * 128;  // dS^T: 128 keys x BM
+  static constexpr uint32_t PS_BYTES = (BM / 64) * 128 * 128;  // P^T or dS^T: 128 keys x BM bf16
   static constexpr int ST = 2;
+  static constexpr int HALF = BM / 2;              // query columns per compute warpgroup
+  static constexpr int NCH = HALF / 32;            // 32-column chunks per compute thread
   // shared-memory offsets from the 1024-aligned base
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = KTILE;
   static constexpr uint32_t OFF_Q = 2 * KTILE;
   static constexpr uint32_t OFF_DO = OFF_Q + ST * QTILE;
-  static constexpr uint32_t OFF_DS = OFF_DO + ST * QTILE;
-  static constexpr uint32_t OFF_LSE = OFF_DS + DS_BYTES;
+  static constexpr uint32_t OFF_PT = OFF_DO + ST * QTILE;
+  static constexpr uint32_t OFF_DST = OFF_PT + PS_BYTES;
+  static constexpr uint32_t OFF_LSE = OFF_DST + PS_BYTES;
   static constexpr uint32_t OFF_DR = OFF_LSE + ST * BM * 4;
   static constexpr uint32_t OFF_BAR = OFF_DR + ST * BM * 4;
-  static constexpr int NBAR = 8 + 2 * ST;
+  static constexpr int NBAR = 16;
   static constexpr uint32_t SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
-  // TMEM columns
-  static constexpr uint32_t T_S = 0, T_DP = BM, T_DV = 2 * BM, T_DK = 2 * BM + HD,
-                            T_DQ = 2 * BM + 2 * HD;
+  // TMEM columns: S^T, dP^T, dV, dK, and two dQ tiles
+  static constexpr uint32_t T_S = 0, T_DP = BM, T_DV = 2 * BM, T_DK = 2 * BM + HD, T_DQ = 2 * BM + 2 * HD;
+  static constexpr uint32_t DQ_COLS = 64;
+  static_assert(T_DQ + 2 * DQ_COLS <= 512, "TMEM budget");
 };
 
-enum BwdSite { B_KV = 21, B_QEMPTY, B_QFULL, B_MMADONE, B_DSREADY, B_DQFREE, B_SPFULL, B_DQFULL, B_FIN };
+// Warps 0-7: P^T / dS^T (thread = key row, half the query columns each) and
+// the dQ readout of the previous step; warp 8 loads; warp 9 issues the MMAs
+// and owns TMEM; warps 10-11 spare.  384 threads: up to 168 registers each.
+constexpr int BWD_THREADS = 384;
+constexpr int BWD_WARP_LOAD = 8;
+constexpr int BWD_WARP_MMA = 9;
+
+enum BwdSite { B_KV = 21, B_QEMPTY, B_QFULL, B_SPFREE, B_PDSFULL, B_DQFREE, B_SPFULL, B_DQFULL, B_FIN, B_PDSFREE };
+
+// Swizzled store of 8 bf16 pairs (16 query columns) of one key row into a
+// [key][query] 128B-swizzled buffer of 64-column slabs.
+__device__ __forceinline__ void store_row16(uint32_t buf, int kr, int col0, const uint32_t* v) {
+  const int slab = col0 >> 6, chunk = (col0 & 63) >> 3;
+  const uint32_t rowaddr = buf + slab * (128 * 128) + (kr >> 3) * 1024 + (kr & 7) * 128;
+  const uint32_t a0 = rowaddr + ((chunk ^ (kr & 7)) << 4);
+  const uint32_t a1 = rowaddr + (((chunk + 1) ^ (kr & 7)) << 4);
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a0), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+               : "memory");
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a1), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
+// One compute thread's share of a dQ tile (32 TMEM columns of its lane) into
+// the fp32 accumulator.  D = 64: lane = query row, columns = features
+// [32 ch, 32 ch + 32).  D = 128: lane = feature, columns = query rows
+// q0 + [32 ch, 32 ch + 32).
+template <int HD, bool QLANE>
+__device__ __forceinline__ void dq_to_global(const uint32_t (&v)[32], float* acc, int q0, int lr, int ch, int S,
+                                             float sc) {
+  if (QLANE) {
+    const int q = q0 + lr;
+    if (q < S) {
+      float4* dst = reinterpret_cast<float4*>(acc + (size_t)q * HD) + 8 * ch;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        atomicAdd(dst + i, make_float4(__uint_as_float(v[4 * i]) * sc, __uint_as_float(v[4 * i + 1]) * sc,
+                                       __uint_as_float(v[4 * i + 2]) * sc, __uint_as_float(v[4 * i + 3]) * sc));
+    }
+  } else {
+    float* col = acc + lr;
+    const int qh = q0 + 32 * ch;
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (qh + e < S) atomicAdd(col + (size_t)(qh + e) * HD, __uint_as_float(v[e]) * sc);
+  }
+}
 
 template <int HD, bool CAUSAL>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(BWD_THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdArgs a) {
   using C = BwdCfg<HD>;
-  constexpr int BM = C::BM, ST = C::ST;
+  constexpr int BM = C::BM, ST = C::ST, HALF = C::HALF, NCH = C::NCH;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
 
-  const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sDS = base + C::OFF_DS;
+  const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
+  const uint32_t sPT = base + C::OFF_PT, sDST = base + C::OFF_DST;
   auto sQ = [&](int s) { return base + C::OFF_Q + s * C::QTILE; };
   auto sDO = [&](int s) { return base + C::OFF_DO + s * C::QTILE; };
   const float* lse_s = reinterpret_cast<const float*>(gbase + C::OFF_LSE);
@@ -90,13 +140,15 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t bars = base + C::OFF_BAR;
   const uint32_t bar_kv = bars;
   auto bar_qfull = [&](int s) { return bars + 8u * (1 + s); };
-  auto bar_qempty = [&](int s) { return bars + 8u * (1 + ST + s); };
-  const uint32_t bar_sp = bars + 8u * (1 + 2 * ST);
-  const uint32_t bar_ds = bars + 8u * (2 + 2 * ST);
-  const uint32_t bar_dqfull = bars + 8u * (3 + 2 * ST);
-  const uint32_t bar_dqfree = bars + 8u * (4 + 2 * ST);
-  const uint32_t bar_done = bars + 8u * (5 + 2 * ST);
-  const uint32_t bar_fin = bars + 8u * (6 + 2 * ST);
+  auto bar_qempty = [&](int s) { return bars + 8u * (3 + s); };
+  const uint32_t bar_spfull = bars + 8u * 5;   // S^T, dP^T of a step are in TMEM
+  const uint32_t bar_spfree = bars + 8u * 6;   // ... and have been read (8 warps)
+  const uint32_t bar_pdsfull = bars + 8u * 7;  // P^T, dS^T of a step are in smem (8 warps)
+  const uint32_t bar_ptfree = bars + 8u * 8;   // dV of a step is done with P^T
+  auto bar_dqfull = [&](int b) { return bars + 8u * (9 + b); };
+  auto bar_dqfree = [&](int b) { return bars + 8u * (11 + b); };
+  const uint32_t bar_fin = bars + 8u * 13;
+  const uint32_t bar_dstfree = bars + 8u * 14;  // dK, dQ of a step are done with dS^T
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 8 * C::NBAR);
   volatile int* abort = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + 8 * C::NBAR + 4);
 
@@ -118,17 +170,19 @@ __global__ void __launch_bounds__(512, 1)
     for (int s = 0; s < ST; ++s) {
       mbar_init(bar_qfull(s), 1);
       mbar_init(bar_qempty(s), 1);
+      mbar_init(bar_dqfull(s), 1);
+      mbar_init(bar_dqfree(s), 8);
     }
-    mbar_init(bar_sp, 1);
-    mbar_init(bar_ds, 8);
-    mbar_init(bar_dqfull, 1);
-    mbar_init(bar_dqfree, 4);
-    mbar_init(bar_done, 1);
+    mbar_init(bar_spfull, 1);
+    mbar_init(bar_spfree, 8);
+    mbar_init(bar_pdsfull, 8);
+    mbar_init(bar_ptfree, 1);
+    mbar_init(bar_dstfree, 1);
     mbar_init(bar_fin, 1);
     *abort = 0;
     fence_barrier_init();
   }
-  if (warp == 13) {
+  if (warp == BWD_WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -137,9 +191,9 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 12) {
-    // ===================================================== loads
+  if (warp == BWD_WARP_LOAD) {
     if (lane == 0) {
+      // ===================================================== loads
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -161,8 +215,8 @@ __global__ void __launch_bounds__(512, 1)
           tma_load_4d(sQ(s) + sl * C::QSLAB, &tm_q, bar_qfull(s), 64 * sl, h, q0, b);
           tma_load_4d(sDO(s) + sl * C::QSLAB, &tm_do, bar_qfull(s), 64 * sl, h, q0, b);
         }
-        bulk_load(base + C::OFF_LSE + s * BM * 4, a.lse2 + row, BM * 4, bar_qfull(s));
-        bulk_load(base + C::OFF_DR + s * BM * 4, a.dr + row, BM * 4, bar_qfull(s));
+        bulk_load(base + C::OFF_LSE + s * BM * 4, a.nlse2 + row, BM * 4, bar_qfull(s));
+        bulk_load(base + C::OFF_DR + s * BM * 4, a.ndr + row, BM * 4, bar_qfull(s));
         issued = it + 1;
       }
       volatile int never = 0;
@@ -170,59 +224,75 @@ __global__ void __launch_bounds__(512, 1)
       for (int it = issued - ST > 0 ? issued - ST : 0; it < issued; ++it)
         mbar_wait_bounded(bar_qfull(it % ST), (it / ST) & 1, &never, B_QFULL);
     }
-  } else if (warp == 13) {
-    // ===================================================== MMA issuer
+  } else if (warp == BWD_WARP_MMA) {
     if (lane == 0) {
+      // ===================================================== MMA issuer
       constexpr uint32_t ID_S = idesc_bf16(128, BM, 0, 0);   // K|V (K-major) x Q|dO (K-major)
-      constexpr uint32_t ID_GV = idesc_bf16(128, HD, 0, 1);  // P^T|dS^T x dO|Q (MN-major)
+      constexpr uint32_t ID_GV = idesc_bf16(128, HD, 0, 1);  // P^T|dS^T (K-major) x dO|Q (MN-major)
       constexpr uint32_t ID_Q = C::QLANE ? idesc_bf16(128, HD, 1, 1) : idesc_bf16(128, BM, 1, 1);
-      bool ok = mbar_wait_bounded(bar_kv, 0, abort, B_KV);
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it % ST;
-        if (!mbar_wait_bounded(bar_qfull(s), (it / ST) & 1, abort, B_QFULL)) break;
-        if (it > 0 && !mbar_wait_bounded(bar_done, (it - 1) & 1, abort, B_MMADONE)) break;
-        tc_fence_after();
-        // S^T = K Q^T, dP^T = V dO^T  (reduction over the feature dim)
+      auto issue_sdp = [&](int s) {
+        // S^T = K Q^T and dP^T = V dO^T (reduction over the features)
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KSLAB + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::QSLAB + (kk & 3) * 32;
-          mma_ss(tmem + C::T_S, sw128_desc(sK + ko, 16, 1024), sw128_desc(sQ(s) + qo, 16, 1024), ID_S,
+          mma_ss(tmem + C::T_S, sw128_desc(sK + ko, 16, 1024), sw128_desc(sQ(s) + qo, 16, 1024), ID_S, kk > 0);
+        }
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * C::KSLAB + (kk & 3) * 32;
+          const uint32_t qo = (kk >> 2) * C::QSLAB + (kk & 3) * 32;
+          mma_ss(tmem + C::T_DP, sw128_desc(sV + ko, 16, 1024), sw128_desc(sDO(s) + qo, 16, 1024), ID_S,
                  kk > 0);
         }
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * C::KSLAB + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * C::QSLAB + (kk & 3) * 32;
-          mma_ss(tmem + C::T_DP, sw128_desc(sV + ko, 16, 1024), sw128_desc(sDO(s) + qo, 16, 1024),
-                 ID_S, kk > 0);
-        }
-        mma_commit(bar_sp);
-        if (!mbar_wait_bounded(bar_ds, it & 1, abort, B_DSREADY)) break;
+      };
+      bool ok = mbar_wait_bounded(bar_kv, 0, abort, B_KV) && n_it > 0 &&
+                mbar_wait_bounded(bar_qfull(0), 0, abort, B_QFULL);
+      if (ok) {
         tc_fence_after();
-        // dV += P^T dO, dK += dS^T Q  (reduction over the BM query rows)
+        issue_sdp(0);
+        mma_commit(bar_spfull);
+      }
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it % ST;
+        // next step's S^T, dP^T as soon as this step's are out of TMEM
+        if (it + 1 < n_it) {
+          if (!mbar_wait_bounded(bar_qfull((it + 1) % ST), ((it + 1) / ST) & 1, abort, B_QFULL) ||
+              !mbar_wait_bounded(bar_spfree, it & 1, abort, B_SPFREE))
+            break;
+          tc_fence_after();
+          issue_sdp((it + 1) % ST);
+          mma_commit(bar_spfull);
+        }
+        if (!mbar_wait_bounded(bar_pdsfull, it & 1, abort, B_PDSFULL)) break;
+        tc_fence_after();
+        // dV += P^T dO (reduction over the BM query rows)
         for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t pcol = kk < BM / 32 ? 8 * kk : BM / 2 + 8 * (kk - BM / 32);
-          mma_ts(tmem + C::T_DV, tmem + C::T_S + pcol, sw128_desc(sDO(s) + kk * 2048, C::QSLAB, 1024),
+          const uint32_t po = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + C::T_DV, sw128_desc(sPT + po, 16, 1024), sw128_desc(sDO(s) + kk * 2048, C::QSLAB, 1024),
                  ID_GV, (it > 0 || kk > 0) ? 1u : 0u);
         }
+        mma_commit(bar_ptfree);
+        // dK += dS^T Q
         for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t dso = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss(tmem + C::T_DK, sw128_desc(sDS + dso, 16, 1024),
-                 sw128_desc(sQ(s) + kk * 2048, C::QSLAB, 1024), ID_GV, (it > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t po = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + C::T_DK, sw128_desc(sDST + po, 16, 1024), sw128_desc(sQ(s) + kk * 2048, C::QSLAB, 1024),
+                 ID_GV, (it > 0 || kk > 0) ? 1u : 0u);
         }
-        // dQ tile (reduction over the 128 keys)
-        if (it > 0 && !mbar_wait_bounded(bar_dqfree, (it - 1) & 1, abort, B_DQFREE)) break;
+        // dQ tile (reduction over the 128 keys) into TMEM buffer it % 2
+        const int qb = it & 1;
+        if (it >= 2 && !mbar_wait_bounded(bar_dqfree(qb), ((it >> 1) - 1) & 1, abort, B_DQFREE)) break;
         tc_fence_after();
+        const uint32_t tdq = tmem + C::T_DQ + qb * C::DQ_COLS;
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ds_mn = sw128_desc(sDS + kk * 2048, 128 * 128, 1024);
+          const uint64_t ds_mn = sw128_desc(sDST + kk * 2048, 128 * 128, 1024);
           const uint64_t k_mn = sw128_desc(sK + kk * 2048, C::KSLAB, 1024);
           if (C::QLANE)
-            mma_ss(tmem + C::T_DQ, ds_mn, k_mn, ID_Q, kk > 0);   // dQ = dS K
+            mma_ss(tdq, ds_mn, k_mn, ID_Q, kk > 0);   // dQ = dS K
           else
-            mma_ss(tmem + C::T_DQ, k_mn, ds_mn, ID_Q, kk > 0);   // dQ^T = K^T dS^T
+            mma_ss(tdq, k_mn, ds_mn, ID_Q, kk > 0);   // dQ^T = K^T dS^T
         }
-        mma_commit(bar_dqfull);
+        mma_commit(bar_dqfull(qb));
         mma_commit(bar_qempty(s));
-        mma_commit(bar_done);
+        mma_commit(bar_dstfree);
       }
       mma_commit(bar_fin);
       volatile int never = 0;
@@ -234,69 +304,108 @@ __global__ void __launch_bounds__(512, 1)
     const int kr = wq * 32 + lane;
     const int key = 128 * j + kr;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const int c0 = ch * (BM / 2);
-    const float c = a.scale_log2;
+    const int c0 = ch * HALF;
+    const uint64_t cc2 = f2_pack(a.scale_log2, a.scale_log2);
+    const float sc = a.scale;
     bool ok = true;
+    // dQ tile of step `t` (previous step) from TMEM to the fp32 accumulator
+    auto dq_readout = [&](int t) -> bool {
+      const int qb = t & 1;
+      if (!wait_warp(bar_dqfull(qb), (t >> 1) & 1, abort, B_DQFULL)) return false;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + C::T_DQ + qb * C::DQ_COLS + 32 * ch, v);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_dqfree(qb));
+      const int h = kvh * G + t / per_head;
+      const int q0 = (i0 + t % per_head) * BM;
+      dq_to_global<HD, C::QLANE>(v, a.dqacc + ((size_t)b * a.Hq + h) * (size_t)a.S * HD, q0, kr, ch, a.S, sc);
+      return true;
+    };
     for (int it = 0; it < n_it; ++it) {
       const int s = it % ST;
-      // the staged LSE2 / Dr rows of this step (TMA-written) and S^T, dP^T in TMEM
+      // the staged -LSE2 / -Dr rows of this step (TMA-written) and S^T, dP^T in TMEM
       if (!wait_warp(bar_qfull(s), (it / ST) & 1, abort, B_QFULL) ||
-          !wait_warp(bar_sp, it & 1, abort, B_SPFULL)) {
+          !wait_warp(bar_spfull, it & 1, abort, B_SPFULL)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const int q0 = (i0 + it % per_head) * BM;
       const bool need_mask = (CAUSAL && q0 < 128 * j + 127) || (128 * j + 128 > a.S);
-      const float* lse_t = lse_s + s * BM;
-      const float* dr_t = dr_s + s * BM;
-#pragma unroll 1
-      for (int cc = 0; cc < BM / 32; ++cc) {
-        const int col0 = c0 + 16 * cc;
-        uint32_t sv[16], dpv[16];
-        tmem_ld16(tmem + lane_off + C::T_S + col0, sv);
-        tmem_ld16(tmem + lane_off + C::T_DP + col0, dpv);
-        tmem_wait_ld();
-        uint32_t pk[8], dk[8];
+      const float* lse_t = lse_s + s * BM + c0;
+      const float* dr_t = dr_s + s * BM + c0;
+      uint32_t dk[NCH][16];
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse_t + col0 + (e & ~3));
-          const float4 d4 = *reinterpret_cast<const float4*>(dr_t + col0 + (e & ~3));
-          const float la = (e & 3) ? l4.z : l4.x, lb = (e & 3) ? l4.w : l4.y;
-          const float da = (e & 3) ? d4.z : d4.x, db = (e & 3) ? d4.w : d4.y;
-          float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), c, -la));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), c, -lb));
-          if (need_mask) {
-            const int q = q0 + col0 + e;
-            if ((CAUSAL && key > q) || key >= a.S) p0 = 0.f;
-            if ((CAUSAL && key > q + 1) || key >= a.S) p1 = 0.f;
-          }
-          const float ds0 = p0 * (__uint_as_float(dpv[e]) - da);
-          const float ds1 = p1 * (__uint_as_float(dpv[e + 1]) - db);
-          pk[e / 2] = pack_bf16x2(p0, p1);
-          dk[e / 2] = pack_bf16x2(ds0, ds1);
+      for (int cc = 0; cc < NCH; ++cc) {
+        uint32_t sv[32], dpv[32];
+        tmem_ld32(tmem + lane_off + C::T_S + c0 + 32 * cc, sv);
+        tmem_ld32(tmem + lane_off + C::T_DP + c0 + 32 * cc, dpv);
+        tmem_wait_ld();
+        if (cc == NCH - 1) {
+          // all of this thread's S^T, dP^T are in registers: TMEM may take the next step's
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_spfree);
         }
-        // P^T (bf16) into TMEM over already-consumed S^T columns of this warp's range
-        tmem_st8(tmem + lane_off + C::T_S + c0 + 8 * cc, pk);
-        // dS^T (bf16) into the 128B-swizzled [key][query] slabs
-        const int slab = col0 >> 6, chunk = (col0 & 63) >> 3;
-        const uint32_t rowaddr = sDS + slab * (128 * 128) + (kr >> 3) * 1024 + (kr & 7) * 128;
-        const uint32_t a0 = rowaddr + (((chunk) ^ (kr & 7)) << 4);
-        const uint32_t a1 = rowaddr + (((chunk + 1) ^ (kr & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a0), "r"(dk[0]), "r"(dk[1]),
-                     "r"(dk[2]), "r"(dk[3])
-                     : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a1), "r"(dk[4]), "r"(dk[5]),
-                     "r"(dk[6]), "r"(dk[7])
-                     : "memory");
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_t + 32 * cc + e);
+          const float4 d4 = *reinterpret_cast<const float4*>(dr_t + 32 * cc + e);
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int ee = e + 2 * h2;
+            const uint64_t nl = h2 ? f2_pack(l4.z, l4.w) : f2_pack(l4.x, l4.y);
+            const uint64_t nd = h2 ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y);
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[ee]), __uint_as_float(sv[ee + 1])), cc2, nl), x0, x1);
+            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            if (need_mask) {
+              const int q = q0 + c0 + 32 * cc + ee;
+              if ((CAUSAL && key > q) || key >= a.S) p0 = 0.f;
+              if ((CAUSAL && key > q + 1) || key >= a.S) p1 = 0.f;
+            }
+            const uint64_t pp = f2_pack(p0, p1);
+            float d0, d1;
+            f2_unpack(f2_mul(pp, f2_add(f2_pack(__uint_as_float(dpv[ee]), __uint_as_float(dpv[ee + 1])), nd)), d0,
+                      d1);
+            pk[ee / 2] = pack_bf16x2(p0, p1);
+            dk[cc][ee / 2] = pack_bf16x2(d0, d1);
+          }
+        }
+        // the previous step's dV must be done with P^T before it is overwritten
+        if (cc == 0 && it > 0 && !wait_warp(bar_ptfree, (it - 1) & 1, abort, B_PDSFREE)) {
+          ok = false;
+          break;
+        }
+        store_row16(sPT, kr, c0 + 32 * cc, &pk[0]);
+        store_row16(sPT, kr, c0 + 32 * cc + 16, &pk[8]);
       }
-      tmem_wait_st();
+      if (!ok) break;
+      // ... and the previous step's dK, dQ with dS^T
+      if (it > 0 && !wait_warp(bar_dstfree, (it - 1) & 1, abort, B_PDSFREE)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int cc = 0; cc < NCH; ++cc) {
+        store_row16(sDST, kr, c0 + 32 * cc, &dk[cc][0]);
+        store_row16(sDST, kr, c0 + 32 * cc + 16, &dk[cc][8]);
+      }
       fence_proxy_async_smem();
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_ds);
+      if (lane == 0) mbar_arrive(bar_pdsfull);
+      // the previous step's dQ tile is ready by now (its MMA was issued before this step's P^T, dS^T)
+      if (it > 0 && !dq_readout(it - 1)) {
+        ok = false;
+        break;
+      }
     }
-    // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK (x scale)
+    if (ok && n_it > 0) ok = dq_readout(n_it - 1);
+    // epilogue: warps 0-3 write dV, warps 4-7 write dK (x scale)
     if (ok && wait_warp(bar_fin, 0, abort, B_FIN)) {
       tc_fence_after();
       const uint32_t tcol = ch == 0 ? C::T_DV : C::T_DK;
@@ -307,82 +416,40 @@ __global__ void __launch_bounds__(512, 1)
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + tcol + cc * 32, v);
         tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t pk2[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+          pk2[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
         if (key < a.S) {
           uint4* dst = reinterpret_cast<uint4*>(dst_row + cc * 32);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk2[4 * i], pk2[4 * i + 1], pk2[4 * i + 2], pk2[4 * i + 3]);
         }
-      }
-    }
-  } else if (warp < 12) {
-    // ===================================================== dQ tile -> fp32 accumulator
-    const int wq = warp & 3;
-    const int lr = wq * 32 + lane;   // TMEM lane: query row (D=64) or feature (D=128)
-    const uint32_t tq = tmem + ((uint32_t)(wq * 32) << 16) + C::T_DQ;
-    for (int it = 0; it < n_it; ++it) {
-      if (!wait_warp(bar_dqfull, it & 1, abort, B_DQFULL)) break;
-      tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld32(tq, v0);
-      tmem_ld32(tq + 32, v1);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_dqfree);
-      const int h = kvh * G + it / per_head;
-      const int q0 = (i0 + it % per_head) * BM;
-      float* acc = a.dqacc + ((size_t)b * a.Hq + h) * (size_t)a.S * HD;
-      const float sc = a.scale;
-      if (C::QLANE) {
-        const int q = q0 + lr;
-        if (q < a.S) {
-          float4* dst = reinterpret_cast<float4*>(acc + (size_t)q * HD);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            atomicAdd(dst + i, make_float4(__uint_as_float(v0[4 * i]) * sc, __uint_as_float(v0[4 * i + 1]) * sc,
-                                           __uint_as_float(v0[4 * i + 2]) * sc, __uint_as_float(v0[4 * i + 3]) * sc));
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            atomicAdd(dst + 8 + i, make_float4(__uint_as_float(v1[4 * i]) * sc, __uint_as_float(v1[4 * i + 1]) * sc,
-                                               __uint_as_float(v1[4 * i + 2]) * sc, __uint_as_float(v1[4 * i + 3]) * sc));
-        }
-      } else {
-        // lane = feature d; columns = the BM query rows of the tile
-        float* col = acc + lr;
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (q0 + e < a.S) atomicAdd(col + (size_t)(q0 + e) * HD, __uint_as_float(v0[e]) * sc);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (q0 + 32 + e < a.S) atomicAdd(col + (size_t)(q0 + 32 + e) * HD, __uint_as_float(v1[e]) * sc);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == BWD_WARP_MMA) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
-// Dr = rowsum(dO * O) (fp32), LSE2 = LSE * log2(e); rows S..S_pad-1 get
-// Dr = 0 and LSE2 = +inf.  Also zeroes the dQ accumulator.  One thread per row.
+// -Dr = -rowsum(dO * O) (fp32) and -LSE2 = -LSE * log2(e); rows S..S_pad-1
+// get 0 and -inf (so their P is exactly 0).  Also zeroes the dQ accumulator.
+// One thread per row.
 template <int HD>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                             const __nv_bfloat16* __restrict__ dout,
-                                                            const float* __restrict__ lse, float* lse2,
-                                                            float* dr, float4* dqacc, size_t dq_vec4,
+                                                            const float* __restrict__ lse, float* nlse2,
+                                                            float* ndr, float4* dqacc, size_t dq_vec4,
                                                             int Hq, int S, int S_pad, int rows) {
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r < rows) {
     const int bh = r / S_pad, i = r % S_pad;
-    float d = 0.f, l2 = INFINITY;
+    float d = 0.f, l2 = -INFINITY;
     if (i < S) {
       const int b = bh / Hq, h = bh % Hq;
       const size_t off = (((size_t)b * S + i) * Hq + h) * HD;
@@ -400,10 +467,11 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
           d = fmaf(xf.y, yf.y, d);
         }
       }
-      l2 = lse[(size_t)bh * S + i] * 1.4426950408889634f;
+      l2 = -lse[(size_t)bh * S + i] * 1.4426950408889634f;
+      d = -d;
     }
-    dr[r] = d;
-    lse2[r] = l2;
+    ndr[r] = d;
+    nlse2[r] = l2;
   }
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < dq_vec4; k += stride)

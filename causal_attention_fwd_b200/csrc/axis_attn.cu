@@ -123,7 +123,7 @@ int launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
   static bool done[64];
   if (int rc = set_smem(kern, BwdCfg<HD>::SMEM, dev, done)) return rc;
   const unsigned grid = (unsigned)((a.S + 127) / 128) * a.B * a.Hkv;
-  kern<<<grid, 512, BwdCfg<HD>::SMEM, st>>>(mq, mk, mv, mdo, a);
+  kern<<<grid, BWD_THREADS, BwdCfg<HD>::SMEM, st>>>(mq, mk, mv, mdo, a);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
@@ -229,8 +229,8 @@ extern "C" int axis_attn_bwd_main(const void* q, const void* k, const void* v, c
   BwdArgs a;
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
-  a.lse2 = p.lse2;
-  a.dr = p.dr;
+  a.nlse2 = p.lse2;
+  a.ndr = p.dr;
   a.dqacc = p.dqacc;
   a.B = B;
   a.Hq = Hq;
@@ -333,10 +333,15 @@ extern "C" int axis_attn_bwd_noalloc(const void* q, const void* k, const void* v
                        (size_t)AXIS_ATTN_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+static unsigned int g_last_status_word;
+
+extern "C" unsigned int axis_attn_last_status_word(void) { return g_last_status_word; }
+
 extern "C" int axis_attn_get_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return AXIS_ATTN_ERR_CUDA;
   unsigned int st = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&st, g_status, sizeof(st)) != cudaSuccess) return AXIS_ATTN_ERR_CUDA;
+  g_last_status_word = st;
   if (st != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return AXIS_ATTN_ERR_CUDA;
   if (st != 0) return AXIS_ATTN_ERR_TIMEOUT;
   return cudaGetLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;

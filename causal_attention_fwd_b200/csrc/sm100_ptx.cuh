@@ -99,8 +99,8 @@ struct Watchdog {
 // AXIS_ATTN_WAIT_LIMIT_NS; in the latter case it raises `*abort` and records
 // the failure in g_status.  Returns true when the phase completed.
 // Called by a single thread, or by all lanes of a warp (see wait_warp).
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort,
-                                            int site) {
+__device__ __forceinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               int site) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -137,19 +137,26 @@ __device__ __forceinline__ bool Watchdog::stalled(volatile int* abort, int site)
   return false;
 }
 
-// Fast path inline (one try_wait); the timed loop only runs on a miss.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort, int site) {
+  return mbar_wait_loop(bar, parity, abort, site);
+}
+
+// Fast path inline (one try_wait); the timed loop only runs on a miss.  INL
+// inlines the loop too: code under setmaxnreg must not make calls.
+template <bool INL = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
                                                   int site) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort, site);
+  return INL ? mbar_wait_loop(bar, parity, abort, site) : mbar_wait_slow(bar, parity, abort, site);
 }
 
 // Warp-uniform bounded wait: every lane polls, and the warp proceeds only if
 // all lanes saw the phase complete, so warp-collective instructions that
 // follow are never reached by a partial warp.
+template <bool INL = false>
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort,
                                           int site) {
-  const bool ok = mbar_wait_bounded(bar, parity, abort, site);
+  const bool ok = mbar_wait_bounded<INL>(bar, parity, abort, site);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -327,6 +334,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
          | ((uint32_t)b_mn << 16)        // B major
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// Per-warpgroup register reconfiguration.  Every warp of a warpgroup executes
+// the same one.  The kernel must be launched with a per-thread count from which
+// the sum over warpgroups of (128 threads x new count) fits.
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ------------------------------------------------------------- arithmetic

@@ -152,6 +152,14 @@ int axis_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
  */
 int axis_attn_get_status(void* stream);
 
+/*
+ * Diagnostics: the raw device status word that the last axis_attn_get_status()
+ * call read before clearing it (0 if none was set).  Bit 0: a wait timed out;
+ * bits 8..15: the wait site that first did (1..9: forward kernel, 21..30:
+ * backward main kernel).
+ */
+unsigned int axis_attn_last_status_word(void);
+
 /* Static, human-readable text for a status code. */
 const char* axis_attn_strerror(int code);
 
