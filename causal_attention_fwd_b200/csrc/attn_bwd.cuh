@@ -49,36 +49,46 @@ struct BwdCfg {
   static constexpr uint32_t KTILE = NSLAB * KSLAB;
   static constexpr uint32_t QSLAB = BM * 128;      // BM query rows x 128 bytes
   static constexpr uint32_t QTILE = NSLAB * QSLAB;
-  static constexpr uint32_t PS_BYTES = (BM / 64) * 128 * 128;  // P^T or dS^T: 128 keys x BM bf16
-  static constexpr int ST = 2;
+  static constexpr uint32_t PS_BYTES = (BM / 64) * 128 * 128;  // dS^T: 128 keys x BM bf16
+  static constexpr int ST = 3;                     // Q / dO / LSE / Dr ring depth
   static constexpr int HALF = BM / 2;              // query columns per compute warpgroup
   static constexpr int NCH = HALF / 32;            // 32-column chunks per compute thread
+  // dQ tile staged for the TMA reduce-add: fp32, four 128B-swizzled boxes of
+  // 32 columns x 64 rows (D = 64: rows = queries, columns = features; D = 128:
+  // the tile is 64 queries x 128 features, one box per 32 features)
+  static constexpr uint32_t DQ_BOX = 64 * 128;
+  static constexpr uint32_t STAGE_BYTES = 4 * DQ_BOX;
   // shared-memory offsets from the 1024-aligned base
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = KTILE;
   static constexpr uint32_t OFF_Q = 2 * KTILE;
   static constexpr uint32_t OFF_DO = OFF_Q + ST * QTILE;
-  static constexpr uint32_t OFF_PT = OFF_DO + ST * QTILE;
-  static constexpr uint32_t OFF_DST = OFF_PT + PS_BYTES;
-  static constexpr uint32_t OFF_LSE = OFF_DST + PS_BYTES;
+  static constexpr uint32_t OFF_DST = OFF_DO + ST * QTILE;
+  static constexpr uint32_t OFF_STG = OFF_DST + PS_BYTES;
+  static constexpr uint32_t OFF_LSE = OFF_STG + STAGE_BYTES;
   static constexpr uint32_t OFF_DR = OFF_LSE + ST * BM * 4;
   static constexpr uint32_t OFF_BAR = OFF_DR + ST * BM * 4;
-  static constexpr int NBAR = 16;
+  static constexpr int NBAR = 20;
   static constexpr uint32_t SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
-  // TMEM columns: S^T, dP^T, dV, dK, and two dQ tiles
-  static constexpr uint32_t T_S = 0, T_DP = BM, T_DV = 2 * BM, T_DK = 2 * BM + HD, T_DQ = 2 * BM + 2 * HD;
-  static constexpr uint32_t DQ_COLS = 64;
-  static_assert(T_DQ + 2 * DQ_COLS <= 512, "TMEM budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
+  // TMEM columns: S^T, dP^T, dV, dK, dQ tile, P^T (bf16 pairs)
+  static constexpr uint32_t T_S = 0, T_DP = BM, T_DV = 2 * BM, T_DK = 2 * BM + HD, T_DQ = 2 * BM + 2 * HD,
+                            T_P = T_DQ + 64;
+  static_assert(T_P + BM / 2 <= 512, "TMEM budget");
 };
 
 // Warps 0-7: P^T / dS^T (thread = key row, half the query columns each) and
-// the dQ readout of the previous step; warp 8 loads; warp 9 issues the MMAs
-// and owns TMEM; warps 10-11 spare.  384 threads: up to 168 registers each.
+// the dQ tile of the previous step into the staging tile; warp 8 loads; warp 9
+// issues the MMAs and owns TMEM; warp 10 issues the TMA reduce-adds of the dQ
+// tiles into the fp32 accumulator; warp 11 spare.  384 threads: up to 168
+// registers each.
 constexpr int BWD_THREADS = 384;
 constexpr int BWD_WARP_LOAD = 8;
 constexpr int BWD_WARP_MMA = 9;
+constexpr int BWD_WARP_RED = 10;
 
-enum BwdSite { B_KV = 21, B_QEMPTY, B_QFULL, B_SPFREE, B_PDSFULL, B_DQFREE, B_SPFULL, B_DQFULL, B_FIN, B_PDSFREE };
+enum BwdSite { B_KV = 21, B_QEMPTY, B_QFULL, B_SPFREE, B_PDSFULL, B_DQFREE, B_SPFULL, B_DQFULL, B_FIN, B_PDSFREE,
+               B_STGFULL, B_STGFREE };
 
 // Swizzled store of 8 bf16 pairs (16 query columns) of one key row into a
 // [key][query] 128B-swizzled buffer of 64-column slabs.
@@ -93,36 +103,11 @@ __device__ __forceinline__ void store_row16(uint32_t buf, int kr, int col0, cons
                : "memory");
 }
 
-// One compute thread's share of a dQ tile (32 TMEM columns of its lane) into
-// the fp32 accumulator.  D = 64: lane = query row, columns = features
-// [32 ch, 32 ch + 32).  D = 128: lane = feature, columns = query rows
-// q0 + [32 ch, 32 ch + 32).
-template <int HD, bool QLANE>
-__device__ __forceinline__ void dq_to_global(const uint32_t (&v)[32], float* acc, int q0, int lr, int ch, int S,
-                                             float sc) {
-  if (QLANE) {
-    const int q = q0 + lr;
-    if (q < S) {
-      float4* dst = reinterpret_cast<float4*>(acc + (size_t)q * HD) + 8 * ch;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        atomicAdd(dst + i, make_float4(__uint_as_float(v[4 * i]) * sc, __uint_as_float(v[4 * i + 1]) * sc,
-                                       __uint_as_float(v[4 * i + 2]) * sc, __uint_as_float(v[4 * i + 3]) * sc));
-    }
-  } else {
-    float* col = acc + lr;
-    const int qh = q0 + 32 * ch;
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-      if (qh + e < S) atomicAdd(col + (size_t)(qh + e) * HD, __uint_as_float(v[e]) * sc);
-  }
-}
-
 template <int HD, bool CAUSAL>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdArgs a) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
   using C = BwdCfg<HD>;
   constexpr int BM = C::BM, ST = C::ST, HALF = C::HALF, NCH = C::NCH;
 
@@ -132,7 +117,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint8_t* gbase = smem_raw + (base - raw);
 
   const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
-  const uint32_t sPT = base + C::OFF_PT, sDST = base + C::OFF_DST;
+  const uint32_t sDST = base + C::OFF_DST, sSTG = base + C::OFF_STG;
   auto sQ = [&](int s) { return base + C::OFF_Q + s * C::QTILE; };
   auto sDO = [&](int s) { return base + C::OFF_DO + s * C::QTILE; };
   const float* lse_s = reinterpret_cast<const float*>(gbase + C::OFF_LSE);
@@ -140,15 +125,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const uint32_t bars = base + C::OFF_BAR;
   const uint32_t bar_kv = bars;
   auto bar_qfull = [&](int s) { return bars + 8u * (1 + s); };
-  auto bar_qempty = [&](int s) { return bars + 8u * (3 + s); };
-  const uint32_t bar_spfull = bars + 8u * 5;   // S^T, dP^T of a step are in TMEM
-  const uint32_t bar_spfree = bars + 8u * 6;   // ... and have been read (8 warps)
-  const uint32_t bar_pdsfull = bars + 8u * 7;  // P^T, dS^T of a step are in smem (8 warps)
-  const uint32_t bar_ptfree = bars + 8u * 8;   // dV of a step is done with P^T
-  auto bar_dqfull = [&](int b) { return bars + 8u * (9 + b); };
-  auto bar_dqfree = [&](int b) { return bars + 8u * (11 + b); };
-  const uint32_t bar_fin = bars + 8u * 13;
-  const uint32_t bar_dstfree = bars + 8u * 14;  // dK, dQ of a step are done with dS^T
+  auto bar_qempty = [&](int s) { return bars + 8u * (1 + ST + s); };
+  const uint32_t bar_spfull = bars + 8u * (1 + 2 * ST);   // S^T, dP^T of a step are in TMEM
+  const uint32_t bar_spfree = bars + 8u * (2 + 2 * ST);   // ... and have been read (8 warps)
+  const uint32_t bar_pdsfull = bars + 8u * (3 + 2 * ST);  // P^T (TMEM), dS^T (smem) written (8 warps)
+  const uint32_t bar_ptfree = bars + 8u * (4 + 2 * ST);   // dV of a step is done with P^T
+  const uint32_t bar_dqfull = bars + 8u * (5 + 2 * ST);   // dQ tile of a step is in TMEM
+  const uint32_t bar_dqfree = bars + 8u * (6 + 2 * ST);   // ... and has been read (8 warps)
+  const uint32_t bar_fin = bars + 8u * (7 + 2 * ST);
+  const uint32_t bar_dstfree = bars + 8u * (8 + 2 * ST);  // dK, dQ of a step are done with dS^T
+  const uint32_t bar_stgfull = bars + 8u * (9 + 2 * ST);  // dQ tile staged (8 warps)
+  const uint32_t bar_stgfree = bars + 8u * (10 + 2 * ST); // staged tile read by the TMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 8 * C::NBAR);
   volatile int* abort = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + 8 * C::NBAR + 4);
 
@@ -170,15 +157,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     for (int s = 0; s < ST; ++s) {
       mbar_init(bar_qfull(s), 1);
       mbar_init(bar_qempty(s), 1);
-      mbar_init(bar_dqfull(s), 1);
-      mbar_init(bar_dqfree(s), 8);
     }
     mbar_init(bar_spfull, 1);
     mbar_init(bar_spfree, 8);
     mbar_init(bar_pdsfull, 8);
     mbar_init(bar_ptfree, 1);
-    mbar_init(bar_dstfree, 1);
+    mbar_init(bar_dqfull, 1);
+    mbar_init(bar_dqfree, 8);
     mbar_init(bar_fin, 1);
+    mbar_init(bar_dstfree, 1);
+    mbar_init(bar_stgfull, 8);
+    mbar_init(bar_stgfree, 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -203,9 +192,21 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tma_load_4d(sK + sl * C::KSLAB, &tm_k, bar_kv, 64 * sl, kvh, 128 * j, b);
         tma_load_4d(sV + sl * C::KSLAB, &tm_v, bar_kv, 64 * sl, kvh, 128 * j, b);
       }
+      // L2 prefetch of the Q / dO tiles PF steps ahead of the loads
+      constexpr int PF = 4;
+      auto prefetch = [&](int it) {
+        const int h = kvh * G + it / per_head;
+        const int q0 = (i0 + it % per_head) * BM;
+        for (int sl = 0; sl < C::NSLAB; ++sl) {
+          tma_prefetch_4d(&tm_q, 64 * sl, h, q0, b);
+          tma_prefetch_4d(&tm_do, 64 * sl, h, q0, b);
+        }
+      };
+      for (int it = 0; it < PF && it < n_it; ++it) prefetch(it);
       int issued = 0;
       for (int it = 0; it < n_it; ++it) {
         const int s = it % ST;
+        if (it + PF < n_it) prefetch(it + PF);
         if (!mbar_wait_bounded(bar_qempty(s), ((it / ST) & 1) ^ 1, abort, B_QEMPTY)) break;
         const int h = kvh * G + it / per_head;
         const int q0 = (i0 + it % per_head) * BM;
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     if (lane == 0) {
       // ===================================================== MMA issuer
       constexpr uint32_t ID_S = idesc_bf16(128, BM, 0, 0);   // K|V (K-major) x Q|dO (K-major)
-      constexpr uint32_t ID_GV = idesc_bf16(128, HD, 0, 1);  // P^T|dS^T (K-major) x dO|Q (MN-major)
+      constexpr uint32_t ID_GV = idesc_bf16(128, HD, 0, 1);  // P^T (TMEM) | dS^T (smem, K-major) x dO|Q (MN-major)
       constexpr uint32_t ID_Q = C::QLANE ? idesc_bf16(128, HD, 1, 1) : idesc_bf16(128, BM, 1, 1);
       auto issue_sdp = [&](int s) {
         // S^T = K Q^T and dP^T = V dO^T (reduction over the features)
@@ -264,12 +265,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         }
         if (!mbar_wait_bounded(bar_pdsfull, it & 1, abort, B_PDSFULL)) break;
         tc_fence_after();
-        // dV += P^T dO (reduction over the BM query rows)
-        for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t po = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss(tmem + C::T_DV, sw128_desc(sPT + po, 16, 1024), sw128_desc(sDO(s) + kk * 2048, C::QSLAB, 1024),
-                 ID_GV, (it > 0 || kk > 0) ? 1u : 0u);
-        }
+        // dV += P^T dO (A = P^T from TMEM; reduction over the BM query rows)
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(tmem + C::T_DV, tmem + C::T_P + 8 * kk, sw128_desc(sDO(s) + kk * 2048, C::QSLAB, 1024), ID_GV,
+                 (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar_ptfree);
         // dK += dS^T Q
         for (int kk = 0; kk < BM / 16; ++kk) {
@@ -277,26 +276,45 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           mma_ss(tmem + C::T_DK, sw128_desc(sDST + po, 16, 1024), sw128_desc(sQ(s) + kk * 2048, C::QSLAB, 1024),
                  ID_GV, (it > 0 || kk > 0) ? 1u : 0u);
         }
-        // dQ tile (reduction over the 128 keys) into TMEM buffer it % 2
-        const int qb = it & 1;
-        if (it >= 2 && !mbar_wait_bounded(bar_dqfree(qb), ((it >> 1) - 1) & 1, abort, B_DQFREE)) break;
+        mma_commit(bar_qempty(s));  // Q, dO of this step are no longer read
+        // dQ tile (reduction over the 128 keys) once the previous one has been read
+        if (it >= 1 && !mbar_wait_bounded(bar_dqfree, (it - 1) & 1, abort, B_DQFREE)) break;
         tc_fence_after();
-        const uint32_t tdq = tmem + C::T_DQ + qb * C::DQ_COLS;
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t ds_mn = sw128_desc(sDST + kk * 2048, 128 * 128, 1024);
           const uint64_t k_mn = sw128_desc(sK + kk * 2048, C::KSLAB, 1024);
           if (C::QLANE)
-            mma_ss(tdq, ds_mn, k_mn, ID_Q, kk > 0);   // dQ = dS K
+            mma_ss(tmem + C::T_DQ, ds_mn, k_mn, ID_Q, kk > 0);   // dQ = dS K
           else
-            mma_ss(tdq, k_mn, ds_mn, ID_Q, kk > 0);   // dQ^T = K^T dS^T
+            mma_ss(tmem + C::T_DQ, k_mn, ds_mn, ID_Q, kk > 0);   // dQ^T = K^T dS^T
         }
-        mma_commit(bar_dqfull(qb));
-        mma_commit(bar_qempty(s));
+        mma_commit(bar_dqfull);
         mma_commit(bar_dstfree);
       }
       mma_commit(bar_fin);
       volatile int never = 0;
       mbar_wait_bounded(bar_fin, 0, &never, B_FIN);
+    }
+  } else if (warp == BWD_WARP_RED) {
+    if (lane == 0) {
+      // ===================================================== dQ tiles -> fp32 accumulator (TMA add)
+      tma_prefetch_desc(&tm_dq);
+      for (int t = 0; t < n_it; ++t) {
+        if (!mbar_wait_bounded(bar_stgfull, t & 1, abort, B_STGFULL)) break;
+        const int h = kvh * G + t / per_head;
+        const int q0 = (i0 + t % per_head) * BM;
+        const int bh = b * a.Hq + h;
+        for (int bx = 0; bx < 4; ++bx) {
+          // D = 64: box (feature block bx & 1, row block bx >> 1); D = 128: feature block bx
+          const int c0 = C::QLANE ? 32 * (bx & 1) : 32 * bx;
+          const int r0 = C::QLANE ? q0 + 64 * (bx >> 1) : q0;
+          if (r0 < a.S) tma_reduce_add_3d(&tm_dq, sSTG + bx * C::DQ_BOX, c0, r0, bh);
+        }
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(bar_stgfree);
+      }
+      bulk_wait0();
     }
   } else if (warp < 8) {
     // ===================================================== P^T, dS^T (thread = key row)
@@ -308,20 +326,40 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint64_t cc2 = f2_pack(a.scale_log2, a.scale_log2);
     const float sc = a.scale;
     bool ok = true;
-    // dQ tile of step `t` (previous step) from TMEM to the fp32 accumulator
+    // dQ tile of step `t` from TMEM into the staging tile for the TMA add
     auto dq_readout = [&](int t) -> bool {
-      const int qb = t & 1;
-      if (!wait_warp(bar_dqfull(qb), (t >> 1) & 1, abort, B_DQFULL)) return false;
+      if (!wait_warp(bar_dqfull, t & 1, abort, B_DQFULL)) return false;
       tc_fence_after();
       uint32_t v[32];
-      tmem_ld32(tmem + lane_off + C::T_DQ + qb * C::DQ_COLS + 32 * ch, v);
+      tmem_ld32(tmem + lane_off + C::T_DQ + 32 * ch, v);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_dqfree(qb));
-      const int h = kvh * G + t / per_head;
-      const int q0 = (i0 + t % per_head) * BM;
-      dq_to_global<HD, C::QLANE>(v, a.dqacc + ((size_t)b * a.Hq + h) * (size_t)a.S * HD, q0, kr, ch, a.S, sc);
+      if (lane == 0) mbar_arrive(bar_dqfree);
+      if (t > 0 && !wait_warp(bar_stgfree, (t - 1) & 1, abort, B_STGFREE)) return false;
+      if (C::QLANE) {
+        // lane = query row kr, columns = features [32 ch, 32 ch + 32): one 128-byte box row
+        const uint32_t row = sSTG + ((kr >> 6) * 2 + ch) * C::DQ_BOX + (kr & 63) * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(row + ((c ^ (kr & 7)) << 4)),
+                       "f"(__uint_as_float(v[4 * c]) * sc), "f"(__uint_as_float(v[4 * c + 1]) * sc),
+                       "f"(__uint_as_float(v[4 * c + 2]) * sc), "f"(__uint_as_float(v[4 * c + 3]) * sc)
+                       : "memory");
+      } else {
+        // lane = feature kr (box kr / 32, column kr % 32), columns = query rows 32 ch + e
+        const uint32_t boxb = sSTG + wq * C::DQ_BOX + ((lane & 3) << 2);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int q = 32 * ch + e;
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(boxb + q * 128 + (((lane >> 2) ^ (q & 7)) << 4)),
+                       "f"(__uint_as_float(v[e]) * sc)
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_stgfull);
       return true;
     };
     for (int it = 0; it < n_it; ++it) {
@@ -381,8 +419,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           ok = false;
           break;
         }
-        store_row16(sPT, kr, c0 + 32 * cc, &pk[0]);
-        store_row16(sPT, kr, c0 + 32 * cc + 16, &pk[8]);
+        tmem_st16(tmem + lane_off + C::T_P + (c0 >> 1) + 16 * cc, pk);
       }
       if (!ok) break;
       // ... and the previous step's dK, dQ with dS^T
@@ -395,10 +432,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         store_row16(sDST, kr, c0 + 32 * cc, &dk[cc][0]);
         store_row16(sDST, kr, c0 + 32 * cc + 16, &dk[cc][8]);
       }
+      tmem_wait_st();
       fence_proxy_async_smem();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_pdsfull);
-      // the previous step's dQ tile is ready by now (its MMA was issued before this step's P^T, dS^T)
+      // the previous step's dQ tile (its MMA was issued before this step's P^T, dS^T)
       if (it > 0 && !dq_readout(it - 1)) {
         ok = false;
         break;

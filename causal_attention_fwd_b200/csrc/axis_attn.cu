@@ -74,6 +74,20 @@ bool make_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int D, int
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over the fp32 dQ accumulator [B*Hq][S][D]: dims (D, S, B*Hq), box
+// (32, 64, 1), 128-byte swizzle; used by TMA reduce-adds (rows past S skipped).
+bool make_dq_map(CUtensorMap* map, const float* ptr, int BH, int S, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)S * D * 4};
+  const cuuint32_t box[3] = {32, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct WsLayout {
@@ -118,12 +132,12 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
 
 template <int HD, bool CAUSAL>
 int launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                    const BwdArgs& a, cudaStream_t st, int dev) {
+                    const CUtensorMap& mdq, const BwdArgs& a, cudaStream_t st, int dev) {
   auto kern = attn_bwd_kernel<HD, CAUSAL>;
   static bool done[64];
   if (int rc = set_smem(kern, BwdCfg<HD>::SMEM, dev, done)) return rc;
   const unsigned grid = (unsigned)((a.S + 127) / 128) * a.B * a.Hkv;
-  kern<<<grid, BWD_THREADS, BwdCfg<HD>::SMEM, st>>>(mq, mk, mv, mdo, a);
+  kern<<<grid, BWD_THREADS, BwdCfg<HD>::SMEM, st>>>(mq, mk, mv, mdo, mdq, a);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
@@ -226,6 +240,8 @@ extern "C" int axis_attn_bwd_main(const void* q, const void* k, const void* v, c
       !make_map(&mk, k, B, S, Hkv, D, 128) || !make_map(&mv, v, B, S, Hkv, D, 128))
     return AXIS_ATTN_ERR_CUDA;
   const WsPtrs p = ws_ptrs(workspace, w);
+  CUtensorMap mdq;
+  if (!make_dq_map(&mdq, p.dqacc, B * Hq, S, D)) return AXIS_ATTN_ERR_CUDA;
   BwdArgs a;
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
@@ -241,10 +257,10 @@ extern "C" int axis_attn_bwd_main(const void* q, const void* k, const void* v, c
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D == 64)
-    return causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, a, st, dev)
-                  : launch_bwd_main<64, false>(mq, mk, mv, mdo, a, st, dev);
-  return causal ? launch_bwd_main<128, true>(mq, mk, mv, mdo, a, st, dev)
-                : launch_bwd_main<128, false>(mq, mk, mv, mdo, a, st, dev);
+    return causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, mdq, a, st, dev)
+                  : launch_bwd_main<64, false>(mq, mk, mv, mdo, mdq, a, st, dev);
+  return causal ? launch_bwd_main<128, true>(mq, mk, mv, mdo, mdq, a, st, dev)
+                : launch_bwd_main<128, false>(mq, mk, mv, mdo, mdq, a, st, dev);
 }
 
 extern "C" int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, int D, void* workspace,
