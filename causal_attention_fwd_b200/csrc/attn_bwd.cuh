@@ -226,74 +226,81 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         mbar_wait_bounded(bar_qfull(it % ST), (it / ST) & 1, &never, B_QFULL);
     }
   } else if (warp == BWD_WARP_MMA) {
-    if (lane == 0) {
+    {
       // ===================================================== MMA issuer
+      // The whole warp runs this loop (warp-uniform waits and descriptors);
+      // one elected lane issues each MMA and commit.
       constexpr uint32_t ID_S = idesc_bf16(128, BM, 0, 0);   // K|V (K-major) x Q|dO (K-major)
       constexpr uint32_t ID_GV = idesc_bf16(128, HD, 0, 1);  // P^T (TMEM) | dS^T (smem, K-major) x dO|Q (MN-major)
       constexpr uint32_t ID_Q = C::QLANE ? idesc_bf16(128, HD, 1, 1) : idesc_bf16(128, BM, 1, 1);
       auto issue_sdp = [&](int s) {
         // S^T = K Q^T and dP^T = V dO^T (reduction over the features)
+#pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KSLAB + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::QSLAB + (kk & 3) * 32;
-          mma_ss(tmem + C::T_S, sw128_desc(sK + ko, 16, 1024), sw128_desc(sQ(s) + qo, 16, 1024), ID_S, kk > 0);
+          mma_ss_w(tmem + C::T_S, sw128_desc(sK + ko, 16, 1024), sw128_desc(sQ(s) + qo, 16, 1024), ID_S, kk > 0);
         }
+#pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t ko = (kk >> 2) * C::KSLAB + (kk & 3) * 32;
           const uint32_t qo = (kk >> 2) * C::QSLAB + (kk & 3) * 32;
-          mma_ss(tmem + C::T_DP, sw128_desc(sV + ko, 16, 1024), sw128_desc(sDO(s) + qo, 16, 1024), ID_S,
-                 kk > 0);
+          mma_ss_w(tmem + C::T_DP, sw128_desc(sV + ko, 16, 1024), sw128_desc(sDO(s) + qo, 16, 1024), ID_S,
+                   kk > 0);
         }
       };
-      bool ok = mbar_wait_bounded(bar_kv, 0, abort, B_KV) && n_it > 0 &&
-                mbar_wait_bounded(bar_qfull(0), 0, abort, B_QFULL);
+      bool ok = wait_warp<true>(bar_kv, 0, abort, B_KV) && n_it > 0 &&
+                wait_warp<true>(bar_qfull(0), 0, abort, B_QFULL);
       if (ok) {
         tc_fence_after();
         issue_sdp(0);
-        mma_commit(bar_spfull);
+        mma_commit_w(bar_spfull);
       }
       for (int it = 0; ok && it < n_it; ++it) {
         const int s = it % ST;
         // next step's S^T, dP^T as soon as this step's are out of TMEM
         if (it + 1 < n_it) {
-          if (!mbar_wait_bounded(bar_qfull((it + 1) % ST), ((it + 1) / ST) & 1, abort, B_QFULL) ||
-              !mbar_wait_bounded(bar_spfree, it & 1, abort, B_SPFREE))
+          if (!wait_warp<true>(bar_qfull((it + 1) % ST), ((it + 1) / ST) & 1, abort, B_QFULL) ||
+              !wait_warp<true>(bar_spfree, it & 1, abort, B_SPFREE))
             break;
           tc_fence_after();
           issue_sdp((it + 1) % ST);
-          mma_commit(bar_spfull);
+          mma_commit_w(bar_spfull);
         }
-        if (!mbar_wait_bounded(bar_pdsfull, it & 1, abort, B_PDSFULL)) break;
+        if (!wait_warp<true>(bar_pdsfull, it & 1, abort, B_PDSFULL)) break;
         tc_fence_after();
         // dV += P^T dO (A = P^T from TMEM; reduction over the BM query rows)
+#pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + C::T_DV, tmem + C::T_P + 8 * kk, sw128_desc(sDO(s) + kk * 2048, C::QSLAB, 1024), ID_GV,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar_ptfree);
+          mma_ts_w(tmem + C::T_DV, tmem + C::T_P + 8 * kk, sw128_desc(sDO(s) + kk * 2048, C::QSLAB, 1024), ID_GV,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_w(bar_ptfree);
         // dK += dS^T Q
+#pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t po = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss(tmem + C::T_DK, sw128_desc(sDST + po, 16, 1024), sw128_desc(sQ(s) + kk * 2048, C::QSLAB, 1024),
-                 ID_GV, (it > 0 || kk > 0) ? 1u : 0u);
+          mma_ss_w(tmem + C::T_DK, sw128_desc(sDST + po, 16, 1024), sw128_desc(sQ(s) + kk * 2048, C::QSLAB, 1024),
+                   ID_GV, (it > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar_qempty(s));  // Q, dO of this step are no longer read
+        mma_commit_w(bar_qempty(s));  // Q, dO of this step are no longer read
         // dQ tile (reduction over the 128 keys) once the previous one has been read
-        if (it >= 1 && !mbar_wait_bounded(bar_dqfree, (it - 1) & 1, abort, B_DQFREE)) break;
+        if (it >= 1 && !wait_warp<true>(bar_dqfree, (it - 1) & 1, abort, B_DQFREE)) break;
         tc_fence_after();
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t ds_mn = sw128_desc(sDST + kk * 2048, 128 * 128, 1024);
           const uint64_t k_mn = sw128_desc(sK + kk * 2048, C::KSLAB, 1024);
           if (C::QLANE)
-            mma_ss(tmem + C::T_DQ, ds_mn, k_mn, ID_Q, kk > 0);   // dQ = dS K
+            mma_ss_w(tmem + C::T_DQ, ds_mn, k_mn, ID_Q, kk > 0);   // dQ = dS K
           else
-            mma_ss(tmem + C::T_DQ, k_mn, ds_mn, ID_Q, kk > 0);   // dQ^T = K^T dS^T
+            mma_ss_w(tmem + C::T_DQ, k_mn, ds_mn, ID_Q, kk > 0);   // dQ^T = K^T dS^T
         }
-        mma_commit(bar_dqfull);
-        mma_commit(bar_dstfree);
+        mma_commit_w(bar_dqfull);
+        mma_commit_w(bar_dstfree);
       }
-      mma_commit(bar_fin);
+      mma_commit_w(bar_fin);
       volatile int never = 0;
-      mbar_wait_bounded(bar_fin, 0, &never, B_FIN);
+      wait_warp<true>(bar_fin, 0, &never, B_FIN);
     }
   } else if (warp == BWD_WARP_RED) {
     if (lane == 0) {
@@ -407,11 +414,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
               if ((CAUSAL && key > q + 1) || key >= a.S) p1 = 0.f;
             }
             const uint64_t pp = f2_pack(p0, p1);
-            float d0, d1;
-            f2_unpack(f2_mul(pp, f2_add(f2_pack(__uint_as_float(dpv[ee]), __uint_as_float(dpv[ee + 1])), nd)), d0,
-                      d1);
-            pk[ee / 2] = pack_bf16x2(p0, p1);
-            dk[cc][ee / 2] = pack_bf16x2(d0, d1);
+            const uint64_t dd =
+                f2_mul(pp, f2_add(f2_pack(__uint_as_float(dpv[ee]), __uint_as_float(dpv[ee + 1])), nd));
+                      pk[ee / 2] = pack_bf16x2(pp);
+            dk[cc][ee / 2] = pack_bf16x2(dd);
           }
         }
         // the previous step's dV must be done with P^T before it is overwritten
@@ -476,45 +482,62 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   }
 }
 
-// -Dr = -rowsum(dO * O) (fp32) and -LSE2 = -LSE * log2(e); rows S..S_pad-1
-// get 0 and -inf (so their P is exactly 0).  Also zeroes the dQ accumulator.
-// One thread per row.
+// -Dr = -rowsum(dO * O) (fp32) and -LSE2 = -LSE * log2(e) per (b, h, i); rows
+// S..S_pad-1 of each (b, h) get 0 and -inf (so their P is exactly 0).  Also
+// zeroes the dQ accumulator.  HBM-bound: the rows are visited in memory order
+// ([B, S, Hq] for O and dO), D/8 threads per row with one 16-byte load each of
+// O and dO, and a shuffle reduction inside the row's thread group.
 template <int HD>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                             const __nv_bfloat16* __restrict__ dout,
                                                             const float* __restrict__ lse, float* nlse2,
                                                             float* ndr, float4* dqacc, size_t dq_vec4,
                                                             int Hq, int S, int S_pad, int rows) {
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r < rows) {
-    const int bh = r / S_pad, i = r % S_pad;
-    float d = 0.f, l2 = -INFINITY;
-    if (i < S) {
-      const int b = bh / Hq, h = bh % Hq;
-      const size_t off = (((size_t)b * S + i) * Hq + h) * HD;
-      const uint4* po = reinterpret_cast<const uint4*>(o + off);
-      const uint4* pd = reinterpret_cast<const uint4*>(dout + off);
+  constexpr int TPR = HD / 8;  // threads per row
+  const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t nthreads = (size_t)gridDim.x * blockDim.x;
+  const size_t real_rows = (size_t)rows / S_pad * S;  // B * Hq * S, in [B, S, Hq] order
+  const size_t total = real_rows * TPR;
+  const size_t warp0 = gtid - (threadIdx.x & 31);  // warp-uniform loop: every lane joins the shuffles
+  for (size_t tw = warp0; tw < total; tw += nthreads) {
+    const size_t t = tw + (threadIdx.x & 31);
+    const bool act = t < total;
+    const size_t r = t / TPR;
+    const int part = (int)(t % TPR);
+    float d = 0.f;
+    if (act) {
+      const uint4 x = reinterpret_cast<const uint4*>(o + r * HD)[part];
+      const uint4 y = reinterpret_cast<const uint4*>(dout + r * HD)[part];
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-      for (int c = 0; c < HD / 8; ++c) {
-        const uint4 x = po[c], y = pd[c];
-        const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[k]));
-          const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ys[k]));
-          d = fmaf(xf.x, yf.x, d);
-          d = fmaf(xf.y, yf.y, d);
-        }
+      for (int k = 0; k < 4; ++k) {
+        const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[k]));
+        const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ys[k]));
+        d = fmaf(xf.x, yf.x, d);
+        d = fmaf(xf.y, yf.y, d);
       }
-      l2 = -lse[(size_t)bh * S + i] * 1.4426950408889634f;
-      d = -d;
     }
-    ndr[r] = d;
-    nlse2[r] = l2;
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off, TPR);
+    if (act && part == 0) {
+      const int h = (int)(r % Hq);
+      const size_t bi = r / Hq;  // b * S + i
+      const int i = (int)(bi % S);
+      const size_t bh = (bi / S) * Hq + h;
+      ndr[bh * S_pad + i] = -d;
+      nlse2[bh * S_pad + i] = -lse[bh * S + i] * 1.4426950408889634f;
+    }
   }
-  const size_t stride = (size_t)gridDim.x * blockDim.x;
-  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < dq_vec4; k += stride)
-    dqacc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  // padding rows of every (b, h)
+  const int pad = S_pad - S;
+  const size_t npad = (size_t)rows / S_pad * pad;
+  for (size_t t = gtid; t < npad; t += nthreads) {
+    const size_t bh = t / pad;
+    const int i = S + (int)(t % pad);
+    ndr[bh * S_pad + i] = 0.f;
+    nlse2[bh * S_pad + i] = -INFINITY;
+  }
+  for (size_t k = gtid; k < dq_vec4; k += nthreads) dqacc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dq[b,i,h,:] = bf16(dqacc[b,h,i,:]); 8 features per thread.

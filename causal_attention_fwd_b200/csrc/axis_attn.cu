@@ -210,7 +210,9 @@ extern "C" int axis_attn_bwd_prepare(const void* o, const void* dO, const float*
   const WsPtrs p = ws_ptrs(workspace, w);
   const int rows = B * Hq * w.S_pad;
   const size_t dq_vec4 = (size_t)B * Hq * S * D / 4;
-  const unsigned grid = (unsigned)((rows + 255) / 256);
+  // grid-stride kernel: a few waves of 256-thread blocks over the 148 SMs
+  const size_t work = (size_t)B * Hq * S * (D / 8);
+  const unsigned grid = (unsigned)((work + 255) / 256 < 148 * 16 ? (work + 255) / 256 : 148 * 16);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const auto* ob = static_cast<const __nv_bfloat16*>(o);
   const auto* db = static_cast<const __nv_bfloat16*>(dO);

@@ -19,24 +19,36 @@ namespace axis_attn {
 // axis_attn_get_status().
 __device__ unsigned int g_status;
 
-// Upper bound on any single wait inside a kernel (1 s).  No wait in a correct
-// run comes near it: every wait here is on work that the same CTA issued.
-// Once any CTA has timed out (g_status bit 0), the other CTAs stop waiting at
-// their next slow wait, so a faulty launch ends quickly instead of timing out
-// CTA by CTA.  The status stays set until axis_attn_get_status() clears it.
-#ifndef AXIS_ATTN_WAIT_LIMIT_NS
-#define AXIS_ATTN_WAIT_LIMIT_NS 1000000000ull
+// Upper bound on any single wait inside a kernel, in SM clock cycles (2^31,
+// about 1.1 s at 1.965 GHz).  No wait in a correct run comes near it: every
+// wait here is on work that the same CTA issued.  Once any CTA has timed out
+// (g_status bit 0), the other CTAs stop waiting at their next status check,
+// so a faulty launch ends quickly instead of timing out CTA by CTA.  The status
+// stays set until axis_attn_get_status() clears it.
+//
+// The polling loops below touch only shared memory and the SM's own cycle
+// counter on each pass; the global status word is read about every 2^16
+// cycles.  (Reading global memory or %globaltimer on every pass would make a
+// waiting thread notice a completed barrier up to a global round trip late.)
+#ifndef AXIS_ATTN_WAIT_LIMIT_CYCLES
+#define AXIS_ATTN_WAIT_LIMIT_CYCLES (1ull << 31)
 #endif
+#define AXIS_ATTN_STATUS_CHECK_CYCLES (1ull << 16)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t global_timer_ns() {
+__device__ __forceinline__ uint64_t sm_cycles() {
   uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
   return t;
 }
+
+__device__ __forceinline__ bool other_cta_timed_out() {
+  return (*reinterpret_cast<volatile unsigned int*>(&g_status) & 1u) != 0;
+}
+
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -84,58 +96,66 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Progress watchdog for event loops: call `stalled()` once per idle pass; it
-// returns true (after raising the abort flag and the status word) when no
-// progress was reported through `progress()` for AXIS_ATTN_WAIT_LIMIT_NS, or
-// when another role or CTA gave up.
+// returns true (after raising the abort flag, and the status word on a
+// timeout) when no progress was reported through `progress()` for
+// AXIS_ATTN_WAIT_LIMIT_CYCLES, or when another role or CTA gave up.
 struct Watchdog {
-  uint64_t t0;
-  __device__ __forceinline__ Watchdog() : t0(0) {}
-  __device__ __forceinline__ void progress() { t0 = 0; }
-  __device__ __forceinline__ bool stalled(volatile int* abort, int site);
+  uint64_t t0 = 0, last_check = 0;
+  bool idle = false;
+  __device__ __forceinline__ void progress() { idle = false; }
+  __device__ __forceinline__ bool stalled(volatile int* abort, int site) {
+    if (*abort) return true;
+    const uint64_t now = sm_cycles();
+    if (!idle) {
+      idle = true;
+      t0 = last_check = now;
+      return false;
+    }
+    if (now - last_check > AXIS_ATTN_STATUS_CHECK_CYCLES) {
+      last_check = now;
+      if (other_cta_timed_out()) {
+        *abort = 1;
+        return true;
+      }
+      if (now - t0 > AXIS_ATTN_WAIT_LIMIT_CYCLES) {
+        *abort = 1;
+        atomicOr(&g_status, 1u | ((unsigned)(site & 0xff) << 8));
+        return true;
+      }
+    }
+    return false;
+  }
 };
 
 // Wait until the phase of `bar` with parity `parity` has completed.  Gives up
-// when `*abort` becomes non-zero (another role of the CTA gave up) or after
-// AXIS_ATTN_WAIT_LIMIT_NS; in the latter case it raises `*abort` and records
-// the failure in g_status.  Returns true when the phase completed.
-// Called by a single thread, or by all lanes of a warp (see wait_warp).
+// when `*abort` becomes non-zero (another role of the CTA gave up), when
+// another CTA has timed out, or after AXIS_ATTN_WAIT_LIMIT_CYCLES; in the
+// last case it raises `*abort` and records the failure in g_status.  Returns
+// true when the phase completed.  Called by a single thread, or by all lanes
+// of a warp (see wait_warp).
 __device__ __forceinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, volatile int* abort,
                                                int site) {
-  const uint64_t t0 = global_timer_ns();
+  const uint64_t t0 = sm_cycles();
+  uint64_t last = t0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    // another CTA already timed out: results are void, stop waiting
-    if (*reinterpret_cast<volatile unsigned int*>(&g_status) & 1u) {
-      *abort = 1;
-      return false;
-    }
-    if (global_timer_ns() - t0 > AXIS_ATTN_WAIT_LIMIT_NS) {
-      *abort = 1;
-      atomicOr(&g_status, 1u | ((unsigned)(site & 0xff) << 8));
-      return false;
+    const uint64_t now = sm_cycles();
+    if (now - last > AXIS_ATTN_STATUS_CHECK_CYCLES) {
+      last = now;
+      if (other_cta_timed_out()) {  // results are void already: stop waiting
+        *abort = 1;
+        return false;
+      }
+      if (now - t0 > AXIS_ATTN_WAIT_LIMIT_CYCLES) {
+        *abort = 1;
+        atomicOr(&g_status, 1u | ((unsigned)(site & 0xff) << 8));
+        return false;
+      }
     }
   }
 }
 
-__device__ __forceinline__ bool Watchdog::stalled(volatile int* abort, int site) {
-  if (*abort) return true;
-  const uint64_t now = global_timer_ns();
-  if (t0 == 0) {
-    t0 = now;
-    return false;
-  }
-  if (*reinterpret_cast<volatile unsigned int*>(&g_status) & 1u) {
-    *abort = 1;
-    return true;
-  }
-  if (now - t0 > AXIS_ATTN_WAIT_LIMIT_NS) {
-    *abort = 1;
-    atomicOr(&g_status, 1u | ((unsigned)(site & 0xff) << 8));
-    return true;
-  }
-  return false;
-}
 
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort, int site) {
   return mbar_wait_loop(bar, parity, abort, site);
@@ -254,6 +274,59 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// ---- warp-wide issue: the whole (converged) warp executes these, with
+// warp-uniform operands; lane 0 issues the instruction (always the same lane:
+// a commit tracks only the MMAs its own thread issued).
+// Keeping the issuing loop warp-uniform lets descriptors live in uniform
+// registers, so each MMA issues in a few cycles instead of tens.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, e;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .u32 l;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "mov.u32 l, %%laneid;\n\t"
+      "setp.eq.u32 e, l, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .u32 l;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "mov.u32 l, %%laneid;\n\t"
+      "setp.eq.u32 e, l, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_w(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .u32 l;\n\t"
+      "mov.u32 l, %%laneid;\n\t"
+      "setp.eq.u32 e, l, 0;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+
+// Warp-uniform non-blocking barrier test (lane 0's view, broadcast).
+__device__ __forceinline__ bool mbar_test_w(uint32_t bar, uint32_t parity) {
+  return __shfl_sync(0xffffffffu, mbar_test(bar, parity) ? 1 : 0, 0) != 0;
 }
 
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far
@@ -397,6 +470,11 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -411,6 +489,11 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(uint64_t x2) {
+  float lo, hi;
+  f2_unpack(x2, lo, hi);
+  return pack_bf16x2(lo, hi);
 }
 
 }  // namespace axis_attn
