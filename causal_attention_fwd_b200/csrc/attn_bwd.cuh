@@ -416,7 +416,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             const uint64_t pp = f2_pack(p0, p1);
             const uint64_t dd =
                 f2_mul(pp, f2_add(f2_pack(__uint_as_float(dpv[ee]), __uint_as_float(dpv[ee + 1])), nd));
-                      pk[ee / 2] = pack_bf16x2(pp);
+            pk[ee / 2] = pack_bf16x2(pp);
             dk[cc][ee / 2] = pack_bf16x2(dd);
           }
         }

@@ -106,6 +106,17 @@ WsLayout ws_layout(int B, int Hq, int S, int D) {
   return w;
 }
 
+// Number of SMs of device `dev` (cached; the persistent kernels launch one CTA per SM).
+int sm_count(int dev) {
+  static int count[64];
+  if (count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    count[dev] = n;
+  }
+  return count[dev];
+}
+
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
 // `done` is a static of the calling template instantiation, so each kernel has
 // its own flags.
@@ -125,7 +136,8 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   auto kern = attn_fwd_kernel<HD, CAUSAL>;
   static bool done[64];
   if (int rc = set_smem(kern, FwdCfg<HD>::SMEM, dev, done)) return rc;
-  const unsigned grid = (unsigned)a.n_qblocks * a.B * a.Hq;
+  // persistent: one CTA per SM (the kernel walks its share of the items)
+  const unsigned grid = (unsigned)(a.n_items < sm_count(dev) ? a.n_items : sm_count(dev));
   kern<<<grid, FWD_THREADS, FwdCfg<HD>::SMEM, st>>>(mq, mk, mv, a);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
@@ -167,6 +179,7 @@ extern "C" int axis_attn_fwd(const void* q, const void* k, const void* v, void* 
   a.S = S;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
   a.n_qblocks = (S + 255) / 256;
+  a.n_items = a.n_qblocks * B * Hq;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D == 64)
     return causal ? launch_fwd<64, true>(mq, mk, mv, a, st, dev) : launch_fwd<64, false>(mq, mk, mv, a, st, dev);

@@ -95,52 +95,21 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Progress watchdog for event loops: call `stalled()` once per idle pass; it
-// returns true (after raising the abort flag, and the status word on a
-// timeout) when no progress was reported through `progress()` for
-// AXIS_ATTN_WAIT_LIMIT_CYCLES, or when another role or CTA gave up.
-struct Watchdog {
-  uint64_t t0 = 0, last_check = 0;
-  bool idle = false;
-  __device__ __forceinline__ void progress() { idle = false; }
-  __device__ __forceinline__ bool stalled(volatile int* abort, int site) {
-    if (*abort) return true;
-    const uint64_t now = sm_cycles();
-    if (!idle) {
-      idle = true;
-      t0 = last_check = now;
-      return false;
-    }
-    if (now - last_check > AXIS_ATTN_STATUS_CHECK_CYCLES) {
-      last_check = now;
-      if (other_cta_timed_out()) {
-        *abort = 1;
-        return true;
-      }
-      if (now - t0 > AXIS_ATTN_WAIT_LIMIT_CYCLES) {
-        *abort = 1;
-        atomicOr(&g_status, 1u | ((unsigned)(site & 0xff) << 8));
-        return true;
-      }
-    }
-    return false;
-  }
-};
-
 // Wait until the phase of `bar` with parity `parity` has completed.  Gives up
 // when `*abort` becomes non-zero (another role of the CTA gave up), when
 // another CTA has timed out, or after AXIS_ATTN_WAIT_LIMIT_CYCLES; in the
 // last case it raises `*abort` and records the failure in g_status.  Returns
 // true when the phase completed.  Called by a single thread, or by all lanes
-// of a warp (see wait_warp).
-__device__ __forceinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, volatile int* abort,
-                                               int site) {
-  const uint64_t t0 = sm_cycles();
-  uint64_t last = t0;
+// of a warp (see wait_warp).  The poll loop reads only the barrier, the
+// 32-bit SM clock and the abort flag; try_wait suspends the thread in
+// hardware between polls.
+__device__ __forceinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, volatile int* abort, int site) {
+  const uint32_t t0 = (uint32_t)clock();
+  uint32_t last = t0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    const uint64_t now = sm_cycles();
+    const uint32_t now = (uint32_t)clock();
     if (now - last > AXIS_ATTN_STATUS_CHECK_CYCLES) {
       last = now;
       if (other_cta_timed_out()) {  // results are void already: stop waiting
@@ -156,13 +125,13 @@ __device__ __forceinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, vo
   }
 }
 
-
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort, int site) {
   return mbar_wait_loop(bar, parity, abort, site);
 }
 
-// Fast path inline (one try_wait); the timed loop only runs on a miss.  INL
-// inlines the loop too: code under setmaxnreg must not make calls.
+// One try_wait inline; on a miss the poll loop, out of line (INL = false: less
+// code at each call site, but the compiler saves the caller's live registers
+// around the call) or inline (INL = true: no call, more code).
 template <bool INL = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
                                                   int site) {

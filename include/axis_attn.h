@@ -155,7 +155,7 @@ int axis_attn_get_status(void* stream);
 /*
  * Diagnostics: the raw device status word that the last axis_attn_get_status()
  * call read before clearing it (0 if none was set).  Bit 0: a wait timed out;
- * bits 8..15: the wait site that first did (1..9: forward kernel, 21..30:
+ * bits 8..15: the wait site that first did (1..10: forward kernel, 21..32:
  * backward main kernel).
  */
 unsigned int axis_attn_last_status_word(void);
