@@ -35,9 +35,9 @@
 //     of the current one has read Q, and its first P V product waits only for
 //     the epilogue to have read O out of TMEM.
 //
-// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+HD) O1 [256+HD,256+2HD),
-// and at D = 64 P0 P1 in the last 128 columns (at D = 128 P is written over the
-// first half of its S).
+// TMEM columns: D = 64: S0 [0,128) S1 [128,256) O0 [256,320) O1 [320,384)
+// P0 [384,448) P1 [448,512); D = 128: S [0,128) (shared by the two tiles, which
+// take turns) P0 [128,192) P1 [192,256) O0 [256,384) O1 [384,512).
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -94,12 +94,14 @@ struct FwdCfg {
   // it, long before the P V products free the V stage)
   static constexpr int KST = HD == 64 ? 5 : 2;
   static constexpr int VST = HD == 64 ? 5 : 2;
-  // TMEM columns.  D = 64: S0 S1 O0 O1 P0 P1 (P has its own columns, so the
-  // next S of a tile can be issued as soon as the softmax has read the last
-  // one).  D = 128: S0 S1 O0 O1 fill all 512 columns and P (bf16) is written
-  // over the first half of its S, so the next S waits for the P V product.
-  static constexpr bool P_SEPARATE = HD == 64;
-  static constexpr uint32_t T_S = 0, T_O = 256, T_P = P_SEPARATE ? 256 + 2 * HD : 0;
+  // TMEM columns (512).  D = 64: S0 S1 O0 O1 P0 P1.  D = 128: one S shared by
+  // the two tiles, P0 P1, O0 O1 (the tiles take turns, so S alternates between
+  // them; the S of one tile is issued as soon as the other tile has read its
+  // own out).  P always has its own columns: the next S never waits for a
+  // P V product.
+  static constexpr bool SHARED_S = HD == 128;
+  static constexpr uint32_t T_P = SHARED_S ? 128 : 384, T_O = 256;
+  static __host__ __device__ constexpr uint32_t t_s(int t) { return SHARED_S ? 0u : 128u * t; }
   static constexpr int NBAR = 23 + 2 * KST + 2 * VST;
   static constexpr uint32_t XCH_OFF = (2 + KST + VST) * TILE;  // row-max / row-sum exchange
   static constexpr uint32_t XCH_BYTES = 2 * 2 * 2 * 128 * 4;   // [parity][tile][half][row] fp32
@@ -306,10 +308,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   } else if (warp == FWD_WARP_MMA) {
     // ===================================================== S issuer
     // S_t(j) = Q_t K_j^T in the order S0(0) S1(0) S0(1) S1(1) ... over all
-    // items.  S_t(j) may overwrite S_t's columns once the softmax has read
-    // S_t(j-1) (D = 64: sfree) or, with P written over S (D = 128), once
-    // P_t(j-1) V has completed (o).  After an item's last S, Q may take the
-    // next item (qempty).  The whole warp runs the loop with warp-uniform
+    // items.  An S may overwrite its columns once the softmax has read the
+    // previous S held there (sfree): S_t(j-1) at D = 64, the previous S of
+    // either tile at D = 128 (one shared S).  After an item's last S, Q may
+    // take the next item (qempty).  The whole warp runs the loop with warp-uniform
     // waits; lane 0 issues each instruction.  js[t]: S products of tile t so
     // far (over all items), g: kv tiles of earlier items.
     constexpr uint32_t ID_S = idesc_bf16(128, 128, 0, 0);   // Q (K-major) x K (K-major)
@@ -329,17 +331,16 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (!ok || j >= n[t]) continue;
-          if (js[t] > 0) {
-            ok = C::P_SEPARATE ? wait_warp<true>(bar_sfree(t), (js[t] - 1) & 1, abort, F_SFULL)
-                               : wait_warp<true>(bar_o(t), (js[t] - 1) & 1, abort, F_OBAR);
-            if (!ok) break;
-          }
+          // S_t may overwrite its columns once their last S has been read
+          const int prev = C::SHARED_S ? js[0] + js[1] - 1 : js[t] - 1;
+          if (prev >= 0 && !(ok = wait_warp<true>(bar_sfree(C::SHARED_S ? 0 : t), prev & 1, abort, F_SFULL)))
+            break;
           if (!(ok = wait_warp<true>(bar_kfull(s), ((g + j) / KST) & 1, abort, F_KFULL))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * SLAB + (kk & 3) * 32;
-            mma_ss_w(tmem + C::T_S + t * 128, sw128_desc(sQ + t * TILE + off, 16, 1024),
+            mma_ss_w(tmem + C::t_s(t), sw128_desc(sQ + t * TILE + off, 16, 1024),
                      sw128_desc(sK + s * TILE + off, 16, 1024), ID_S, kk > 0);
           }
           mma_commit_w(bar_sfull(t));
@@ -386,7 +387,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           if (!(ok = wait_warp<true>(bar_vfull(s), ((g + j) / VST) & 1, abort, F_VFULL))) break;
           tc_fence_after();
           const uint32_t tO = tmem + C::T_O + t * HD;
-          const uint32_t tP = tmem + C::T_P + t * (C::P_SEPARATE ? 64 : 128);
+          const uint32_t tP = tmem + C::T_P + t * 64;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts_w(tO, tP + kk * 8, sw128_desc(sV + s * TILE + kk * 2048, SLAB, 1024), ID_PV,
@@ -411,9 +412,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     const int t = warp >> 3, hf = (warp >> 2) & 1, wq = warp & 3;
     const int r = wq * 32 + lane;                   // row in tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::T_S + t * 128 + hf * 64;
+    const uint32_t tS = tmem + lane_off + C::t_s(t) + hf * 64;
     const uint32_t tO = tmem + lane_off + C::T_O + t * HD + hf * (HD / 2);
-    const uint32_t tP = tmem + lane_off + C::T_P + t * (C::P_SEPARATE ? 64 : 128) + hf * 32;
+    const uint32_t tP = tmem + lane_off + C::T_P + t * 64 + hf * 32;
     const uint32_t bx = bar_xch(t, wq);
     // exchange slot of this thread's row: [parity][tile][half][row]
     auto xslot = [&](int par, int half) { return xch + ((par * 2 + t) * 2 + half) * 128 + r; };
@@ -446,12 +447,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         tmem_ld32(tS, v0);
         tmem_ld32(tS + 32, v1);
         tmem_wait_ld();
-        if (C::P_SEPARATE) {
-          // S_t is in registers: its columns may take the next S
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_sfree(t));
-        }
+        // S is in registers: its columns may take the next S
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_sfree(C::SHARED_S ? 0 : t));
         if (masked) {
           mask_row(v0, 0, limit);
           mask_row(v1, 32, limit);
