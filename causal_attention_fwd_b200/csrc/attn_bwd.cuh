@@ -13,13 +13,16 @@
 //     exactly 0); zero the fp32 dQ accumulator;
 //   * main kernel: one CTA per (b, kv head, 128-key tile); K_j, V_j stay in
 //     shared memory while the CTA walks every query head of the group and every
-//     query tile that can see the keys.  Per tile (one thread issues all MMAs):
+//     query tile that can see the keys.  Per tile (two threads issue the
+//     MMAs, one the score products, one the gradient products):
 //       S^T = K Q^T and dP^T = V dO^T into TMEM (thread = key row),
 //       P^T = 2^(S^T c - LSE2), dS^T = P^T (dP^T - Dr) by 8 warps from TMEM,
 //       P^T back to TMEM (bf16), dS^T to shared memory (bf16, 128B swizzle),
 //       dV += P^T dO (A from TMEM), dK += dS^T Q, and dQ of the tile,
-//     dQ is read from TMEM by a fourth warpgroup and added into the fp32
-//     accumulator with vector atomics; dK, dV stay in TMEM until the end;
+//     the compute warps copy each dQ tile from TMEM into a swizzled
+//     shared-memory staging tile, which one thread adds into the fp32
+//     accumulator with TMA reduce-add copies; dK, dV stay in TMEM until the
+//     end;
 //   * dQ finalize (HBM-bound): bf16 copy of the accumulator in [B,S,Hq,D].
 // D = 64 uses 128-row query tiles and dQ = dS K (TMEM lane = query row);
 // D = 128 uses 64-row query tiles (shared memory) and dQ^T = K^T dS^T (TMEM
@@ -79,13 +82,14 @@ struct BwdCfg {
 
 // Warps 0-7: P^T / dS^T (thread = key row, half the query columns each) and
 // the dQ tile of the previous step into the staging tile; warp 8 loads; warp 9
-// issues the MMAs and owns TMEM; warp 10 issues the TMA reduce-adds of the dQ
-// tiles into the fp32 accumulator; warp 11 spare.  384 threads: up to 168
-// registers each.
+// issues the score MMAs and owns TMEM; warp 10 issues the TMA reduce-adds of
+// the dQ tiles into the fp32 accumulator; warp 11 issues the gradient MMAs.
+// 384 threads: up to 168 registers each.
 constexpr int BWD_THREADS = 384;
 constexpr int BWD_WARP_LOAD = 8;
 constexpr int BWD_WARP_MMA = 9;
 constexpr int BWD_WARP_RED = 10;
+constexpr int BWD_WARP_GRAD = 11;
 
 enum BwdSite { B_KV = 21, B_QEMPTY, B_QFULL, B_SPFREE, B_PDSFULL, B_DQFREE, B_SPFULL, B_DQFULL, B_FIN, B_PDSFREE,
                B_STGFULL, B_STGFREE };
@@ -156,7 +160,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(bar_kv, 1);
     for (int s = 0; s < ST; ++s) {
       mbar_init(bar_qfull(s), 1);
-      mbar_init(bar_qempty(s), 1);
+      mbar_init(bar_qempty(s), 2);  // one commit from each MMA issuer
     }
     mbar_init(bar_spfull, 1);
     mbar_init(bar_spfree, 8);
@@ -164,7 +168,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(bar_ptfree, 1);
     mbar_init(bar_dqfull, 1);
     mbar_init(bar_dqfree, 8);
-    mbar_init(bar_fin, 1);
+    mbar_init(bar_fin, 2);
     mbar_init(bar_dstfree, 1);
     mbar_init(bar_stgfull, 8);
     mbar_init(bar_stgfree, 1);
@@ -225,15 +229,26 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       for (int it = issued - ST > 0 ? issued - ST : 0; it < issued; ++it)
         mbar_wait_bounded(bar_qfull(it % ST), (it / ST) & 1, &never, B_QFULL);
     }
-  } else if (warp == BWD_WARP_MMA) {
-    {
-      // ===================================================== MMA issuer
-      // The whole warp runs this loop (warp-uniform waits and descriptors);
-      // one elected lane issues each MMA and commit.
-      constexpr uint32_t ID_S = idesc_bf16(128, BM, 0, 0);   // K|V (K-major) x Q|dO (K-major)
-      constexpr uint32_t ID_GV = idesc_bf16(128, HD, 0, 1);  // P^T (TMEM) | dS^T (smem, K-major) x dO|Q (MN-major)
-      constexpr uint32_t ID_Q = C::QLANE ? idesc_bf16(128, HD, 1, 1) : idesc_bf16(128, BM, 1, 1);
-      auto issue_sdp = [&](int s) {
+  } else if (warp == BWD_WARP_MMA || warp == BWD_WARP_GRAD) {
+    // ===================================================== MMA issuers
+    // Two warps issue the MMAs, each running as far ahead as its own barriers
+    // allow: warp 9 the score products S^T = K Q^T, dP^T = V dO^T of every
+    // step (into TMEM once the compute warps have read the previous ones),
+    // warp 11 the gradient products of every step (dV, dK, dQ).  Q and dO of
+    // a step are released once both have read them (qempty counts two
+    // commits).  Each whole warp runs its loop (warp-uniform waits and
+    // descriptors); lane 0 issues each MMA and commit.
+    constexpr uint32_t ID_S = idesc_bf16(128, BM, 0, 0);   // K|V (K-major) x Q|dO (K-major)
+    constexpr uint32_t ID_GV = idesc_bf16(128, HD, 0, 1);  // P^T (TMEM) | dS^T (smem, K-major) x dO|Q (MN-major)
+    constexpr uint32_t ID_Q = C::QLANE ? idesc_bf16(128, HD, 1, 1) : idesc_bf16(128, BM, 1, 1);
+    bool ok = wait_warp<true>(bar_kv, 0, abort, B_KV);
+    if (warp == BWD_WARP_MMA) {
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it % ST;
+        if (!wait_warp<true>(bar_qfull(s), (it / ST) & 1, abort, B_QFULL) ||
+            (it > 0 && !wait_warp<true>(bar_spfree, (it - 1) & 1, abort, B_SPFREE)))
+          break;
+        tc_fence_after();
         // S^T = K Q^T and dP^T = V dO^T (reduction over the features)
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
@@ -248,25 +263,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           mma_ss_w(tmem + C::T_DP, sw128_desc(sV + ko, 16, 1024), sw128_desc(sDO(s) + qo, 16, 1024), ID_S,
                    kk > 0);
         }
-      };
-      bool ok = wait_warp<true>(bar_kv, 0, abort, B_KV) && n_it > 0 &&
-                wait_warp<true>(bar_qfull(0), 0, abort, B_QFULL);
-      if (ok) {
-        tc_fence_after();
-        issue_sdp(0);
         mma_commit_w(bar_spfull);
+        mma_commit_w(bar_qempty(s));  // this warp is done with Q, dO of the step
       }
+    } else {
       for (int it = 0; ok && it < n_it; ++it) {
         const int s = it % ST;
-        // next step's S^T, dP^T as soon as this step's are out of TMEM
-        if (it + 1 < n_it) {
-          if (!wait_warp<true>(bar_qfull((it + 1) % ST), ((it + 1) / ST) & 1, abort, B_QFULL) ||
-              !wait_warp<true>(bar_spfree, it & 1, abort, B_SPFREE))
-            break;
-          tc_fence_after();
-          issue_sdp((it + 1) % ST);
-          mma_commit_w(bar_spfull);
-        }
         if (!wait_warp<true>(bar_pdsfull, it & 1, abort, B_PDSFULL)) break;
         tc_fence_after();
         // dV += P^T dO (A = P^T from TMEM; reduction over the BM query rows)
@@ -282,7 +284,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           mma_ss_w(tmem + C::T_DK, sw128_desc(sDST + po, 16, 1024), sw128_desc(sQ(s) + kk * 2048, C::QSLAB, 1024),
                    ID_GV, (it > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit_w(bar_qempty(s));  // Q, dO of this step are no longer read
+        mma_commit_w(bar_qempty(s));  // this warp is done with Q, dO of the step
         // dQ tile (reduction over the 128 keys) once the previous one has been read
         if (it >= 1 && !wait_warp<true>(bar_dqfree, (it - 1) & 1, abort, B_DQFREE)) break;
         tc_fence_after();
@@ -298,10 +300,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         mma_commit_w(bar_dqfull);
         mma_commit_w(bar_dstfree);
       }
-      mma_commit_w(bar_fin);
-      volatile int never = 0;
-      wait_warp<true>(bar_fin, 0, &never, B_FIN);
     }
+    // Drain: all MMAs issued by this warp complete before TMEM is freed.
+    mma_commit_w(bar_fin);
+    volatile int never = 0;
+    wait_warp<true>(bar_fin, 0, &never, B_FIN);
   } else if (warp == BWD_WARP_RED) {
     if (lane == 0) {
       // ===================================================== dQ tiles -> fp32 accumulator (TMA add)
