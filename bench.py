@@ -165,6 +165,13 @@ def cpu_sample(w, budget_s: float, max_heads: int | None = None):
     return tflops, oracle.max_threads(), desc, t_total
 
 
+def workload_config(w, world: int) -> dict:
+    """The `config` object of the JSON line; the same for both arms."""
+    return {"workload": f"{w.name}: {w.describe()}", "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv,
+            "D": w.D, "global_batch": w.B * world, "parallelism": f"replicas x{world} (no collective)",
+            "l2": "GPU arm: flushed before every step (256 MiB write, outside the timed events)"}
+
+
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return 0
@@ -188,8 +195,7 @@ def run_reference(args, rank: int, world: int):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,sigma^2), bf16-rounded)",
-        "config": {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                   "causal": w.causal, "sample_per_step": "one whole query head (fwd+bwd)"},
+        "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": "one whole query head of the workload per step, fwd+bwd, fp64"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -399,9 +405,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,sigma^2), bf16-rounded; each rank its own batch)",
-            "config": {"workload": f"{w.name}: {w.describe()}", "B": B, "S": S, "Hq": Hq, "Hkv": Hkv,
-                       "D": D, "global_batch": B * world, "parallelism": f"replicas x{world} (no collective)",
-                       "l2": "flushed before every step (256 MiB write, outside the timed events)"},
+            "config": workload_config(w, world),
             "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
             "fwd_frac_of_nominal_2250": fwd_tf / P_NOM_TFLOPS, "bwd_frac_of_nominal_2250": bwd_tf / P_NOM_TFLOPS,
             "fwd_frac_of_measured": fwd_tf / p_meas, "bwd_frac_of_measured": bwd_tf / p_meas,
