@@ -32,7 +32,14 @@ sys.path.insert(0, ROOT)
 P_NOM_TFLOPS = 2250.0  # B200 dense bf16, NVIDIA's published figure
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "attention fwd / bwd TFLOP/s (bf16, causal) and % of B200 tensor peak"
-KERNEL_SOURCES = ("attn_fwd.cuh", "attn_bwd.cuh", "sm100_ptx.cuh", "axis_attn.cu")
+# The sources each kernel is compiled from (its own header, the shared PTX
+# helpers, and the host file with its launch configuration).
+KERNEL_SOURCES = {
+    "attn_fwd_kernel": ("attn_fwd.cuh", "sm100_ptx.cuh", "axis_attn.cu"),
+    "attn_bwd_kernel": ("attn_bwd.cuh", "sm100_ptx.cuh", "axis_attn.cu"),
+    "attn_bwd_prep_kernel": ("attn_bwd.cuh", "axis_attn.cu"),
+    "attn_bwd_dq_convert_kernel": ("attn_bwd.cuh", "axis_attn.cu"),
+}
 
 
 def peaks():
@@ -43,10 +50,15 @@ def peaks():
     return dict(FALLBACK), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str, read=None) -> str:
+    """Hash of the sources `kernel` is built from; `read(name)` returns a
+    source's bytes (default: the working tree)."""
+    if read is None:
+        def read(name):
+            return open(os.path.join(ROOT, "causal_attention_fwd_b200", "csrc", name), "rb").read()
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
-        h.update(open(os.path.join(ROOT, "causal_attention_fwd_b200", "csrc", name), "rb").read())
+    for name in KERNEL_SOURCES[kernel]:
+        h.update(read(name))
     return h.hexdigest()[:16]
 
 
@@ -58,7 +70,7 @@ def profiled_traffic(kernel: str, workload: str):
         return None
     d = json.load(open(p))
     e = d.get(kernel, {})
-    if e.get("workload") == workload and e.get("source_hash") == kernel_source_hash():
+    if e.get("workload") == workload and e.get("source_hash") == kernel_source_hash(kernel):
         return e.get("dram_bytes_per_launch")
     return None
 

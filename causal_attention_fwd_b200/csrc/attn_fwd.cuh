@@ -149,6 +149,32 @@ __device__ __forceinline__ uint64_t exp_pairs(const uint32_t (&v)[32], uint64_t 
   return acc;
 }
 
+// Within each group of N lanes, transpose the N 16-byte chunks every lane
+// holds (chunk k = c[4k .. 4k+3]): afterwards lane g*N + i holds, as its
+// chunk k, chunk i of what lane g*N + k held.  A butterfly over the lane bits
+// (shfl_xor with distance N/2, ..., 1), 2 N log2(N) shuffles per lane.
+template <int N>
+__device__ __forceinline__ void xpose_chunks(uint32_t (&c)[4 * N], int lane) {
+#pragma unroll
+  for (int b = N / 2; b >= 1; b >>= 1) {
+    const bool hi = (lane & b) != 0;
+#pragma unroll
+    for (int k0 = 0; k0 < N; ++k0) {
+      if (k0 & b) continue;
+      const int k1 = k0 | b;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t send = hi ? c[4 * k0 + w] : c[4 * k1 + w];
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, b);
+        if (hi)
+          c[4 * k0 + w] = recv;
+        else
+          c[4 * k1 + w] = recv;
+      }
+    }
+  }
+}
+
 // Warp roles: 0-7 softmax of Q tile 0 (0-3 columns 0-63, 4-7 columns 64-127),
 // 8-15 softmax of Q tile 1, 16 TMA producer of Q and K, 17 S issuer (and TMEM
 // owner), 18 TMA producer of V, 19 P V issuer.  Five warps per SM
@@ -528,26 +554,36 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       if (!wait_warp<true>(bar_o(t), (J - 1) & 1, abort, F_OFIN)) { ok = false; break; }
       tc_fence_after();
       const float inv_l = __fdividef(1.f, l);  // l >= 1: the row max contributes 2^(>= 0)
-      __nv_bfloat16* orow = a.o + (((size_t)I.b * a.S + row_g) * a.Hq + I.h) * HD + hf * (HD / 2);
-#pragma unroll 1
+      // O / l as bf16: this thread's half row is NCK 16-byte chunks
+      constexpr int NCK = HD / 16;
+      uint32_t pk[4 * NCK];
+#pragma unroll
       for (int cc = 0; cc < HD / 64; ++cc) {
         uint32_t v[32];
         tmem_ld32(tO + cc * 32, v);
         tmem_wait_ld();
-        uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l);
-        if (row_g < a.S) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-        }
+          pk[16 * cc + i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l, __uint_as_float(v[2 * i + 1]) * inv_l);
       }
       // O_t is out of TMEM: the next item's first P V may overwrite it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_ofree(t));
+      // Coalesced stores: after the chunk transpose, store k of the warp
+      // writes 32 / NCK whole half rows (NCK consecutive lanes per row)
+      // instead of 32 scattered 16-byte pieces.
+      xpose_chunks<NCK>(pk, lane);
+      const int ck = lane % NCK, rbase = qt * 128 + wq * 32 + (lane / NCK) * NCK;
+#pragma unroll
+      for (int k = 0; k < NCK; ++k) {
+        const int row = rbase + k;
+        if (row < a.S) {
+          uint4* dst =
+              reinterpret_cast<uint4*>(a.o + (((size_t)I.b * a.S + row) * a.Hq + I.h) * HD + hf * (HD / 2)) + ck;
+          *dst = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+      }
       if (hf == 0 && row_g < a.S) a.lse[(size_t)I.bh * a.S + row_g] = (m_used + __log2f(l)) * 0.69314718055994531f;
     }
   }
