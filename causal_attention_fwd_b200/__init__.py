@@ -11,6 +11,8 @@ from .binding import (  # noqa: F401
     attention_backward,
     attention_forward,
     axis_attn_bwd,
+    axis_attn_bwd_det,
+    axis_attn_bwd_det_workspace_bytes,
     axis_attn_bwd_finalize,
     axis_attn_bwd_main,
     axis_attn_bwd_noalloc,

@@ -26,6 +26,8 @@ EXPORTS = (
     "axis_attn_bwd_main",
     "axis_attn_bwd_finalize",
     "axis_attn_bwd_noalloc",
+    "axis_attn_bwd_det_workspace_bytes",
+    "axis_attn_bwd_det",
     "axis_attn_get_status",
     "axis_attn_last_status_word",
     "axis_attn_strerror",
@@ -81,6 +83,10 @@ def load():
             lib.axis_attn_bwd_finalize.restype = i
             lib.axis_attn_bwd_noalloc.argtypes = [vp] * 9 + [i] * 5 + [f, i, vp]
             lib.axis_attn_bwd_noalloc.restype = i
+            lib.axis_attn_bwd_det_workspace_bytes.argtypes = [i] * 5
+            lib.axis_attn_bwd_det_workspace_bytes.restype = sz
+            lib.axis_attn_bwd_det.argtypes = [vp] * 9 + [i] * 5 + [f, i, vp, sz, vp]
+            lib.axis_attn_bwd_det.restype = i
             lib.axis_attn_get_status.argtypes = [vp]
             lib.axis_attn_get_status.restype = i
             lib.axis_attn_last_status_word.argtypes = []
@@ -126,6 +132,18 @@ def axis_attn_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, sca
     for callers that cannot allocate device memory (see include/axis_attn.h)."""
     return load().axis_attn_bwd_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
                                         stream)
+
+
+def axis_attn_bwd_det_workspace_bytes(B, Hq, Hkv, S, D) -> int:
+    return int(load().axis_attn_bwd_det_workspace_bytes(B, Hq, Hkv, S, D))
+
+
+def axis_attn_bwd_det(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
+                      workspace, workspace_bytes, stream) -> int:
+    """Backward whose results are bitwise reproducible run to run (dQ summed over
+    the key tiles in a fixed order; see include/axis_attn.h)."""
+    return load().axis_attn_bwd_det(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
+                                    workspace, workspace_bytes, stream)
 
 
 def axis_attn_get_status(stream) -> int:
@@ -178,23 +196,27 @@ def attention_forward(q, k, v, causal: bool = True, scale: float | None = None, 
 
 
 def attention_backward(q, k, v, o, lse, dout, causal: bool = True, scale: float | None = None,
-                       workspace=None, grads=None, stream=None):
-    """dQ, dK, dV (bf16) of sum(dO * O)."""
+                       workspace=None, grads=None, stream=None, deterministic: bool = False):
+    """dQ, dK, dV (bf16) of sum(dO * O).  deterministic=True: axis_attn_bwd_det
+    (bitwise reproducible, larger workspace)."""
     import torch
 
     B, Hq, Hkv, S, D = _dims(q, k)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    need = axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D)
+    size_fn, call, name = ((axis_attn_bwd_det_workspace_bytes, axis_attn_bwd_det, "axis_attn_bwd_det")
+                           if deterministic else
+                           (axis_attn_bwd_workspace_bytes, axis_attn_bwd, "axis_attn_bwd"))
+    need = size_fn(B, Hq, Hkv, S, D)
     if workspace is None:
         workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k),
                                                   torch.empty_like(v))
-    rc = axis_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
-                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                       B, Hq, Hkv, S, D, scale, int(causal), workspace.data_ptr(),
-                       workspace.numel() * workspace.element_size(), _stream(stream))
+    rc = call(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+              lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+              B, Hq, Hkv, S, D, scale, int(causal), workspace.data_ptr(),
+              workspace.numel() * workspace.element_size(), _stream(stream))
     if rc:
-        raise AxisAttnError(rc, "axis_attn_bwd")
+        raise AxisAttnError(rc, name)
     return dq, dk, dv
 
 

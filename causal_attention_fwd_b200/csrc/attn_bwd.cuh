@@ -41,6 +41,7 @@ struct BwdArgs {
   float* dqacc;        // [B*Hq][S][HD]  fp32, pre-scaled by `scale`
   int B, Hq, Hkv, S, S_pad;
   float scale, scale_log2;
+  int det;             // 1: store each key tile's dQ tile into its own slice (deterministic mode)
 };
 
 template <int HD>
@@ -318,7 +319,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           // D = 64: box (feature block bx & 1, row block bx >> 1); D = 128: feature block bx
           const int c0 = C::QLANE ? 32 * (bx & 1) : 32 * bx;
           const int r0 = C::QLANE ? q0 + 64 * (bx >> 1) : q0;
-          if (r0 < a.S) tma_reduce_add_3d(&tm_dq, sSTG + bx * C::DQ_BOX, c0, r0, bh);
+          if (r0 >= a.S) continue;
+          if (a.det)  // slice of key tile j: [j][b*Hq + h][S][HD]
+            tma_store_3d(&tm_dq, sSTG + bx * C::DQ_BOX, c0, r0, bh + a.B * a.Hq * j);
+          else
+            tma_reduce_add_3d(&tm_dq, sSTG + bx * C::DQ_BOX, c0, r0, bh);
         }
         bulk_commit();
         bulk_wait_read0();
@@ -564,6 +569,41 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
     out.z = pack_bf16x2(y.x, y.y);
     out.w = pack_bf16x2(y.z, y.w);
     reinterpret_cast<uint4*>(dq + row * HD)[c8] = out;
+  }
+}
+
+// Deterministic mode: dq[b,i,h,:] = bf16(sum over key tiles j of the slices
+// part[j][b*Hq+h][i][:]), added in the order j = 0, 1, ... (only the tiles row
+// i sees when causal: j <= i / 128, the ones whose CTA wrote a tile for i).
+// 8 features per thread, slices read row-contiguously.
+template <int HD>
+__global__ void __launch_bounds__(256) attn_bwd_dq_sum_kernel(const float* __restrict__ part,
+                                                              __nv_bfloat16* __restrict__ dq, int Hq, int S,
+                                                              int nkv, int causal, size_t n8) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  const size_t slice = n8 * 8;  // floats per key-tile slice: B * Hq * S * HD
+  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < n8; k += stride) {
+    const int c8 = (int)(k % (HD / 8));
+    const size_t bi_row = k / (HD / 8);  // (b*Hq + h) * S + i
+    const int i = (int)(bi_row % S);
+    const size_t bh = bi_row / S;
+    const int h = (int)(bh % Hq);
+    const size_t b = bh / Hq;
+    const int last = causal ? i / 128 : nkv - 1;
+    const float* src = part + bi_row * HD + 8 * c8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j <= last; ++j) {
+      const float4 x = reinterpret_cast<const float4*>(src + (size_t)j * slice)[0];
+      const float4 y = reinterpret_cast<const float4*>(src + (size_t)j * slice)[1];
+      acc[0] += x.x; acc[1] += x.y; acc[2] += x.z; acc[3] += x.w;
+      acc[4] += y.x; acc[5] += y.y; acc[6] += y.z; acc[7] += y.w;
+    }
+    uint4 out;
+    out.x = pack_bf16x2(acc[0], acc[1]);
+    out.y = pack_bf16x2(acc[2], acc[3]);
+    out.z = pack_bf16x2(acc[4], acc[5]);
+    out.w = pack_bf16x2(acc[6], acc[7]);
+    reinterpret_cast<uint4*>(dq + ((b * S + i) * Hq + h) * HD)[c8] = out;
   }
 }
 

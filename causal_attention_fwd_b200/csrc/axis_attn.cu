@@ -95,14 +95,17 @@ struct WsLayout {
   int S_pad;
 };
 
-WsLayout ws_layout(int B, int Hq, int S, int D) {
+// det: one fp32 dQ slice per 128-key tile ([nkv][B*Hq][S][D]) instead of one
+// shared accumulator.
+WsLayout ws_layout(int B, int Hq, int S, int D, bool det = false) {
   WsLayout w;
   w.S_pad = (S + 127) / 128 * 128;
   const size_t rows = (size_t)B * Hq * w.S_pad;
+  const size_t slices = det ? (size_t)((S + 127) / 128) : 1;
   w.lse2 = 0;
   w.dr = round256(rows * 4);
   w.dqacc = w.dr + round256(rows * 4);
-  w.total = w.dqacc + round256((size_t)B * Hq * S * D * 4);
+  w.total = w.dqacc + round256(slices * B * Hq * S * D * 4);
   return w;
 }
 
@@ -211,22 +214,17 @@ WsPtrs ws_ptrs(void* workspace, const WsLayout& w) {
 
 }  // namespace
 
-extern "C" int axis_attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, int Hkv,
-                                     int S, int D, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!o || !dO || !lse) return AXIS_ATTN_ERR_NULL;
-  if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return AXIS_ATTN_ERR_ALIGN;
-  if (int rc = check_shape(B, Hq, Hkv, S, D, 1.f)) return rc;
-  const WsLayout w = ws_layout(B, Hq, S, D);
-  if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
-  int dev = 0;
-  if (int rc = check_device(&dev)) return rc;
-  const WsPtrs p = ws_ptrs(workspace, w);
+namespace {
+
+// Stage 1: -Dr and -LSE*log2(e) rows (padding rows 0 / -inf); zero the dQ
+// accumulator unless the deterministic mode's slices are used.
+int run_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, int S, int D, const WsLayout& w,
+                const WsPtrs& p, bool zero_dq, cudaStream_t st) {
   const int rows = B * Hq * w.S_pad;
-  const size_t dq_vec4 = (size_t)B * Hq * S * D / 4;
+  const size_t dq_vec4 = zero_dq ? (size_t)B * Hq * S * D / 4 : 0;
   // grid-stride kernel: a few waves of 256-thread blocks over the 148 SMs
   const size_t work = (size_t)B * Hq * S * (D / 8);
   const unsigned grid = (unsigned)((work + 255) / 256 < 148 * 16 ? (work + 255) / 256 : 148 * 16);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const auto* ob = static_cast<const __nv_bfloat16*>(o);
   const auto* db = static_cast<const __nv_bfloat16*>(dO);
   if (D == 64)
@@ -238,25 +236,18 @@ extern "C" int axis_attn_bwd_prepare(const void* o, const void* dO, const float*
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
-extern "C" int axis_attn_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
-                                  int B, int Hq, int Hkv, int S, int D, float scale, int causal, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
-  if (!q || !k || !v || !dO || !dk || !dv) return AXIS_ATTN_ERR_NULL;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv))
-    return AXIS_ATTN_ERR_ALIGN;
-  if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
-  const WsLayout w = ws_layout(B, Hq, S, D);
-  if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
-  int dev = 0;
-  if (int rc = check_device(&dev)) return rc;
+// Stage 2: the main kernel; det stores each key tile's dQ tiles into its slice.
+int run_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int Hq,
+             int Hkv, int S, int D, float scale, int causal, const WsLayout& w, const WsPtrs& p, bool det,
+             cudaStream_t st, int dev) {
   const int BM = D == 64 ? BwdCfg<64>::BM : BwdCfg<128>::BM;
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, q, B, S, Hq, D, BM) || !make_map(&mdo, dO, B, S, Hq, D, BM) ||
       !make_map(&mk, k, B, S, Hkv, D, 128) || !make_map(&mv, v, B, S, Hkv, D, 128))
     return AXIS_ATTN_ERR_CUDA;
-  const WsPtrs p = ws_ptrs(workspace, w);
+  const int nkv = (S + 127) / 128;
   CUtensorMap mdq;
-  if (!make_dq_map(&mdq, p.dqacc, B * Hq, S, D)) return AXIS_ATTN_ERR_CUDA;
+  if (!make_dq_map(&mdq, p.dqacc, B * Hq * (det ? nkv : 1), S, D)) return AXIS_ATTN_ERR_CUDA;
   BwdArgs a;
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
@@ -270,12 +261,60 @@ extern "C" int axis_attn_bwd_main(const void* q, const void* k, const void* v, c
   a.S_pad = w.S_pad;
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  a.det = det ? 1 : 0;
   if (D == 64)
     return causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, mdq, a, st, dev)
                   : launch_bwd_main<64, false>(mq, mk, mv, mdo, mdq, a, st, dev);
   return causal ? launch_bwd_main<128, true>(mq, mk, mv, mdo, mdq, a, st, dev)
                 : launch_bwd_main<128, false>(mq, mk, mv, mdo, mdq, a, st, dev);
+}
+
+// Stage 3: dQ to bf16 [B,S,Hq,D] (det: the key-tile slices summed in order).
+int run_finalize(void* dq, int B, int Hq, int S, int D, int causal, const WsPtrs& p, bool det, cudaStream_t st) {
+  const size_t n8 = (size_t)B * S * Hq * D / 8;
+  const unsigned grid = (unsigned)((n8 + 255) / 256 < 4096 ? (n8 + 255) / 256 : 4096);
+  auto* out = static_cast<__nv_bfloat16*>(dq);
+  const int nkv = (S + 127) / 128;
+  if (det) {
+    if (D == 64)
+      attn_bwd_dq_sum_kernel<64><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, nkv, causal, n8);
+    else
+      attn_bwd_dq_sum_kernel<128><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, nkv, causal, n8);
+  } else if (D == 64) {
+    attn_bwd_dq_convert_kernel<64><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, n8);
+  } else {
+    attn_bwd_dq_convert_kernel<128><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, n8);
+  }
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int axis_attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, int Hkv,
+                                     int S, int D, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!o || !dO || !lse) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return AXIS_ATTN_ERR_ALIGN;
+  if (int rc = check_shape(B, Hq, Hkv, S, D, 1.f)) return rc;
+  const WsLayout w = ws_layout(B, Hq, S, D);
+  if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  return run_prepare(o, dO, lse, B, Hq, S, D, w, ws_ptrs(workspace, w), true, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int axis_attn_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                                  int B, int Hq, int Hkv, int S, int D, float scale, int causal, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !dO || !dk || !dv) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv))
+    return AXIS_ATTN_ERR_ALIGN;
+  if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
+  const WsLayout w = ws_layout(B, Hq, S, D);
+  if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  return run_main(q, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, w, ws_ptrs(workspace, w), false,
+                  static_cast<cudaStream_t>(stream), dev);
 }
 
 extern "C" int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, int D, void* workspace,
@@ -287,34 +326,51 @@ extern "C" int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, i
   if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
-  const WsPtrs p = ws_ptrs(workspace, w);
-  const size_t n8 = (size_t)B * S * Hq * D / 8;
-  const unsigned grid = (unsigned)((n8 + 255) / 256 < 4096 ? (n8 + 255) / 256 : 4096);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 64)
-    attn_bwd_dq_convert_kernel<64><<<grid, 256, 0, st>>>(p.dqacc, static_cast<__nv_bfloat16*>(dq), Hq, S, n8);
-  else
-    attn_bwd_dq_convert_kernel<128><<<grid, 256, 0, st>>>(p.dqacc, static_cast<__nv_bfloat16*>(dq), Hq, S, n8);
-  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+  return run_finalize(dq, B, Hq, S, D, 1, ws_ptrs(workspace, w), false, static_cast<cudaStream_t>(stream));
 }
 
-extern "C" int axis_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
-                             const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D,
-                             float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+
+int run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
+            void* dk, void* dv, int B, int Hq, int Hkv, int S, int D, float scale, int causal, void* workspace,
+            size_t workspace_bytes, void* stream, bool det) {
   // Validate everything first so that no stage runs when a later one would fail.
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return AXIS_ATTN_ERR_NULL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(lse) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return AXIS_ATTN_ERR_ALIGN;
   if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
-  if (int rc = check_ws(workspace, workspace_bytes, ws_layout(B, Hq, S, D))) return rc;
+  const WsLayout w = ws_layout(B, Hq, S, D, det);
+  if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
-  if (int rc = axis_attn_bwd_prepare(o, dO, lse, B, Hq, Hkv, S, D, workspace, workspace_bytes, stream)) return rc;
-  if (int rc = axis_attn_bwd_main(q, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, workspace,
-                                  workspace_bytes, stream))
-    return rc;
-  return axis_attn_bwd_finalize(dq, B, Hq, Hkv, S, D, workspace, workspace_bytes, stream);
+  const WsPtrs p = ws_ptrs(workspace, w);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (int rc = run_prepare(o, dO, lse, B, Hq, S, D, w, p, !det, st)) return rc;
+  if (int rc = run_main(q, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, w, p, det, st, dev)) return rc;
+  return run_finalize(dq, B, Hq, S, D, causal, p, det, st);
+}
+
+}  // namespace
+
+extern "C" int axis_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                             const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S, int D,
+                             float scale, int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  return run_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, workspace, workspace_bytes,
+                 stream, false);
+}
+
+extern "C" size_t axis_attn_bwd_det_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
+  if (check_shape(B, Hq, Hkv, S, D, 1.f) != AXIS_ATTN_OK) return 0;
+  return ws_layout(B, Hq, S, D, true).total;
+}
+
+extern "C" int axis_attn_bwd_det(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                 const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S,
+                                 int D, float scale, int causal, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  return run_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, workspace, workspace_bytes,
+                 stream, true);
 }
 
 // ----------------------------------------------------------------------------

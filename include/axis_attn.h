@@ -113,6 +113,35 @@ int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, int D, void*
                            size_t workspace_bytes, void* stream);
 
 /*
+ * Deterministic backward: the gradients of axis_attn_bwd(), bitwise the same
+ * from run to run on the same device and inputs.  The Axis page
+ * (zyoralabs.com/axis, list of published checks) reports multi-GPU weights
+ * bit-identical to replicated data parallel, and the axis repository page
+ * (its table of claims, "The run can be reproduced") ties reproducibility to
+ * the training step; with the ordinary backward, dQ is the one output whose
+ * fp32 additions happen in a run-dependent order.
+ *
+ * How: every 128-key tile writes its dQ contribution into its own fp32 slice
+ * of the workspace, and the last stage adds the slices of each row in the
+ * fixed order of the key tiles.  dk and dv take no cross-tile additions in
+ * either mode.  Results agree with axis_attn_bwd() to rounding (the same
+ * products, summed in another order).
+ *
+ * Arguments, layouts, ownership and errors as for axis_attn_bwd(), with a
+ * larger workspace:
+ *   axis_attn_bwd_det_workspace_bytes() = the row statistics of
+ *   axis_attn_bwd() + 4 * ceil(S / 128) * B * Hq * S * D bytes
+ * (about 1.07 GB for B=4, Hq=32, S=2048, D=64; it grows as S^2).  A workspace
+ * shorter than that returns AXIS_ATTN_ERR_WORKSPACE and launches nothing.
+ * Returns 0 from the size function for invalid sizes.
+ */
+size_t axis_attn_bwd_det_workspace_bytes(int B, int Hq, int Hkv, int S, int D);
+int axis_attn_bwd_det(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                      const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int S,
+                      int D, float scale, int causal, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
  * Backward for callers that cannot allocate device memory: same arguments,
  * results and errors as axis_attn_bwd(), minus the workspace.  (No counterpart
  * on the pages: this is a packaging variant of the backward, not a different

@@ -57,6 +57,20 @@ def test_workspace_bytes(lib):
     assert aa.axis_attn_bwd_workspace_bytes(1, 1, 1, 0, 64) == 0        # empty sequence
 
 
+def test_det_workspace_bytes(lib):
+    # the same row sections + one fp32 dQ slice per 128-key tile
+    B, Hq, Hkv, S, D = 2, 12, 4, 1000, 64
+    rows = B * Hq * 1024
+    r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    nkv = (S + 127) // 128
+    assert aa.axis_attn_bwd_det_workspace_bytes(B, Hq, Hkv, S, D) == 2 * r256(rows * 4) + r256(
+        nkv * B * Hq * S * D * 4)
+    # the header's example: B=4, Hq=32, S=2048, D=64 needs about 1.07 GB
+    assert abs(aa.axis_attn_bwd_det_workspace_bytes(4, 32, 8, 2048, 64) / 1.07e9 - 1) < 0.01
+    assert aa.axis_attn_bwd_det_workspace_bytes(1, 3, 2, 128, 64) == 0
+    assert aa.axis_attn_bwd_det_workspace_bytes(1, 1, 1, 128, 96) == 0
+
+
 A = 1 << 20  # a fake, 16-byte aligned "device" address; never dereferenced
 
 
@@ -95,6 +109,22 @@ def test_fwd_rejects(lib, over, code):
 ])
 def test_bwd_rejects(lib, over, code):
     assert _bwd(**over) == code
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(dO=None), 1), (dict(dq=None), 1), (dict(dk=A + 8), 2), (dict(S=0), 3), (dict(D=80), 4),
+    (dict(workspace=None), 5), (dict(workspace=A + 16), 5),
+    # enough for axis_attn_bwd (about 0.5 MB here) but not for the key-tile slices (about 4.1 MB)
+    (dict(S=1000, workspace_bytes=3 << 20), 5),
+])
+def test_bwd_det_rejects(lib, over, code):
+    args = dict(q=A, k=A, v=A, o=A, dO=A, lse=A, dq=A, dk=A, dv=A, B=1, Hq=2, Hkv=1, S=128, D=64,
+                scale=0.125, causal=1, workspace=A, workspace_bytes=1 << 30, stream=None)
+    args.update(over)
+    if "S" in over and over["S"] == 1000:
+        assert aa.axis_attn_bwd_workspace_bytes(1, 2, 1, 1000, 64) < args["workspace_bytes"]
+        assert aa.axis_attn_bwd_det_workspace_bytes(1, 2, 1, 1000, 64) > args["workspace_bytes"]
+    assert aa.axis_attn_bwd_det(*args.values()) == code
 
 
 def test_torch_helpers_raise_without_valid_args(lib):
