@@ -253,6 +253,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time the bitwise-reproducible backward (axis_attn_bwd_det) instead")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -283,7 +285,8 @@ def main():
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, S), device=dev, dtype=torch.float32)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws_bytes = aa.axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D)
+    det = args.deterministic
+    ws_bytes = (aa.axis_attn_bwd_det_workspace_bytes if det else aa.axis_attn_bwd_workspace_bytes)(B, Hq, Hkv, S, D)
     ws = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
     flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream(dev)
@@ -301,6 +304,16 @@ def main():
                                B, Hq, Hkv, S, D, w.scale, causal, sp), "fwd")
         if ev:
             ev[1].record(stream)
+        if det:  # one call, three kernels: timed as a whole (the stage events coincide)
+            if ev:
+                ev[2].record(stream)
+                ev[3].record(stream)
+            check(aa.axis_attn_bwd_det(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv,
+                                       S, D, w.scale, causal, ws.data_ptr(), ws_bytes, sp), "bwd_det")
+            if ev:
+                ev[4].record(stream)
+            return
         check(aa.axis_attn_bwd_prepare(o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, Hq, Hkv, S, D,
                                        ws.data_ptr(), ws_bytes, sp), "bwd_prepare")
         if ev:
@@ -349,6 +362,8 @@ def main():
     flops_step = w.fwd_flops + w.bwd_flops
     value = whole_job_tflops(flops_step, K, total_ms, world)
     names = ["attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_kernel", "attn_bwd_dq_convert_kernel"]
+    if det:
+        names = ["attn_fwd_kernel", "-", "-", "axis_attn_bwd_det (prep + main + dq_sum)"]
     avg_ms = [float(totals[i]) / K for i in range(4)]
     fwd_tf = w.fwd_flops / (avg_ms[0] * 1e-3) / 1e12
     bwd_ms = sum(avg_ms[1:])
@@ -360,7 +375,7 @@ def main():
     dom = max(range(4), key=lambda i: avg_ms[i])
     dom_flops = w.fwd_flops if dom == 0 else w.bwd_flops
     roof = None
-    if dom in (0, 2):
+    if dom in (0, 2) or (det and dom == 3):
         achieved = dom_flops / (avg_ms[dom] * 1e-3) / 1e12
         roof = {"kernel": names[dom], "bound": "tensor", "achieved": achieved, "peak": p_meas,
                 "peak_source": f"{pk_src} bf16_tflops (burst)", "unit": "TFLOP/s",
@@ -382,7 +397,7 @@ def main():
                 dst.copy_(src, non_blocking=True)
             oo, ll = aa.attention_forward(qq, kk, vv, causal=w.causal, scale=w.scale, out=o, lse=lse)
             g = aa.attention_backward(qq, kk, vv, oo, ll, dd, causal=w.causal, scale=w.scale, workspace=ws,
-                                      grads=(dq, dk, dv))
+                                      grads=(dq, dk, dv), deterministic=det)
             for dst, src in ((ho, oo), (hl, ll), (hdq, g[0]), (hdk, g[1]), (hdv, g[2])):
                 dst.copy_(src, non_blocking=True)
 
@@ -421,7 +436,8 @@ def main():
             "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
             "fwd_frac_of_nominal_2250": fwd_tf / P_NOM_TFLOPS, "bwd_frac_of_nominal_2250": bwd_tf / P_NOM_TFLOPS,
             "fwd_frac_of_measured": fwd_tf / p_meas, "bwd_frac_of_measured": bwd_tf / p_meas,
-            "kernel_ms": dict(zip(names, avg_ms)),
+            "kernel_ms": {n: t for n, t in zip(names, avg_ms) if n != "-"},
+            "bwd_mode": "deterministic (axis_attn_bwd_det)" if det else "ordinary (axis_attn_bwd stages)",
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": 4 * K, "clocks": clocks,
         }
