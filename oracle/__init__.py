@@ -12,4 +12,5 @@ from .oracle import (  # noqa: F401
     build,
     max_threads,
     probs_row,
+    rope,
 )

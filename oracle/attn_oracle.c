@@ -373,6 +373,38 @@ int oracle_attn_bwd_dkdv_rows(const double* q, const double* k, const double* v,
     return 0;
 }
 
+/*
+ * Rotary position embedding, the step the axiomlm models apply to Q and K
+ * before attention: axiomlm (PyPI), Key Features ("Rotary Position Embeddings
+ * (RoPE)") and Quick Start section 8 (precompute_rope_frequencies(dim, end),
+ * then apply_rope(q, k, freqs_cis)).  The page names the calls, not the
+ * formula; the reading taken is the complex-pair form that the name freqs_cis
+ * points to: in a row at sequence position s, the pair (x[2p], x[2p+1]) is
+ * turned by the angle s * base^(-2p/D) -- the complex number x[2p] + i x[2p+1]
+ * times exp(i s base^(-2p/D)).  base is the caller's (the page gives none;
+ * 10000 is the usual value).  inverse != 0 turns by minus the angle: the
+ * transpose of the rotation, which carries dQ, dK back through it.
+ * x is [B, S, H, D] (D even), rotated in place.  Returns 0, or -1 for bad sizes.
+ */
+int oracle_rope(double* x, int B, int S, int H, int D, double base, int inverse) {
+    if (B < 1 || S < 1 || H < 1 || D < 2 || (D & 1) || !(base > 0.0)) return -1;
+    const double sgn = inverse ? -1.0 : 1.0;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int s = 0; s < S; ++s)
+            for (int h = 0; h < H; ++h) {
+                double* row = x + (((size_t)b * S + s) * H + h) * D;
+                for (int p = 0; p < D / 2; ++p) {
+                    const double ang = sgn * (double)s * pow(base, -2.0 * p / D);
+                    const double c = cos(ang), sn = sin(ang);
+                    const double x0 = row[2 * p], x1 = row[2 * p + 1];
+                    row[2 * p] = x0 * c - x1 * sn;
+                    row[2 * p + 1] = x0 * sn + x1 * c;
+                }
+            }
+    return 0;
+}
+
 /* Threads OpenMP will use (1 when built without OpenMP). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

@@ -83,14 +83,24 @@ class Oracle:
         lib.oracle_attn_bwd.argtypes = [_dp] * 8 + dims
         lib.oracle_attn_bwd_dq_rows.argtypes = [_dp] * 4 + dims + [i, _ip, _dp, _dp]
         lib.oracle_attn_bwd_dkdv_rows.argtypes = [_dp] * 4 + dims + [i, _ip, _dp, _dp]
+        lib.oracle_rope.argtypes = [_dp, i, i, i, i, d, i]
         for f in ("oracle_attn_fwd", "oracle_attn_fwd_rows", "oracle_attn_probs_row",
                   "oracle_attn_bwd", "oracle_attn_bwd_dq_rows", "oracle_attn_bwd_dkdv_rows",
-                  "oracle_max_threads"):
+                  "oracle_rope", "oracle_max_threads"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
 
     def max_threads(self) -> int:
         return int(self.lib.oracle_max_threads())
+
+    def rope(self, x, base: float = 10000.0, inverse: bool = False):
+        """Rotary position embedding of x [B, S, H, D] (a rotated float64 copy);
+        inverse=True applies the transposed rotation (for gradients)."""
+        y = _f64(x).copy()
+        B, S, H, D = y.shape
+        if self.lib.oracle_rope(_ptr(y), B, S, H, D, float(base), int(bool(inverse))):
+            raise ValueError("oracle_rope rejected the arguments")
+        return y
 
     def attn_fwd(self, q, k, v, scale: float, causal: bool = True):
         """Full forward.  Returns (O [B,S,Hq,D], LSE [B,Hq,S]), float64."""
@@ -195,3 +205,4 @@ attn_fwd_rows = _forward("attn_fwd_rows")
 probs_row = _forward("probs_row")
 attn_bwd_dq_rows = _forward("attn_bwd_dq_rows")
 attn_bwd_dkdv_rows = _forward("attn_bwd_dkdv_rows")
+rope = _forward("rope")
