@@ -21,9 +21,10 @@
 //       dV += P^T dO (A from TMEM), dK += dS^T Q, and dQ of the tile,
 //     the compute warps copy each dQ tile from TMEM into a swizzled
 //     shared-memory staging tile, which one thread adds into the fp32
-//     accumulator with TMA reduce-add copies; dK, dV stay in TMEM until the
-//     end;
-//   * dQ finalize (HBM-bound): bf16 copy of the accumulator in [B,S,Hq,D].
+//     accumulator with TMA reduce-add copies (deterministic mode: TMA stores
+//     into a slice of this key tile's own); dK, dV stay in TMEM until the end;
+//   * dQ finalize (HBM-bound): bf16 copy of the accumulator in [B,S,Hq,D]
+//     (deterministic mode: the key tiles' slices added in key-tile order).
 // D = 64 uses 128-row query tiles and dQ = dS K (TMEM lane = query row);
 // D = 128 uses 64-row query tiles (shared memory) and dQ^T = K^T dS^T (TMEM
 // lane = feature), so every MMA has M = 128.
@@ -38,7 +39,7 @@ struct BwdArgs {
   __nv_bfloat16* dv;
   const float* nlse2;  // [B*Hq][S_pad]  -LSE * log2(e); -inf on padding rows
   const float* ndr;    // [B*Hq][S_pad]  -rowsum(dO * O); 0 on padding rows
-  float* dqacc;        // [B*Hq][S][HD]  fp32, pre-scaled by `scale`
+  float* dqacc;        // [B*Hq][S][HD] fp32, pre-scaled by `scale` (det: [nkv][B*Hq][S][HD] slices)
   int B, Hq, Hkv, S, S_pad;
   float scale, scale_log2;
   int det;             // 1: store each key tile's dQ tile into its own slice (deterministic mode)
@@ -84,7 +85,8 @@ struct BwdCfg {
 // Warps 0-7: P^T / dS^T (thread = key row, half the query columns each) and
 // the dQ tile of the previous step into the staging tile; warp 8 loads; warp 9
 // issues the score MMAs and owns TMEM; warp 10 issues the TMA reduce-adds of
-// the dQ tiles into the fp32 accumulator; warp 11 issues the gradient MMAs.
+// the dQ tiles into the fp32 accumulator (or their stores into this key tile's
+// slice); warp 11 issues the gradient MMAs.
 // 384 threads: up to 168 registers each.
 constexpr int BWD_THREADS = 384;
 constexpr int BWD_WARP_LOAD = 8;
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     wait_warp<true>(bar_fin, 0, &never, B_FIN);
   } else if (warp == BWD_WARP_RED) {
     if (lane == 0) {
-      // ===================================================== dQ tiles -> fp32 accumulator (TMA add)
+      // ===================================================== dQ tiles -> fp32 accumulator (TMA add or store)
       tma_prefetch_desc(&tm_dq);
       for (int t = 0; t < n_it; ++t) {
         if (!mbar_wait_bounded(bar_stgfull, t & 1, abort, B_STGFULL)) break;
