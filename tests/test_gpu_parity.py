@@ -36,6 +36,10 @@ FUZZ = [
     (2, 2, 1, 1000, 128, False),
     (1, 16, 2, 513, 64, False),
     (1, 4, 2, 777, 128, True),
+    # more work items than SMs: every CTA of the persistent forward walks several
+    # items, some without a second query tile (S = 300: rows 256-299 are one tile)
+    (8, 40, 8, 300, 64, True),
+    (4, 40, 5, 300, 128, False),
 ]
 
 
