@@ -8,11 +8,14 @@ FLOPs counted as half of dense (fwd 2*B*Hq*S^2*D, bwd 5*B*Hq*S^2*D).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
         python bench.py --impl reference ...   (the fp64 CPU oracle, host cores)
-Under torchrun (N > 1) every rank runs its own batch of the workload (weak
-scaling; no collective on the data path).  Timing: CUDA events around each
-step on the launching stream, L2 flushed (256 MiB write) before every step,
-outside the events; the reported time is the max over ranks.  Rank 0 prints one
-JSON line.
+The headline workload (default llm1b, B=4 S=2048 Hq=32 Hkv=8 D=64) gives the
+line's value, roofline, e2e and cpu_baseline; the other four workloads are
+timed after it the same way (fewer steps) and reported under "workloads", each
+with its own clocks and oracle baseline.  Under torchrun (N > 1) every rank
+runs its own batch of each workload (weak scaling; no collective on the data
+path).  Timing: CUDA events around each step on the launching stream, L2
+flushed (256 MiB write) before every step, outside the events; the reported
+time is the max over ranks.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -148,32 +151,64 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------- reference arm
+def oracle_head_seconds(w) -> float:
+    """Rough time of the oracle on one whole query head (fwd + bwd): it was
+    measured at 0.4 s for S = 2048, D = 64 and grows as S^2 D."""
+    return 0.4 * (w.S / 2048.0) ** 2 * (w.D / 64.0)
+
+
 def cpu_sample(w, budget_s: float, max_heads: int | None = None):
-    """The oracle, as it stands, on whole query heads of the workload (each with
-    its kv head), until `budget_s` of CPU time has passed.  Returns TFLOP/s
-    counted like the GPU metric, the threads used and a description."""
+    """The oracle, as it stands, on a bounded sample of the workload.  Returns
+    TFLOP/s counted like the GPU metric, the threads used, a description and
+    the seconds spent.
+
+    Whole query heads (each with its kv head, fwd + bwd) while one head fits
+    the budget; otherwise (the longest sequences) sampled query rows through
+    the oracle's row functions -- the forward rows and the dQ rows, which
+    repeat the full backward's per-row work except its dK/dV accumulation --
+    extrapolated to all B*Hq*S rows (so the figure overstates the oracle's
+    throughput a little)."""
+    import numpy as np
+
     import oracle
     from causal_attention_fwd_b200.synthetic import workload_inputs
 
     q, k, v, do = workload_inputs(w)
     G = w.Hq // w.Hkv
-    per_head = (w.fwd_flops + w.bwd_flops) / (w.B * w.Hq)
-    done, t_total, heads = 0, 0.0, []
-    n = 0
-    while n == 0 or (t_total < budget_s and (max_heads is None or n < max_heads)):
-        b, h = n % w.B, (n // w.B) % w.Hq
-        sl = lambda t, hh: t[b:b + 1, :, hh:hh + 1].contiguous()  # noqa: E731
-        qs, ks, vs, dos = sl(q, h), sl(k, h // G), sl(v, h // G), sl(do, h)
+    flops = w.fwd_flops + w.bwd_flops
+    if oracle_head_seconds(w) <= budget_s or max_heads is not None:
+        per_head = flops / (w.B * w.Hq)
+        done, t_total, n = 0, 0.0, 0
+        while n == 0 or (t_total < budget_s and (max_heads is None or n < max_heads)):
+            b, h = n % w.B, (n // w.B) % w.Hq
+            sl = lambda t, hh: t[b:b + 1, :, hh:hh + 1].contiguous()  # noqa: E731
+            qs, ks, vs, dos = sl(q, h), sl(k, h // G), sl(v, h // G), sl(do, h)
+            t0 = time.perf_counter()
+            oracle.attn_fwd(qs, ks, vs, w.scale, w.causal)
+            oracle.attn_bwd(qs, ks, vs, dos, w.scale, w.causal)
+            t_total += time.perf_counter() - t0
+            done += 1
+            n += 1
+        tflops = done * per_head / t_total / 1e12
+        desc = (f"{done} whole query head(s) of the workload, each fwd+bwd with its kv head "
+                f"(B=1 Hq=1 Hkv=1 S={w.S} D={w.D}); {t_total:.1f} s; the forward runs on all threads, "
+                f"the backward of one (b, kv) unit on one")
+        return tflops, oracle.max_threads(), desc, t_total
+    g = np.random.default_rng(99)
+    rows_total = w.B * w.Hq * w.S
+    done, t_total, R = 0, 0.0, 64
+    while t_total < budget_s / 2:
+        rows = [(int(g.integers(w.B)), int(g.integers(w.Hq)), int(g.integers(w.S))) for _ in range(R)]
         t0 = time.perf_counter()
-        oracle.attn_fwd(qs, ks, vs, w.scale, w.causal)
-        oracle.attn_bwd(qs, ks, vs, dos, w.scale, w.causal)
+        oracle.attn_fwd_rows(q, k, v, w.scale, w.causal, rows)
+        oracle.attn_bwd_dq_rows(q, k, v, do, w.scale, w.causal, rows)
         t_total += time.perf_counter() - t0
-        done += 1
-        heads.append((b, h))
-        n += 1
-    tflops = done * per_head / t_total / 1e12
-    desc = (f"{done} whole query head(s) of the workload, each fwd+bwd with its kv head "
-            f"(B=1 Hq=1 Hkv=1 S={w.S} D={w.D}); {t_total:.1f} s")
+        done += R
+        R *= 2
+    est = t_total / done * rows_total
+    tflops = flops / est / 1e12
+    desc = (f"extrapolated: {done} sampled query rows through the oracle's forward-row and dQ-row functions "
+            f"({t_total:.1f} s), scaled to all {rows_total} rows (a full run would take ~{est:.0f} s)")
     return tflops, oracle.max_threads(), desc, t_total
 
 
@@ -243,6 +278,134 @@ def whole_job_tflops(flops_per_step_per_rank: float, steps: int, max_ms: float, 
 
 
 # ---------------------------------------------------------------- GPU arm
+STAGES = ["attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_kernel", "attn_bwd_dq_convert_kernel"]
+
+
+class Problem:
+    """Device buffers of one workload and its step through the C ABI."""
+
+    def __init__(self, aa, w, seed: int, dev, det: bool, host=None):
+        import ctypes
+
+        import torch
+
+        from causal_attention_fwd_b200.synthetic import workload_inputs
+
+        self.aa, self.w, self.det = aa, w, det
+        self.host = workload_inputs(w, seed=seed) if host is None else host
+        self.q, self.k, self.v, self.do = (t.to(dev) for t in self.host)
+        B, Hq, S = w.B, w.Hq, w.S
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((B, Hq, S), device=dev, dtype=torch.float32)
+        self.dq, self.dk, self.dv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
+        size_fn = aa.axis_attn_bwd_det_workspace_bytes if det else aa.axis_attn_bwd_workspace_bytes
+        self.ws_bytes = size_fn(B, Hq, w.Hkv, S, w.D)
+        self.ws = torch.empty(self.ws_bytes, device=dev, dtype=torch.uint8)
+        self.stream = torch.cuda.current_stream(dev)
+        self.sp = ctypes.c_void_p(self.stream.cuda_stream)
+
+    def _check(self, rc, what):
+        if rc:
+            raise self.aa.AxisAttnError(rc, what)
+
+    def step(self, ev=None):
+        """fwd, then the backward (three stages, or the deterministic call);
+        ev: 5 events recorded between the stages."""
+        aa, w, st = self.aa, self.w, self.stream
+        B, Hq, Hkv, S, D, c = w.B, w.Hq, w.Hkv, w.S, w.D, int(w.causal)
+        q, k, v, do = self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(), self.do.data_ptr()
+        ws, wsb, sp = self.ws.data_ptr(), self.ws_bytes, self.sp
+        rec = (lambda i: ev[i].record(st)) if ev else (lambda i: None)
+        rec(0)
+        self._check(aa.axis_attn_fwd(q, k, v, self.o.data_ptr(), self.lse.data_ptr(), B, Hq, Hkv, S, D, w.scale,
+                                     c, sp), "fwd")
+        rec(1)
+        if self.det:  # one call, three kernels: timed as a whole (the stage events coincide)
+            rec(2)
+            rec(3)
+            self._check(aa.axis_attn_bwd_det(q, k, v, self.o.data_ptr(), do, self.lse.data_ptr(),
+                                             self.dq.data_ptr(), self.dk.data_ptr(), self.dv.data_ptr(), B, Hq,
+                                             Hkv, S, D, w.scale, c, ws, wsb, sp), "bwd_det")
+            rec(4)
+            return
+        self._check(aa.axis_attn_bwd_prepare(self.o.data_ptr(), do, self.lse.data_ptr(), B, Hq, Hkv, S, D, ws,
+                                             wsb, sp), "bwd_prepare")
+        rec(2)
+        self._check(aa.axis_attn_bwd_main(q, k, v, do, self.dk.data_ptr(), self.dv.data_ptr(), B, Hq, Hkv, S, D,
+                                          w.scale, c, ws, wsb, sp), "bwd_main")
+        rec(3)
+        self._check(aa.axis_attn_bwd_finalize(self.dq.data_ptr(), B, Hq, Hkv, S, D, ws, wsb, sp), "bwd_finalize")
+        rec(4)
+
+
+def time_steps(prob, steps: int, warmup: int, flush, world: int, dev, sampler):
+    """W untimed steps, then K timed steps (events on the launching stream, L2
+    flushed before each, outside the events), barrier + synchronize on both
+    sides.  Returns (total ms max over ranks, per-stage ms totals max over
+    ranks, wall-clock window)."""
+    import torch
+    import torch.distributed as dist
+
+    for n in range(warmup):
+        flush.fill_(1)
+        prob.step()
+        if n == 0:
+            prob.aa.check_status(prob.stream)  # fail fast on a device-side timeout
+    prob.aa.check_status(prob.stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for s in range(steps):
+        flush.fill_(s & 0xFF)
+        prob.step(evs[s])
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        dist.barrier()
+    prob.aa.check_status(prob.stream)
+    per = [[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs]
+    stage_ms = [sum(p[i] for p in per) for i in range(4)]
+    step_ms = sum(e[0].elapsed_time(e[4]) for e in evs)
+    red = reduce_max([step_ms] + stage_ms, world, dev)
+    return red[0], red[1:], (t0, t1)
+
+
+def shard_problem(aa, w, seed: int, dev, det: bool, world: int, rank: int):
+    """Head-sharded mode: this rank's (b, kv) units of ONE problem (every rank
+    draws the same inputs), packed as a batch of units (B' = units, Hq' = G,
+    Hkv' = 1).  Returns the Problem and the whole problem's FLOPs."""
+    import dataclasses
+
+    from causal_attention_fwd_b200 import shard
+    from causal_attention_fwd_b200.synthetic import workload_inputs
+
+    q, k, v, do = workload_inputs(w, seed=seed)
+    G = w.Hq // w.Hkv
+    units = shard.rank_units(w.B, w.Hkv, world, rank)
+    host = (shard.pack(q, units, G), shard.pack(k, units, 1), shard.pack(v, units, 1), shard.pack(do, units, G))
+    wl = dataclasses.replace(w, name=f"{w.name}[units {rank}/{world}]", B=len(units), Hq=G, Hkv=1)
+    return Problem(aa, wl, seed, dev, det, host=host)
+
+
+def summarize(w, total_ms, stage_totals, steps, world, p_meas, det):
+    """Per-workload figures: fwd / bwd TFLOP/s and fractions of the peaks."""
+    avg = [float(t) / steps for t in stage_totals]
+    fwd_tf = w.fwd_flops / (avg[0] * 1e-3) / 1e12
+    bwd_ms = sum(avg[1:])
+    bwd_tf = w.bwd_flops / (bwd_ms * 1e-3) / 1e12
+    names = STAGES if not det else ["attn_fwd_kernel", "-", "-", "axis_attn_bwd_det (prep + main + dq_sum)"]
+    return {
+        "value": whole_job_tflops(w.fwd_flops + w.bwd_flops, steps, total_ms, world),
+        "ms_per_step": total_ms / steps, "steps": steps,
+        "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+        "fwd_frac_of_measured": fwd_tf / p_meas, "bwd_frac_of_measured": bwd_tf / p_meas,
+        "fwd_frac_of_nominal_2250": fwd_tf / P_NOM_TFLOPS, "bwd_frac_of_nominal_2250": bwd_tf / P_NOM_TFLOPS,
+        "kernel_ms": {n: t for n, t in zip(names, avg) if n != "-"},
+    }, avg, names
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -251,11 +414,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llm1b")
+    ap.add_argument("--others", default="tiny,gpt2s_gqa,llm8b_gqa,longseq",
+                    help="further workloads timed after the headline one (comma list; '' for none)")
+    ap.add_argument("--other-steps", type=int, default=20)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--deterministic", action="store_true",
                     help="time the bitwise-reproducible backward (axis_attn_bwd_det) instead")
+    ap.add_argument("--shard", action="store_true",
+                    help="N > 1: split ONE problem's (b, kv) units over the ranks (strong scaling) instead of "
+                         "one replica per rank")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -265,13 +434,11 @@ def main():
     if args.impl == "reference":
         return run_reference(args, rank, world)
 
-    import ctypes
-
     import torch
     import torch.distributed as dist
 
     import causal_attention_fwd_b200 as aa
-    from causal_attention_fwd_b200.synthetic import WORKLOAD_SEED, WORKLOADS, workload_inputs
+    from causal_attention_fwd_b200.synthetic import WORKLOAD_SEED, WORKLOADS
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -279,102 +446,31 @@ def main():
         import datetime
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    w = WORKLOADS[args.workload]
-    B, Hq, Hkv, S, D = w.B, w.Hq, w.Hkv, w.S, w.D
-    q_h, k_h, v_h, do_h = workload_inputs(w, seed=rank_seed(WORKLOAD_SEED[w.name], rank))
-    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
-    o = torch.empty_like(q)
-    lse = torch.empty((B, Hq, S), device=dev, dtype=torch.float32)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     det = args.deterministic
-    ws_bytes = (aa.axis_attn_bwd_det_workspace_bytes if det else aa.axis_attn_bwd_workspace_bytes)(B, Hq, Hkv, S, D)
-    ws = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    pk, pk_src = peaks()
+    p_meas = pk["bf16_tflops"]
     flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
-    stream = torch.cuda.current_stream(dev)
-    sp = ctypes.c_void_p(stream.cuda_stream)
-    causal = int(w.causal)
-
-    def check(rc, what):
-        if rc:
-            raise aa.AxisAttnError(rc, what)
-
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        check(aa.axis_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                               B, Hq, Hkv, S, D, w.scale, causal, sp), "fwd")
-        if ev:
-            ev[1].record(stream)
-        if det:  # one call, three kernels: timed as a whole (the stage events coincide)
-            if ev:
-                ev[2].record(stream)
-                ev[3].record(stream)
-            check(aa.axis_attn_bwd_det(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv,
-                                       S, D, w.scale, causal, ws.data_ptr(), ws_bytes, sp), "bwd_det")
-            if ev:
-                ev[4].record(stream)
-            return
-        check(aa.axis_attn_bwd_prepare(o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, Hq, Hkv, S, D,
-                                       ws.data_ptr(), ws_bytes, sp), "bwd_prepare")
-        if ev:
-            ev[2].record(stream)
-        check(aa.axis_attn_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(),
-                                    dv.data_ptr(), B, Hq, Hkv, S, D, w.scale, causal, ws.data_ptr(),
-                                    ws_bytes, sp), "bwd_main")
-        if ev:
-            ev[3].record(stream)
-        check(aa.axis_attn_bwd_finalize(dq.data_ptr(), B, Hq, Hkv, S, D, ws.data_ptr(), ws_bytes, sp),
-              "bwd_finalize")
-        if ev:
-            ev[4].record(stream)
-
-    for n in range(args.warmup):
-        flush.fill_(1)
-        step()
-        if n == 0:
-            aa.check_status(stream)  # fail fast on a device-side timeout
-    aa.check_status(stream)
-
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.05)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t_wall0 = time.time()
-    for s in range(args.steps):
-        flush.fill_(s & 0xFF)  # L2 flush, outside the events
-        step(evs[s])
-    torch.cuda.synchronize()
-    t_wall1 = time.time()
-    if world > 1:
-        dist.barrier()
-    sampler.stop()
-    aa.check_status(stream)
 
-    per = [[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs]
-    stage_ms = [sum(p[i] for p in per) for i in range(4)]  # ms per stage over all steps
-    step_ms = sum(e[0].elapsed_time(e[4]) for e in evs)
-    reduced = reduce_max([step_ms] + stage_ms, world, dev)
-    total_ms, totals = reduced[0], reduced[1:]
+    # ---- the headline workload
+    w = WORKLOADS[args.workload]
+    sharded = args.shard and world > 1
+    if sharded:  # one problem, its units over the ranks; kernels time this rank's share
+        prob = shard_problem(aa, w, WORKLOAD_SEED[w.name], dev, det, world, rank)
+    else:
+        prob = Problem(aa, w, rank_seed(WORKLOAD_SEED[w.name], rank), dev, det)
     K = args.steps
-    flops_step = w.fwd_flops + w.bwd_flops
-    value = whole_job_tflops(flops_step, K, total_ms, world)
-    names = ["attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_kernel", "attn_bwd_dq_convert_kernel"]
-    if det:
-        names = ["attn_fwd_kernel", "-", "-", "axis_attn_bwd_det (prep + main + dq_sum)"]
-    avg_ms = [float(totals[i]) / K for i in range(4)]
-    fwd_tf = w.fwd_flops / (avg_ms[0] * 1e-3) / 1e12
-    bwd_ms = sum(avg_ms[1:])
-    bwd_tf = w.bwd_flops / (bwd_ms * 1e-3) / 1e12
-    pk, pk_src = peaks()
-    p_meas = pk["bf16_tflops"]
+    total_ms, totals, win = time_steps(prob, K, args.warmup, flush, world, dev, sampler)
+    head, avg_ms, names = summarize(prob.w, total_ms, totals, K, world, p_meas, det)
+    if sharded:  # whole-job throughput: the one problem's FLOPs over the slowest rank's time
+        head["value"] = (w.fwd_flops + w.bwd_flops) * K / (total_ms * 1e-3) / 1e12
+    value = head["value"]
 
     # dominant kernel and its roofline
     dom = max(range(4), key=lambda i: avg_ms[i])
-    dom_flops = w.fwd_flops if dom == 0 else w.bwd_flops
+    dom_flops = prob.w.fwd_flops if dom == 0 else prob.w.bwd_flops
     roof = None
     if dom in (0, 2) or (det and dom == 3):
         achieved = dom_flops / (avg_ms[dom] * 1e-3) / 1e12
@@ -386,19 +482,21 @@ def main():
 
     # ---- end to end through the public API, host buffers, copies inside the timed region
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and not sharded:
         pin = lambda t: t.pin_memory()  # noqa: E731
+        q_h, k_h, v_h, do_h = prob.host
         hq, hk, hv, hdo = pin(q_h), pin(k_h), pin(v_h), pin(do_h)
-        ho, hl = torch.empty_like(hq).pin_memory(), torch.empty((B, Hq, S), dtype=torch.float32).pin_memory()
+        ho, hl = torch.empty_like(hq).pin_memory(), torch.empty((w.B, w.Hq, w.S), dtype=torch.float32).pin_memory()
         hdq, hdk, hdv = (torch.empty_like(t).pin_memory() for t in (hq, hk, hv))
-        qq, kk, vv, dd = (torch.empty_like(t) for t in (q, k, v, do))
+        qq, kk, vv, dd = (torch.empty_like(t) for t in (prob.q, prob.k, prob.v, prob.do))
+        stream = prob.stream
 
         def e2e_step():
             for dst, src in ((qq, hq), (kk, hk), (vv, hv), (dd, hdo)):
                 dst.copy_(src, non_blocking=True)
-            oo, ll = aa.attention_forward(qq, kk, vv, causal=w.causal, scale=w.scale, out=o, lse=lse)
-            g = aa.attention_backward(qq, kk, vv, oo, ll, dd, causal=w.causal, scale=w.scale, workspace=ws,
-                                      grads=(dq, dk, dv), deterministic=det)
+            oo, ll = aa.attention_forward(qq, kk, vv, causal=w.causal, scale=w.scale, out=prob.o, lse=prob.lse)
+            g = aa.attention_backward(qq, kk, vv, oo, ll, dd, causal=w.causal, scale=w.scale, workspace=prob.ws,
+                                      grads=(prob.dq, prob.dk, prob.dv), deterministic=det)
             for dst, src in ((ho, oo), (hl, ll), (hdq, g[0]), (hdk, g[1]), (hdv, g[2])):
                 dst.copy_(src, non_blocking=True)
 
@@ -417,30 +515,55 @@ def main():
         aa.check_status(stream)
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
         d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
-        e2e = {"value": whole_job_tflops(flops_step, args.e2e_steps, ems[0], world),
+        e2e = {"value": whole_job_tflops(w.fwd_flops + w.bwd_flops, args.e2e_steps, ems[0], world),
                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": args.e2e_steps}
+    clocks = sampler.summary(*win)
+    del prob
+    torch.cuda.empty_cache()
 
-    clocks = sampler.summary(t_wall0, t_wall1)
+    # ---- the other workloads: the same step, timed the same way, fewer steps
+    others = {}
+    for name in [n for n in args.others.split(",") if n and n != w.name and not sharded]:
+        wo = WORKLOADS[name]
+        po = Problem(aa, wo, rank_seed(WORKLOAD_SEED[wo.name], rank), dev, det)
+        ko = max(3, args.other_steps // 2) if wo.S >= 16384 else args.other_steps
+        t_ms, tot, wwin = time_steps(po, ko, 3, flush, world, dev, sampler)
+        summ, _, _ = summarize(wo, t_ms, tot, ko, world, p_meas, det)
+        summ["config"] = wo.describe()
+        summ["clocks"] = sampler.summary(*wwin)
+        others[name] = summ
+        summ["gpu_launches"] = 4 * ko
+        del po
+        torch.cuda.empty_cache()
+    sampler.stop()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         tf, cores, desc, t = cpu_sample(w, args.cpu_budget)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+        for name, summ in others.items():
+            tf, cores, desc, t = cpu_sample(WORKLOADS[name], args.cpu_budget)
+            summ["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                    "sample": desc}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,sigma^2), bf16-rounded; each rank its own batch)",
-            "config": workload_config(w, world),
-            "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
-            "fwd_frac_of_nominal_2250": fwd_tf / P_NOM_TFLOPS, "bwd_frac_of_nominal_2250": bwd_tf / P_NOM_TFLOPS,
-            "fwd_frac_of_measured": fwd_tf / p_meas, "bwd_frac_of_measured": bwd_tf / p_meas,
-            "kernel_ms": {n: t for n, t in zip(names, avg_ms) if n != "-"},
+            "scaling": "strong" if sharded else "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,sigma^2), bf16-rounded; " + (
+                "one problem, its (b, kv) units dealt round robin over the ranks)" if sharded else
+                "each rank its own batch)"),
+            "config": dict(workload_config(w, world), **({"parallelism": f"head-sharded units x{world} "
+                                                          "(no collective)"} if sharded else {})),
+            **{k: head[k] for k in ("fwd_tflops", "bwd_tflops", "fwd_frac_of_nominal_2250",
+                                    "bwd_frac_of_nominal_2250", "fwd_frac_of_measured", "bwd_frac_of_measured",
+                                    "kernel_ms")},
             "bwd_mode": "deterministic (axis_attn_bwd_det)" if det else "ordinary (axis_attn_bwd stages)",
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": 4 * K, "clocks": clocks,
+            "workloads": others,
         }
         print(json.dumps(line))
     if world > 1:

@@ -49,9 +49,9 @@ _lib = None
 
 
 class AxisAttnError(RuntimeError):
-    def __init__(self, code: int, where: str):
+    def __init__(self, code: int, where: str, detail: str | None = None):
         self.code = code
-        super().__init__(f"{where}: {STATUS.get(code, code)} ({strerror(code)})")
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({detail or strerror(code)})")
 
 
 def library_path() -> str:
@@ -166,30 +166,79 @@ def strerror(code: int) -> str:
 
 
 # ------------------------------------------------------------ torch helpers
-def _dims(q, k):
+ERR_SHAPE, ERR_UNSUPPORTED = 3, 4
+
+
+def _require(cond: bool, code: int, where: str, detail: str):
+    if not cond:
+        raise AxisAttnError(code, where, detail)
+
+
+def _check_tensor(t, name: str, shape, dtype, where: str):
+    """Shape, then dtype, then layout: everything the C ABI cannot see."""
+    import torch
+
+    _require(isinstance(t, torch.Tensor), ERR_SHAPE, where, f"{name} must be a torch.Tensor")
+    _require(tuple(t.shape) == tuple(shape), ERR_SHAPE, where,
+             f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    _require(t.dtype == dtype, ERR_UNSUPPORTED, where, f"{name} is {t.dtype}, expected {dtype}")
+    _require(t.is_contiguous(), ERR_SHAPE, where, f"{name} must be contiguous (row-major)")
+
+
+def _check_device(tensors: dict, where: str):
+    import torch
+
+    devs = {n: t.device for n, t in tensors.items()}
+    first = next(iter(devs.values()))
+    _require(first.type == "cuda", ERR_UNSUPPORTED, where, f"tensors must be on a CUDA device, got {first}")
+    bad = [n for n, d in devs.items() if d != first]
+    _require(not bad, ERR_SHAPE, where, f"{', '.join(bad)} not on {first}")
+    return torch.device(first)
+
+
+def _dims(q, k, v, where: str):
+    import torch
+
+    _require(isinstance(q, torch.Tensor) and q.dim() == 4, ERR_SHAPE, where, "q must be a 4-D tensor [B, S, Hq, D]")
+    _require(isinstance(k, torch.Tensor) and k.dim() == 4, ERR_SHAPE, where, "k must be a 4-D tensor [B, S, Hkv, D]")
     B, S, Hq, D = q.shape
     Hkv = k.shape[2]
+    _require(Hkv >= 1 and Hq % Hkv == 0, ERR_SHAPE, where, f"Hq = {Hq} is not a multiple of Hkv = {Hkv}")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(t, name, (B, S, Hq if name == "q" else Hkv, D), torch.bfloat16, where)
     return B, Hq, Hkv, S, D
 
 
-def _stream(stream):
+def _stream(stream, device=None):
+    """The caller's stream, else the current stream of `device` (the tensors'
+    device; the current device if None)."""
     import torch
 
-    s = torch.cuda.current_stream() if stream is None else stream
+    s = torch.cuda.current_stream(device) if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
 
 
 def attention_forward(q, k, v, causal: bool = True, scale: float | None = None, out=None,
                       lse=None, stream=None):
-    """O, LSE for bf16 CUDA tensors q [B,S,Hq,D], k/v [B,S,Hkv,D]."""
+    """O, LSE for bf16 CUDA tensors q [B,S,Hq,D], k/v [B,S,Hkv,D] (contiguous,
+    one device).  Raises AxisAttnError before any launch on a wrong dtype,
+    shape, layout or device."""
     import torch
 
-    B, Hq, Hkv, S, D = _dims(q, k)
+    where = "attention_forward"
+    B, Hq, Hkv, S, D = _dims(q, k, v, where)
+    if out is not None:
+        _check_tensor(out, "out", (B, S, Hq, D), torch.bfloat16, where)
+    if lse is not None:
+        _check_tensor(lse, "lse", (B, Hq, S), torch.float32, where)
+    dev = _check_device({n: t for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse))
+                         if t is not None}, where)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    o = torch.empty_like(q) if out is None else out
-    l = torch.empty((B, Hq, S), device=q.device, dtype=torch.float32) if lse is None else lse
-    rc = axis_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
-                       B, Hq, Hkv, S, D, scale, int(causal), _stream(stream))
+    with torch.cuda.device(dev):
+        o = torch.empty_like(q) if out is None else out
+        l = torch.empty((B, Hq, S), device=dev, dtype=torch.float32) if lse is None else lse
+        rc = axis_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                           B, Hq, Hkv, S, D, scale, int(causal), _stream(stream, dev))
     if rc:
         raise AxisAttnError(rc, "axis_attn_fwd")
     return o, l
@@ -198,23 +247,40 @@ def attention_forward(q, k, v, causal: bool = True, scale: float | None = None, 
 def attention_backward(q, k, v, o, lse, dout, causal: bool = True, scale: float | None = None,
                        workspace=None, grads=None, stream=None, deterministic: bool = False):
     """dQ, dK, dV (bf16) of sum(dO * O).  deterministic=True: axis_attn_bwd_det
-    (bitwise reproducible, larger workspace)."""
+    (bitwise reproducible, larger workspace).  Every tensor is checked (dtype,
+    shape, contiguity, one CUDA device) before any launch."""
     import torch
 
-    B, Hq, Hkv, S, D = _dims(q, k)
+    where = "attention_backward"
+    B, Hq, Hkv, S, D = _dims(q, k, v, where)
+    _check_tensor(o, "o", (B, S, Hq, D), torch.bfloat16, where)
+    _check_tensor(dout, "dout", (B, S, Hq, D), torch.bfloat16, where)
+    _check_tensor(lse, "lse", (B, Hq, S), torch.float32, where)
+    named = {"q": q, "k": k, "v": v, "o": o, "lse": lse, "dout": dout}
+    if grads is not None:
+        _require(len(grads) == 3, ERR_SHAPE, where, "grads must be (dq, dk, dv)")
+        for name, t, shp in zip(("dq", "dk", "dv"), grads, ((B, S, Hq, D), (B, S, Hkv, D), (B, S, Hkv, D))):
+            _check_tensor(t, name, shp, torch.bfloat16, where)
+            named[name] = t
+    if workspace is not None:
+        _require(isinstance(workspace, torch.Tensor) and workspace.is_contiguous(), ERR_SHAPE, where,
+                 "workspace must be a contiguous tensor")
+        named["workspace"] = workspace
+    dev = _check_device(named, where)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     size_fn, call, name = ((axis_attn_bwd_det_workspace_bytes, axis_attn_bwd_det, "axis_attn_bwd_det")
                            if deterministic else
                            (axis_attn_bwd_workspace_bytes, axis_attn_bwd, "axis_attn_bwd"))
     need = size_fn(B, Hq, Hkv, S, D)
-    if workspace is None:
-        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
-    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k),
-                                                  torch.empty_like(v))
-    rc = call(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
-              lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-              B, Hq, Hkv, S, D, scale, int(causal), workspace.data_ptr(),
-              workspace.numel() * workspace.element_size(), _stream(stream))
+    with torch.cuda.device(dev):
+        if workspace is None:
+            workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+        dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k),
+                                                      torch.empty_like(v))
+        rc = call(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                  lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                  B, Hq, Hkv, S, D, scale, int(causal), workspace.data_ptr(),
+                  workspace.numel() * workspace.element_size(), _stream(stream, dev))
     if rc:
         raise AxisAttnError(rc, name)
     return dq, dk, dv

@@ -32,16 +32,20 @@ def sources():
                   + [os.path.join(ROOT, "include", "axis_attn.h")])
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+def build(force: bool = False, verbose: bool = False, extra=(), out: str | None = None) -> str:
+    """Compile ``csrc/axis_attn.cu`` into ``out`` (default: the in-tree
+    ``libaxis_attn.so``).  ``extra`` adds nvcc flags (e.g. ``-D`` switches
+    for a test-only build, which then goes to its own ``out``)."""
+    lib = out or LIB
     newest = max(os.path.getmtime(p) for p in sources())
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest and not extra:
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= newest and not extra:
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [NVCC, *FLAGS, *(["-Xptxas", "-v"] if verbose else []), *extra,
            "-o", tmp, os.path.join(CSRC, "axis_attn.cu")]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

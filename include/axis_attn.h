@@ -24,7 +24,9 @@
  *    all bf16, contiguous, row-major.  lse is fp32 [B, Hq, S].
  *  - Pointers are DEVICE pointers owned by the caller and must be 16-byte
  *    aligned.  The library allocates no device memory and keeps no pointer
- *    after a call returns.
+ *    after a call returns, apart from the fixed scratch array of
+ *    axis_attn_bwd_noalloc() (below), which is part of the library's image
+ *    and whose device address it looks up once per device.
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
  *    is the legacy default stream), perform no host synchronisation and may be
  *    captured in a CUDA graph.
@@ -84,8 +86,9 @@ size_t axis_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int S, int D);
  * caller-owned device buffer of at least axis_attn_bwd_workspace_bytes() bytes,
  * 256-byte aligned; its contents on entry do not matter and on return are
  * unspecified.  Two calls that overlap on the device must not share it.
- * dq is accumulated in fp32 with atomic adds, so its low-order bits may vary
- * from run to run; dk and dv do not.
+ * dq is accumulated in fp32 by TMA reduce-add copies (cp.reduce.async.bulk,
+ * one 32 KB tile per key tile) applied in arrival order, so its low-order bits
+ * may vary from run to run; dk and dv do not (see axis_attn_bwd_det()).
  */
 int axis_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                   const void* dO, const float* lse, void* dq, void* dk, void* dv,
@@ -177,7 +180,9 @@ int axis_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
  * this library on the current device has reported a timed-out device wait since
  * the last call (and clears that report), AXIS_ATTN_ERR_CUDA if the CUDA
  * context holds an error, else AXIS_ATTN_OK.  For tests and debugging: it
- * blocks the host.
+ * blocks the host.  A launch that timed out leaves its outputs undefined; it
+ * does not affect later launches, whether or not this function is called in
+ * between (each launch only reacts to timeouts of its own CTAs).
  */
 int axis_attn_get_status(void* stream);
 

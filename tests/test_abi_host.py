@@ -132,8 +132,9 @@ def test_torch_helpers_raise_without_valid_args(lib):
 
     q = torch.zeros(1, 128, 2, 32, dtype=torch.bfloat16)  # CPU tensors, D = 32: rejected
     with pytest.raises(aa.AxisAttnError) as e:
-        aa.attention_forward(q, q[:, :, :1], q[:, :, :1], stream=type("S", (), {"cuda_stream": 0})())
-    assert e.value.code == 4
+        aa.attention_forward(q, q[:, :, :1].contiguous(), q[:, :, :1].contiguous(),
+                             stream=type("S", (), {"cuda_stream": 0})())
+    assert e.value.code == 4  # CPU tensors: rejected by the helper before the library is called
 
 
 def test_no_cpu_fallback(tmp_path, monkeypatch):

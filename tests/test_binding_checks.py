@@ -1,0 +1,91 @@
+"""CPU checks of the torch helpers' argument validation.
+
+attention_forward / attention_backward hand raw pointers to the C ABI, which
+cannot see dtypes, strides or devices.  So the helpers check every tensor
+(shape, then dtype, then contiguity, then one CUDA device) and raise
+AxisAttnError before any library call; on this CPU-only machine a correct call
+therefore stops at the device check, and each wrong one must stop earlier with
+its own message.
+"""
+import pytest
+import torch
+
+import causal_attention_fwd_b200 as aa
+
+B, S, Hq, Hkv, D = 1, 8, 4, 2, 64
+
+
+def bf(*shape):
+    return torch.zeros(shape, dtype=torch.bfloat16)
+
+
+def qkv():
+    return bf(B, S, Hq, D), bf(B, S, Hkv, D), bf(B, S, Hkv, D)
+
+
+def fwd_error(*args, **kw):
+    with pytest.raises(aa.AxisAttnError) as e:
+        aa.attention_forward(*args, **kw)
+    return e.value
+
+
+def bwd_error(**over):
+    q, k, v = qkv()
+    a = dict(q=q, k=k, v=v, o=bf(B, S, Hq, D), lse=torch.zeros(B, Hq, S), dout=bf(B, S, Hq, D))
+    a.update(over)
+    with pytest.raises(aa.AxisAttnError) as e:
+        aa.attention_backward(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dout"],
+                              grads=over.get("grads"), workspace=over.get("workspace"))
+    return e.value
+
+
+def test_correct_cpu_call_stops_at_the_device_check():
+    e = fwd_error(*qkv())
+    assert e.code == 4 and "CUDA device" in str(e)
+    e = bwd_error()
+    assert e.code == 4 and "CUDA device" in str(e)
+
+
+def test_forward_rejects_wrong_dtype():
+    q, k, v = qkv()
+    e = fwd_error(q.float(), k, v)
+    assert e.code == 4 and "q is torch.float32" in str(e)
+    e = fwd_error(q, k.half(), v)
+    assert "k is torch.float16" in str(e)
+
+
+def test_forward_rejects_non_contiguous():
+    q, k, v = qkv()
+    qt = bf(B, Hq, S, D).transpose(1, 2)  # right shape, wrong strides
+    e = fwd_error(qt, k, v)
+    assert e.code == 3 and "contiguous" in str(e)
+
+
+def test_forward_rejects_shape_mismatches():
+    q, k, v = qkv()
+    assert "Hq = 4 is not a multiple of Hkv = 3" in str(fwd_error(q, bf(B, S, 3, D), bf(B, S, 3, D)))
+    assert "v has shape" in str(fwd_error(q, k, bf(B, S + 1, Hkv, D)))
+    assert "k has shape" in str(fwd_error(q, bf(B, S, Hkv, D // 2), v))
+    assert "4-D" in str(fwd_error(q[0], k, v))
+    e = fwd_error(q, k, v, lse=torch.zeros(B, Hq, S + 1))
+    assert "lse has shape" in str(e)
+    e = fwd_error(q, k, v, out=bf(B, S, Hq, D).float())
+    assert "out is torch.float32" in str(e)
+
+
+def test_backward_rejects_each_bad_tensor():
+    assert "o has shape" in str(bwd_error(o=bf(B, S, Hkv, D)))
+    assert "dout is torch.float32" in str(bwd_error(dout=torch.zeros(B, S, Hq, D)))
+    assert "lse is torch.bfloat16" in str(bwd_error(lse=bf(B, Hq, S)))
+    grads = (bf(B, S, Hq, D), bf(B, S, Hq, D), bf(B, S, Hkv, D))
+    assert "dk has shape" in str(bwd_error(grads=grads))
+    assert "grads must be" in str(bwd_error(grads=grads[:2]))
+    ws = torch.zeros(64, dtype=torch.uint8)[::2]
+    assert "workspace must be a contiguous" in str(bwd_error(workspace=ws))
+
+
+def test_mixed_devices_are_rejected_before_any_call():
+    # a 'meta' tensor stands in for a second device: the check compares devices
+    q, k, v = qkv()
+    e = fwd_error(q, k, torch.empty((B, S, Hkv, D), dtype=torch.bfloat16, device="meta"))
+    assert e.code == 4  # the first tensor is not on CUDA

@@ -4,11 +4,11 @@ Some callers cannot allocate device memory at the point where they run the
 backward (inside an allocator callback, with a memory pool reserved up front,
 or on a path that must not block on the allocator) and have no workspace to
 hand over.  For them the library keeps a fixed 32 MiB scratch array of its own.
-This test calls that entry point through the C ABI twice in a row, on two
-different problems, and checks each result against the ordinary entry point
-(caller-provided workspace) with the parity tolerance of the other GPU tests.
-The second call checks that what the first call left in the shared scratch
-does not leak into the next result.  It also checks the size limit.
+This test calls that entry point through the C ABI three times in a row (a
+larger problem, a smaller one, the larger one again) and checks each result
+against the ordinary entry point (caller-provided workspace) with the parity
+tolerance of the other GPU tests.  The later calls check that what an earlier
+call left in the shared scratch does not leak into the next result.  It also checks the size limit.
 
 Kept in its own file, named to be collected last.
 """
@@ -52,11 +52,15 @@ def _rel(a, b):
     return float((a - b).norm() / b.norm())
 
 
-def test_noalloc_matches_workspace_entry_point_twice():
+def test_noalloc_matches_workspace_entry_point_in_a_row():
     dev = torch.device("cuda:0")
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    problems = [(2, 12, 4, 1024, 64, True, 31), (1, 4, 2, 777, 128, False, 32)]
-    for B, Hq, Hkv, S, D, causal, seed in problems:
+    # the larger problem, a smaller one with other region boundaries, then the
+    # larger one again: nothing the smaller call left in the shared scratch may
+    # leak into the third result
+    problems = [(2, 12, 4, 1024, 64, True, 31), (1, 4, 2, 777, 128, False, 32), (2, 12, 4, 1024, 64, True, 31)]
+    first = None
+    for n, (B, Hq, Hkv, S, D, causal, seed) in enumerate(problems):
         assert aa.axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D) <= LIMIT
         sc = 1.0 / math.sqrt(D)
         q, k, v, do = (t.to(dev) for t in make_inputs(B, Hq, Hkv, S, D, seed))
@@ -67,8 +71,13 @@ def test_noalloc_matches_workspace_entry_point_twice():
         for name, g, r in zip(("dq", "dk", "dv"), got, ref):
             assert torch.isfinite(g.float()).all(), name
             assert _rel(g, r) <= TOL_GRAD, (name, _rel(g, r))
-        # dK and dV take no atomics: the same kernels give the same bits
+        # dK and dV take no cross-CTA additions: the same kernels give the same bits
         assert torch.equal(got[1], ref[1]) and torch.equal(got[2], ref[2])
+        if n == 0:
+            first = got
+        elif n == 2:
+            assert torch.equal(got[1], first[1]) and torch.equal(got[2], first[2])
+            assert _rel(got[0], first[0]) <= TOL_GRAD
 
 
 def test_noalloc_rejects_sizes_beyond_the_scratch():
