@@ -405,6 +405,58 @@ int oracle_rope(double* x, int B, int S, int H, int D, double base, int inverse)
     return 0;
 }
 
+/*
+ * Decode step: one new query row per sequence against the keys and values
+ * already cached for it -- the step the axiomlm inference engine repeats per
+ * generated token: axiomlm (PyPI), Key Features ("State-cached Key-Value (KV)
+ * decode engine achieving O(1) step latency") and Quick Start section 4 ("Use
+ * the Paged KV-Cache engine for O(1) step decoding"), with the GQA heads of
+ * Key Features ("4-head Grouped-Query Attention").  The new token is the last
+ * position of its sequence, so the causal mask lets it see every cached key,
+ * itself included:
+ *   s_j  = scale * sum_d q[b,h,d] K[b,j,kv,d]       for j < lens[b], kv = h / G
+ *   o[b,h,:] = sum_j softmax(s)_j V[b,j,kv,:]         lse[b,h] = ln sum_j exp(s_j)
+ * q, o: [B, Hq, D]; k, v: [B, Smax, Hkv, D], of which sequence b uses its first
+ * lens[b] rows (1 <= lens[b] <= Smax); lse: [B, Hq].  (The cache's layout in
+ * device memory -- pages, a block table -- is the kernel's business; the
+ * definition reads it as one row per position.)  Returns 0, or -1 for bad sizes.
+ */
+int oracle_attn_decode(const double* q, const double* k, const double* v, const int* lens,
+                       double* o, double* lse, int B, int Hq, int Hkv, int Smax, int D,
+                       double scale) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Smax < 1 || D < 1 || Hq % Hkv) return -1;
+    for (int b = 0; b < B; ++b)
+        if (lens[b] < 1 || lens[b] > Smax) return -1;
+    const int G = Hq / Hkv;
+#pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)Smax);
+#pragma omp for collapse(2) schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < Hq; ++h) {
+                const int kv = h / G, L = lens[b];
+                const double* qh = q + ((size_t)b * Hq + h) * D;
+                double m = -INFINITY;
+                for (int j = 0; j < L; ++j) {
+                    s[j] = scale * dot(qh, k + (((size_t)b * Smax + j) * Hkv + kv) * D, D);
+                    if (s[j] > m) m = s[j];
+                }
+                double l = 0.0;
+                for (int j = 0; j < L; ++j) l += exp(s[j] - m);
+                double* oh = o + ((size_t)b * Hq + h) * D;
+                for (int d = 0; d < D; ++d) oh[d] = 0.0;
+                for (int j = 0; j < L; ++j) {
+                    const double pj = exp(s[j] - m) / l;
+                    const double* vj = v + (((size_t)b * Smax + j) * Hkv + kv) * D;
+                    for (int d = 0; d < D; ++d) oh[d] += pj * vj[d];
+                }
+                lse[(size_t)b * Hq + h] = m + log(l);
+            }
+        free(s);
+    }
+    return 0;
+}
+
 /* Threads OpenMP will use (1 when built without OpenMP). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

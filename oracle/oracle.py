@@ -84,9 +84,10 @@ class Oracle:
         lib.oracle_attn_bwd_dq_rows.argtypes = [_dp] * 4 + dims + [i, _ip, _dp, _dp]
         lib.oracle_attn_bwd_dkdv_rows.argtypes = [_dp] * 4 + dims + [i, _ip, _dp, _dp]
         lib.oracle_rope.argtypes = [_dp, i, i, i, i, d, i]
+        lib.oracle_attn_decode.argtypes = [_dp] * 3 + [_ip] + [_dp] * 2 + [i] * 5 + [d]
         for f in ("oracle_attn_fwd", "oracle_attn_fwd_rows", "oracle_attn_probs_row",
                   "oracle_attn_bwd", "oracle_attn_bwd_dq_rows", "oracle_attn_bwd_dkdv_rows",
-                  "oracle_rope", "oracle_max_threads"):
+                  "oracle_rope", "oracle_attn_decode", "oracle_max_threads"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
 
@@ -101,6 +102,24 @@ class Oracle:
         if self.lib.oracle_rope(_ptr(y), B, S, H, D, float(base), int(bool(inverse))):
             raise ValueError("oracle_rope rejected the arguments")
         return y
+
+    def attn_decode(self, q, k, v, lens, scale: float):
+        """Decode step: q [B, Hq, D] (one new row per sequence), cache k, v
+        [B, Smax, Hkv, D] of which sequence b uses its first lens[b] rows.
+        Returns (O [B, Hq, D], LSE [B, Hq]), float64."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, Hq, D = q.shape
+        Bk, Smax, Hkv, Dk = k.shape
+        if (B, D) != (Bk, Dk) or v.shape != k.shape:
+            raise ValueError(f"incompatible shapes q{q.shape} k{k.shape} v{v.shape}")
+        ln = np.ascontiguousarray(np.asarray(lens, dtype=np.int32).reshape(-1))
+        o = np.empty((B, Hq, D))
+        lse = np.empty((B, Hq))
+        rc = self.lib.oracle_attn_decode(_ptr(q), _ptr(k), _ptr(v), ln.ctypes.data_as(_ip), _ptr(o), _ptr(lse),
+                                         B, Hq, Hkv, Smax, D, float(scale))
+        if rc:
+            raise ValueError("oracle_attn_decode rejected the arguments")
+        return o, lse
 
     def attn_fwd(self, q, k, v, scale: float, causal: bool = True):
         """Full forward.  Returns (O [B,S,Hq,D], LSE [B,Hq,S]), float64."""
@@ -206,3 +225,4 @@ probs_row = _forward("probs_row")
 attn_bwd_dq_rows = _forward("attn_bwd_dq_rows")
 attn_bwd_dkdv_rows = _forward("attn_bwd_dkdv_rows")
 rope = _forward("rope")
+attn_decode = _forward("attn_decode")
