@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     EXPORTS,
     AxisAttnError,
     attention_backward,
+    attention_decode,
     attention_forward,
     axis_attn_bwd,
     axis_attn_bwd_det,
@@ -18,6 +19,8 @@ from .binding import (  # noqa: F401
     axis_attn_bwd_noalloc,
     axis_attn_bwd_prepare,
     axis_attn_bwd_workspace_bytes,
+    axis_attn_decode,
+    axis_attn_decode_workspace_bytes,
     axis_attn_fwd,
     axis_attn_get_status,
     axis_attn_last_status_word,

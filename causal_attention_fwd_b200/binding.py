@@ -28,6 +28,8 @@ EXPORTS = (
     "axis_attn_bwd_noalloc",
     "axis_attn_bwd_det_workspace_bytes",
     "axis_attn_bwd_det",
+    "axis_attn_decode_workspace_bytes",
+    "axis_attn_decode",
     "axis_attn_get_status",
     "axis_attn_last_status_word",
     "axis_attn_strerror",
@@ -42,6 +44,7 @@ STATUS = {
     5: "AXIS_ATTN_ERR_WORKSPACE",
     6: "AXIS_ATTN_ERR_CUDA",
     7: "AXIS_ATTN_ERR_TIMEOUT",
+    8: "AXIS_ATTN_ERR_INDEX",
 }
 
 _lock = threading.Lock()
@@ -87,6 +90,10 @@ def load():
             lib.axis_attn_bwd_det_workspace_bytes.restype = sz
             lib.axis_attn_bwd_det.argtypes = [vp] * 9 + [i] * 5 + [f, i, vp, sz, vp]
             lib.axis_attn_bwd_det.restype = i
+            lib.axis_attn_decode_workspace_bytes.argtypes = [i] * 6
+            lib.axis_attn_decode_workspace_bytes.restype = sz
+            lib.axis_attn_decode.argtypes = [vp] * 7 + [i] * 7 + [f, vp, sz, vp]
+            lib.axis_attn_decode.restype = i
             lib.axis_attn_get_status.argtypes = [vp]
             lib.axis_attn_get_status.restype = i
             lib.axis_attn_last_status_word.argtypes = []
@@ -144,6 +151,17 @@ def axis_attn_bwd_det(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, 
     the key tiles in a fixed order; see include/axis_attn.h)."""
     return load().axis_attn_bwd_det(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
                                     workspace, workspace_bytes, stream)
+
+
+def axis_attn_decode_workspace_bytes(B, Hq, Hkv, D, page_size, max_pages) -> int:
+    return int(load().axis_attn_decode_workspace_bytes(B, Hq, Hkv, D, page_size, max_pages))
+
+
+def axis_attn_decode(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size, max_pages,
+                     num_pages, scale, workspace, workspace_bytes, stream) -> int:
+    """Decode step against a paged KV cache (see include/axis_attn.h)."""
+    return load().axis_attn_decode(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
+                                   max_pages, num_pages, scale, workspace, workspace_bytes, stream)
 
 
 def axis_attn_get_status(stream) -> int:
@@ -284,6 +302,52 @@ def attention_backward(q, k, v, o, lse, dout, causal: bool = True, scale: float 
     if rc:
         raise AxisAttnError(rc, name)
     return dq, dk, dv
+
+
+def attention_decode(q, k_cache, v_cache, block_table, seq_lens, scale: float | None = None, out=None,
+                     lse=None, workspace=None, stream=None):
+    """Decode step: q [B, Hq, D] bf16, k_cache / v_cache [num_pages, page_size,
+    Hkv, D] bf16, block_table [B, max_pages] int32, seq_lens [B] int32, all on
+    one CUDA device.  Returns (o [B, Hq, D] bf16, lse [B, Hq] fp32)."""
+    import torch
+
+    where = "attention_decode"
+    _require(isinstance(q, torch.Tensor) and q.dim() == 3, ERR_SHAPE, where, "q must be a 3-D tensor [B, Hq, D]")
+    _require(isinstance(k_cache, torch.Tensor) and k_cache.dim() == 4, ERR_SHAPE, where,
+             "k_cache must be a 4-D tensor [num_pages, page_size, Hkv, D]")
+    B, Hq, D = q.shape
+    num_pages, page_size, Hkv, _ = k_cache.shape
+    _check_tensor(q, "q", (B, Hq, D), torch.bfloat16, where)
+    _check_tensor(k_cache, "k_cache", (num_pages, page_size, Hkv, D), torch.bfloat16, where)
+    _check_tensor(v_cache, "v_cache", (num_pages, page_size, Hkv, D), torch.bfloat16, where)
+    _require(isinstance(block_table, torch.Tensor) and block_table.dim() == 2, ERR_SHAPE, where,
+             "block_table must be a 2-D tensor [B, max_pages]")
+    max_pages = block_table.shape[1]
+    _check_tensor(block_table, "block_table", (B, max_pages), torch.int32, where)
+    _check_tensor(seq_lens, "seq_lens", (B,), torch.int32, where)
+    named = {"q": q, "k_cache": k_cache, "v_cache": v_cache, "block_table": block_table, "seq_lens": seq_lens}
+    if out is not None:
+        _check_tensor(out, "out", (B, Hq, D), torch.bfloat16, where)
+        named["out"] = out
+    if lse is not None:
+        _check_tensor(lse, "lse", (B, Hq), torch.float32, where)
+        named["lse"] = lse
+    dev = _check_device(named, where)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    need = axis_attn_decode_workspace_bytes(B, Hq, Hkv, D, page_size, max_pages)
+    with torch.cuda.device(dev):
+        o = torch.empty_like(q) if out is None else out
+        l = torch.empty((B, Hq), device=dev, dtype=torch.float32) if lse is None else lse
+        if workspace is None and need > 0:
+            workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+        wp = workspace.data_ptr() if workspace is not None else None
+        wb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        rc = axis_attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
+                              seq_lens.data_ptr(), o.data_ptr(), l.data_ptr(), B, Hq, Hkv, D, page_size, max_pages,
+                              num_pages, scale, wp, wb, _stream(stream, dev))
+    if rc:
+        raise AxisAttnError(rc, "axis_attn_decode")
+    return o, l
 
 
 def check_status(stream=None):

@@ -21,10 +21,10 @@
 //       dV += P^T dO (A from TMEM), dK += dS^T Q, and dQ of the tile,
 //     the compute warps copy each dQ tile from TMEM into a swizzled
 //     shared-memory staging tile, which one thread adds into the fp32
-//     accumulator with TMA reduce-add copies (deterministic mode: TMA stores
-//     into a slice of this key tile's own); dK, dV stay in TMEM until the end;
-//   * dQ finalize (HBM-bound): bf16 copy of the accumulator in [B,S,Hq,D]
-//     (deterministic mode: the key tiles' slices added in key-tile order).
+//     accumulator with TMA reduce-add copies; dK, dV stay in TMEM until the
+//     end.  In the deterministic mode the kernel skips dQ altogether (the
+//     separate pass of attn_bwd_dq.cuh recomputes it per query tile);
+//   * dQ finalize (HBM-bound): bf16 copy of the accumulator in [B,S,Hq,D].
 // D = 64 uses 128-row query tiles and dQ = dS K (TMEM lane = query row);
 // D = 128 uses 64-row query tiles (shared memory) and dQ^T = K^T dS^T (TMEM
 // lane = feature), so every MMA has M = 128.
@@ -39,10 +39,10 @@ struct BwdArgs {
   __nv_bfloat16* dv;
   const float* nlse2;  // [B*Hq][S_pad]  -LSE * log2(e); -inf on padding rows
   const float* ndr;    // [B*Hq][S_pad]  -rowsum(dO * O); 0 on padding rows
-  float* dqacc;        // [B*Hq][S][HD] fp32, pre-scaled by `scale` (det: [nkv][B*Hq][S][HD] slices)
+  float* dqacc;        // [B*Hq][S][HD] fp32, pre-scaled by `scale` (unused when no_dq)
   int B, Hq, Hkv, S, S_pad;
   float scale, scale_log2;
-  int det;             // 1: store each key tile's dQ tile into its own slice (deterministic mode)
+  int no_dq;           // 1: dK, dV only (deterministic mode: attn_bwd_dq_kernel computes dQ)
 };
 
 template <int HD>
@@ -82,17 +82,24 @@ struct BwdCfg {
   static_assert(T_P + BM / 2 <= 512, "TMEM budget");
 };
 
-// Warps 0-7: P^T / dS^T (thread = key row, half the query columns each) and
-// the dQ tile of the previous step into the staging tile; warp 8 loads; warp 9
-// issues the score MMAs and owns TMEM; warp 10 issues the TMA reduce-adds of
-// the dQ tiles into the fp32 accumulator (or their stores into this key tile's
-// slice); warp 11 issues the gradient MMAs.
-// 384 threads: up to 168 registers each.
-constexpr int BWD_THREADS = 384;
+// Which of the 16 column pairs of a 32-column block take the FP32-pipe
+// polynomial for 2^x instead of the MUFU (bit i: pair i).
+#ifndef AXIS_ATTN_BWD_POLY_MASK
+#define AXIS_ATTN_BWD_POLY_MASK 0x0000
+#endif
+
+// Warps 0-7: P^T / dS^T (thread = key row, half the query columns each);
+// warp 8 loads; warp 9 issues the score MMAs and owns TMEM; warp 10 issues
+// the TMA reduce-adds of the dQ tiles into the fp32 accumulator; warp 11
+// issues the gradient MMAs; warps 12-15 copy each dQ tile from TMEM into the
+// swizzled staging tile (one TMEM lane quarter each), off the compute warps'
+// critical path.  512 threads: up to 128 registers each.
+constexpr int BWD_THREADS = 512;
 constexpr int BWD_WARP_LOAD = 8;
 constexpr int BWD_WARP_MMA = 9;
 constexpr int BWD_WARP_RED = 10;
 constexpr int BWD_WARP_GRAD = 11;
+constexpr int BWD_WARP_DQ0 = 12;
 
 enum BwdSite { B_KV = 21, B_QEMPTY, B_QFULL, B_SPFREE, B_PDSFULL, B_DQFREE, B_SPFULL, B_DQFULL, B_FIN, B_PDSFREE,
                B_STGFULL, B_STGFREE };
@@ -108,6 +115,29 @@ __device__ __forceinline__ void store_row16(uint32_t buf, int kr, int col0, cons
                : "memory");
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a1), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
                : "memory");
+}
+
+// Launch order of the (key tile j, (b, kv head) unit) work items.  The
+// (b, kv) units are taken in groups of UG; within a group the key tiles with
+// the most query tiles come first (causal), every unit of the group at each
+// key tile.  CTAs resident at the same time then share the Q and dO tiles and
+// the dQ accumulator rows of only about UG units, which stay in L2; UG = 0
+// puts all units in one group (key-tile-major order over the whole grid).
+#ifndef AXIS_ATTN_BWD_UNIT_GROUP
+#define AXIS_ATTN_BWD_UNIT_GROUP 0
+#endif
+__device__ __forceinline__ void bwd_item(int BKV, int nkv, int x, int& j, int& bkv) {
+  const int UG = AXIS_ATTN_BWD_UNIT_GROUP > 0 && AXIS_ATTN_BWD_UNIT_GROUP < BKV ? AXIS_ATTN_BWD_UNIT_GROUP : BKV;
+  const int full = BKV / UG * UG;  // units in whole groups
+  if (x < full * nkv) {
+    const int g = x / (UG * nkv), r = x % (UG * nkv);
+    j = r / UG;
+    bkv = g * UG + r % UG;
+  } else {  // the last, partial group
+    const int rem = BKV - full, r = x - full * nkv;
+    j = r / rem;
+    bkv = full + r % rem;
+  }
 }
 
 template <int HD, bool CAUSAL>
@@ -144,14 +174,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const uint32_t bar_stgfull = bars + 8u * (9 + 2 * ST);  // dQ tile staged (8 warps)
   const uint32_t bar_stgfree = bars + 8u * (10 + 2 * ST); // staged tile read by the TMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 8 * C::NBAR);
-  volatile int* abort = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + 8 * C::NBAR + 4);
+  volatile WaitCtl* abort = reinterpret_cast<volatile WaitCtl*>(gbase + C::OFF_BAR + 8 * C::NBAR + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work item: key tiles with the most query tiles first
+  // ---- work item
   const int BKV = a.B * a.Hkv;
-  const int j = (int)(blockIdx.x / BKV);
-  const int bkv = (int)(blockIdx.x % BKV);
+  int j, bkv;
+  bwd_item(BKV, (a.S + 127) / 128, (int)blockIdx.x, j, bkv);
   const int b = bkv / a.Hkv, kvh = bkv % a.Hkv;
   const int G = a.Hq / a.Hkv;
   const int nqt = (a.S + BM - 1) / BM;
@@ -170,12 +200,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(bar_pdsfull, 8);
     mbar_init(bar_ptfree, 1);
     mbar_init(bar_dqfull, 1);
-    mbar_init(bar_dqfree, 8);
+    mbar_init(bar_dqfree, 4);
     mbar_init(bar_fin, 2);
     mbar_init(bar_dstfree, 1);
-    mbar_init(bar_stgfull, 8);
+    mbar_init(bar_stgfull, 4);
     mbar_init(bar_stgfree, 1);
-    *abort = 0;
+    wait_ctl_init(abort);
     fence_barrier_init();
   }
   if (warp == BWD_WARP_MMA) {
@@ -227,7 +257,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         bulk_load(base + C::OFF_DR + s * BM * 4, a.ndr + row, BM * 4, bar_qfull(s));
         issued = it + 1;
       }
-      volatile int never = 0;
+      volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
       mbar_wait_bounded(bar_kv, 0, &never, B_KV);
       for (int it = issued - ST > 0 ? issued - ST : 0; it < issued; ++it)
         mbar_wait_bounded(bar_qfull(it % ST), (it / ST) & 1, &never, B_QFULL);
@@ -288,6 +318,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                    ID_GV, (it > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit_w(bar_qempty(s));  // this warp is done with Q, dO of the step
+        if (a.no_dq) {  // dQ comes from the separate deterministic pass
+          mma_commit_w(bar_dstfree);
+          continue;
+        }
         // dQ tile (reduction over the 128 keys) once the previous one has been read
         if (it >= 1 && !wait_warp<true>(bar_dqfree, (it - 1) & 1, abort, B_DQFREE)) break;
         tc_fence_after();
@@ -306,11 +340,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
     // Drain: all MMAs issued by this warp complete before TMEM is freed.
     mma_commit_w(bar_fin);
-    volatile int never = 0;
+    volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
     wait_warp<true>(bar_fin, 0, &never, B_FIN);
   } else if (warp == BWD_WARP_RED) {
-    if (lane == 0) {
-      // ===================================================== dQ tiles -> fp32 accumulator (TMA add or store)
+    if (lane == 0 && !a.no_dq) {
+      // ===================================================== dQ tiles -> fp32 accumulator (TMA reduce-add)
       tma_prefetch_desc(&tm_dq);
       for (int t = 0; t < n_it; ++t) {
         if (!mbar_wait_bounded(bar_stgfull, t & 1, abort, B_STGFULL)) break;
@@ -322,16 +356,62 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           const int c0 = C::QLANE ? 32 * (bx & 1) : 32 * bx;
           const int r0 = C::QLANE ? q0 + 64 * (bx >> 1) : q0;
           if (r0 >= a.S) continue;
-          if (a.det)  // slice of key tile j: [j][b*Hq + h][S][HD]
-            tma_store_3d(&tm_dq, sSTG + bx * C::DQ_BOX, c0, r0, bh + a.B * a.Hq * j);
-          else
-            tma_reduce_add_3d(&tm_dq, sSTG + bx * C::DQ_BOX, c0, r0, bh);
+          tma_reduce_add_3d(&tm_dq, sSTG + bx * C::DQ_BOX, c0, r0, bh);
         }
         bulk_commit();
         bulk_wait_read0();
         mbar_arrive(bar_stgfree);
       }
       bulk_wait0();
+    }
+  } else if (warp >= BWD_WARP_DQ0) {
+    // ===================================================== dQ tiles: TMEM -> staging tile
+    // D = 64: TMEM lane = query row, 64 feature columns; D = 128: lane =
+    // feature, 64 query-row columns.  Both halves of the tile go to the
+    // staging tile as four 128B-swizzled fp32 boxes of 64 rows x 32 columns.
+    if (!a.no_dq) {
+      const int wq = warp & 3;
+      const int kr = wq * 32 + lane;
+      const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+      const float sc = a.scale;
+      for (int t = 0; t < n_it; ++t) {
+        if (!wait_warp(bar_dqfull, t & 1, abort, B_DQFULL)) break;
+        tc_fence_after();
+        uint32_t v[2][32];
+        tmem_ld32(tmem + lane_off + C::T_DQ, v[0]);
+        tmem_ld32(tmem + lane_off + C::T_DQ + 32, v[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_dqfree);
+        if (t > 0 && !wait_warp(bar_stgfree, (t - 1) & 1, abort, B_STGFREE)) break;
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          if (C::QLANE) {
+            // lane = query row kr, columns = features [32 ch, 32 ch + 32): one 128-byte box row
+            const uint32_t row = sSTG + ((kr >> 6) * 2 + ch) * C::DQ_BOX + (kr & 63) * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(row + ((c ^ (kr & 7)) << 4)),
+                           "f"(__uint_as_float(v[ch][4 * c]) * sc), "f"(__uint_as_float(v[ch][4 * c + 1]) * sc),
+                           "f"(__uint_as_float(v[ch][4 * c + 2]) * sc), "f"(__uint_as_float(v[ch][4 * c + 3]) * sc)
+                           : "memory");
+          } else {
+            // lane = feature kr (box kr / 32, column kr % 32), columns = query rows 32 ch + e
+            const uint32_t boxb = sSTG + wq * C::DQ_BOX + ((lane & 3) << 2);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int q = 32 * ch + e;
+              asm volatile("st.shared.f32 [%0], %1;" ::"r"(boxb + q * 128 + (((lane >> 2) ^ (q & 7)) << 4)),
+                           "f"(__uint_as_float(v[ch][e]) * sc)
+                           : "memory");
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_stgfull);
+      }
     }
   } else if (warp < 8) {
     // ===================================================== P^T, dS^T (thread = key row)
@@ -341,44 +421,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int c0 = ch * HALF;
     const uint64_t cc2 = f2_pack(a.scale_log2, a.scale_log2);
-    const float sc = a.scale;
     bool ok = true;
-    // dQ tile of step `t` from TMEM into the staging tile for the TMA add
-    auto dq_readout = [&](int t) -> bool {
-      if (!wait_warp(bar_dqfull, t & 1, abort, B_DQFULL)) return false;
-      tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_off + C::T_DQ + 32 * ch, v);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_dqfree);
-      if (t > 0 && !wait_warp(bar_stgfree, (t - 1) & 1, abort, B_STGFREE)) return false;
-      if (C::QLANE) {
-        // lane = query row kr, columns = features [32 ch, 32 ch + 32): one 128-byte box row
-        const uint32_t row = sSTG + ((kr >> 6) * 2 + ch) * C::DQ_BOX + (kr & 63) * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(row + ((c ^ (kr & 7)) << 4)),
-                       "f"(__uint_as_float(v[4 * c]) * sc), "f"(__uint_as_float(v[4 * c + 1]) * sc),
-                       "f"(__uint_as_float(v[4 * c + 2]) * sc), "f"(__uint_as_float(v[4 * c + 3]) * sc)
-                       : "memory");
-      } else {
-        // lane = feature kr (box kr / 32, column kr % 32), columns = query rows 32 ch + e
-        const uint32_t boxb = sSTG + wq * C::DQ_BOX + ((lane & 3) << 2);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int q = 32 * ch + e;
-          asm volatile("st.shared.f32 [%0], %1;" ::"r"(boxb + q * 128 + (((lane >> 2) ^ (q & 7)) << 4)),
-                       "f"(__uint_as_float(v[e]) * sc)
-                       : "memory");
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_stgfull);
-      return true;
-    };
     for (int it = 0; it < n_it; ++it) {
       const int s = it % ST;
       // the staged -LSE2 / -Dr rows of this step (TMA-written) and S^T, dP^T in TMEM
@@ -392,7 +435,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const bool need_mask = (CAUSAL && q0 < 128 * j + 127) || (128 * j + 128 > a.S);
       const float* lse_t = lse_s + s * BM + c0;
       const float* dr_t = dr_s + s * BM + c0;
-      uint32_t dk[NCH][16];
 #pragma unroll
       for (int cc = 0; cc < NCH; ++cc) {
         uint32_t sv[32], dpv[32];
@@ -405,7 +447,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(bar_spfree);
         }
-        uint32_t pk[16];
+        uint32_t pk[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(lse_t + 32 * cc + e);
@@ -415,9 +457,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             const int ee = e + 2 * h2;
             const uint64_t nl = h2 ? f2_pack(l4.z, l4.w) : f2_pack(l4.x, l4.y);
             const uint64_t nd = h2 ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y);
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[ee]), __uint_as_float(sv[ee + 1])), cc2, nl), x0, x1);
-            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[ee]), __uint_as_float(sv[ee + 1])), cc2, nl);
+            float p0, p1;
+            if ((AXIS_ATTN_BWD_POLY_MASK >> (ee / 2)) & 1) {
+              f2_unpack(f2_exp2_poly(x), p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(x, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
             if (need_mask) {
               const int q = q0 + c0 + 32 * cc + ee;
               if ((CAUSAL && key > q) || key >= a.S) p0 = 0.f;
@@ -427,7 +476,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             const uint64_t dd =
                 f2_mul(pp, f2_add(f2_pack(__uint_as_float(dpv[ee]), __uint_as_float(dpv[ee + 1])), nd));
             pk[ee / 2] = pack_bf16x2(pp);
-            dk[cc][ee / 2] = pack_bf16x2(dd);
+            dk[ee / 2] = pack_bf16x2(dd);
           }
         }
         // the previous step's dV must be done with P^T before it is overwritten
@@ -436,30 +485,21 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           break;
         }
         tmem_st16(tmem + lane_off + C::T_P + (c0 >> 1) + 16 * cc, pk);
+        // ... and the previous step's dK, dQ with dS^T
+        if (cc == 0 && it > 0 && !wait_warp(bar_dstfree, (it - 1) & 1, abort, B_PDSFREE)) {
+          ok = false;
+          break;
+        }
+        store_row16(sDST, kr, c0 + 32 * cc, &dk[0]);
+        store_row16(sDST, kr, c0 + 32 * cc + 16, &dk[8]);
       }
       if (!ok) break;
-      // ... and the previous step's dK, dQ with dS^T
-      if (it > 0 && !wait_warp(bar_dstfree, (it - 1) & 1, abort, B_PDSFREE)) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int cc = 0; cc < NCH; ++cc) {
-        store_row16(sDST, kr, c0 + 32 * cc, &dk[cc][0]);
-        store_row16(sDST, kr, c0 + 32 * cc + 16, &dk[cc][8]);
-      }
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pdsfull);
-      // the previous step's dQ tile (its MMA was issued before this step's P^T, dS^T)
-      if (it > 0 && !dq_readout(it - 1)) {
-        ok = false;
-        break;
-      }
+      if (lane == 0 && !(AXIS_ATTN_TEST_DROP_ARRIVE == 2 && it == 0)) mbar_arrive(bar_pdsfull);
     }
-    if (ok && n_it > 0) ok = dq_readout(n_it - 1);
     // epilogue: warps 0-3 write dV, warps 4-7 write dK (x scale)
     if (ok && wait_warp(bar_fin, 0, abort, B_FIN)) {
       tc_fence_after();
@@ -571,41 +611,6 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
     out.z = pack_bf16x2(y.x, y.y);
     out.w = pack_bf16x2(y.z, y.w);
     reinterpret_cast<uint4*>(dq + row * HD)[c8] = out;
-  }
-}
-
-// Deterministic mode: dq[b,i,h,:] = bf16(sum over key tiles j of the slices
-// part[j][b*Hq+h][i][:]), added in the order j = 0, 1, ... (only the tiles row
-// i sees when causal: j <= i / 128, the ones whose CTA wrote a tile for i).
-// 8 features per thread, slices read row-contiguously.
-template <int HD>
-__global__ void __launch_bounds__(256) attn_bwd_dq_sum_kernel(const float* __restrict__ part,
-                                                              __nv_bfloat16* __restrict__ dq, int Hq, int S,
-                                                              int nkv, int causal, size_t n8) {
-  const size_t stride = (size_t)gridDim.x * blockDim.x;
-  const size_t slice = n8 * 8;  // floats per key-tile slice: B * Hq * S * HD
-  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < n8; k += stride) {
-    const int c8 = (int)(k % (HD / 8));
-    const size_t bi_row = k / (HD / 8);  // (b*Hq + h) * S + i
-    const int i = (int)(bi_row % S);
-    const size_t bh = bi_row / S;
-    const int h = (int)(bh % Hq);
-    const size_t b = bh / Hq;
-    const int last = causal ? i / 128 : nkv - 1;
-    const float* src = part + bi_row * HD + 8 * c8;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j <= last; ++j) {
-      const float4 x = reinterpret_cast<const float4*>(src + (size_t)j * slice)[0];
-      const float4 y = reinterpret_cast<const float4*>(src + (size_t)j * slice)[1];
-      acc[0] += x.x; acc[1] += x.y; acc[2] += x.z; acc[3] += x.w;
-      acc[4] += y.x; acc[5] += y.y; acc[6] += y.z; acc[7] += y.w;
-    }
-    uint4 out;
-    out.x = pack_bf16x2(acc[0], acc[1]);
-    out.y = pack_bf16x2(acc[2], acc[3]);
-    out.z = pack_bf16x2(acc[4], acc[5]);
-    out.w = pack_bf16x2(acc[6], acc[7]);
-    reinterpret_cast<uint4*>(dq + ((b * S + i) * Hq + h) * HD)[c8] = out;
   }
 }
 

@@ -131,18 +131,43 @@ __device__ __forceinline__ float row_max32(const uint32_t (&v)[32]) {
   return fmax3(a, b, fmax3(d, __uint_as_float(v[30]), __uint_as_float(v[31])));
 }
 
+// Which of the 16 column pairs of a 32-column block take the FP32-pipe
+// polynomial for 2^x instead of the MUFU (bit i: pair i).  The MUFU does 16
+// exponentials per clock per SM, which at head dim 64 is below the rate of
+// the two MMAs; moving a share of them to the FP32 pipe balances the two.
+#ifndef AXIS_ATTN_FWD_POLY_MASK
+#define AXIS_ATTN_FWD_POLY_MASK 0x0000
+#endif
+// 1: the two query tiles take turns on the exponentials (a token barrier);
+// 0: both run them whenever their scores are ready.
+#ifndef AXIS_ATTN_FWD_TOKEN
+#define AXIS_ATTN_FWD_TOKEN 0
+#endif
+// 1: each half-row thread reads the other half's 64 scores from TMEM for the
+// row max (a second TMEM pass) instead of swapping partial maxima with its
+// partner warp through shared memory (a barrier round trip per kv tile).
+#ifndef AXIS_ATTN_FWD_NOXCH
+#define AXIS_ATTN_FWD_NOXCH 0
+#endif
+
 // Scores v[2 I0 .. 2 (I0 + N)) -> probabilities 2^(s*c - m): packed FMA for
-// the argument, MUFU ex2 for the exponential, packed add into the running row
-// sum, and the bf16 pairs into pk[I0 .. I0 + N) (to be stored to TMEM).
+// the argument, MUFU ex2 (or the polynomial, for the pairs the mask selects)
+// for the exponential, packed add into the running row sum, and the bf16
+// pairs into pk[I0 .. I0 + N) (to be stored to TMEM).
 template <int I0, int N>
 __device__ __forceinline__ uint64_t exp_pairs(const uint32_t (&v)[32], uint64_t cc2, uint64_t nm2, uint64_t acc,
                                               uint32_t (&pk)[16]) {
 #pragma unroll
   for (int i = I0; i < I0 + N; ++i) {
     const uint64_t x = f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), cc2, nm2);
-    float x0, x1;
-    f2_unpack(x, x0, x1);
-    const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+    uint64_t pp;
+    if ((AXIS_ATTN_FWD_POLY_MASK >> i) & 1) {
+      pp = f2_exp2_poly(x);
+    } else {
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+    }
     acc = f2_add(acc, pp);
     pk[i] = pack_bf16x2(pp);
   }
@@ -222,7 +247,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   auto bar_ofree = [&](int t) { return bars + 8u * (B2 + 19 + t); };
   float* xch = reinterpret_cast<float*>(gbase + C::XCH_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::BAR_OFF + 8 * C::NBAR);
-  volatile int* abort = reinterpret_cast<volatile int*>(gbase + C::BAR_OFF + 8 * C::NBAR + 4);
+  volatile WaitCtl* abort = reinterpret_cast<volatile WaitCtl*>(gbase + C::BAR_OFF + 8 * C::NBAR + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkv = (a.S + 127) / 128;
@@ -248,7 +273,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       for (int wq = 0; wq < 4; ++wq) mbar_init(bar_xch(t, wq), 2);
     }
     mbar_init(bar_fin, 2);  // one commit from each MMA issuer
-    *abort = 0;
+    wait_ctl_init(abort);
     fence_barrier_init();
   }
   if (warp == FWD_WARP_MMA) {
@@ -324,7 +349,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       }
       // Drain: every copy this thread started has landed before the CTA exits
       // (each stage's most recent phase; nothing newer can have started).
-      volatile int never = 0;
+      volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
       const int NS = is_k ? KST : VST;
       if (is_k && nq > 0) mbar_wait_bounded<true>(bar_q, (nq - 1) & 1, &never, F_Q);
       for (int x = g - NS > 0 ? g - NS : 0; x < g; ++x)
@@ -383,7 +408,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     }
     // Drain: all MMAs issued by this warp complete before TMEM is freed.
     mma_commit_w(bar_fin);
-    volatile int never = 0;
+    volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
     wait_warp<true>(bar_fin, 0, &never, F_OFIN);
   } else if (warp == FWD_WARP_PV) {
     // ===================================================== P V issuer
@@ -431,7 +456,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       g += I.nmax;
     }
     mma_commit_w(bar_fin);
-    volatile int never = 0;
+    volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
     wait_warp<true>(bar_fin, 0, &never, F_OFIN);
   } else if (warp < FWD_SOFTMAX_WARPS) {
     // ===================================================== softmax (tile t, half hf)
@@ -458,7 +483,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       const int qt = 2 * I.m + t;
       const int row_g = qt * 128 + r;
       float m_used = -INFINITY, l = 0.f;
-      for (int j = 0; j < n_t; ++j, ++J, ++X) {
+      for (int j = 0; j < n_t; ++j, ++J, X += !AXIS_ATTN_FWD_NOXCH) {
         if (!wait_warp<true>(bar_sfull(t), J & 1, abort, F_SFULL)) { ok = false; break; }
         tc_fence_after();
         const bool masked = CAUSAL ? (j == qt) : (j == nkv - 1 && (a.S & 127) != 0);
@@ -467,9 +492,22 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           limit = a.S - 128 * j;
           if (CAUSAL && r + 1 < limit) limit = r + 1;
         }
+        float mo = -INFINITY;  // the other half's partial max (second TMEM pass)
+        uint32_t v0[32], v1[32];
+        if (AXIS_ATTN_FWD_NOXCH) {
+          const uint32_t tSo = tS + (hf ? -64 : 64);
+          tmem_ld32(tSo, v0);
+          tmem_ld32(tSo + 32, v1);
+          tmem_wait_ld();
+          if (masked) {
+            const int lo = limit - (hf ^ 1) * 64;
+            mask_row(v0, 0, lo);
+            mask_row(v1, 32, lo);
+          }
+          mo = fmaxf(row_max32(v0), row_max32(v1));
+        }
         limit -= hf * 64;  // in this half's columns
         // this half of the 128-column row of S in registers (one TMEM pass)
-        uint32_t v0[32], v1[32];
         tmem_ld32(tS, v0);
         tmem_ld32(tS + 32, v1);
         tmem_wait_ld();
@@ -481,13 +519,17 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           mask_row(v0, 0, limit);
           mask_row(v1, 32, limit);
         }
-        // row max: this half's, then the other half's through shared memory
+        // row max: this half's, then the other half's (from TMEM, or through shared memory)
         float mx = fmaxf(row_max32(v0), row_max32(v1));
-        *xslot(X & 1, hf) = mx;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bx);
-        if (!wait_warp<true>(bx, X & 1, abort, F_XCH)) { ok = false; break; }
-        mx = fmaxf(mx, *xslot(X & 1, hf ^ 1));
+        if (AXIS_ATTN_FWD_NOXCH) {
+          mx = fmaxf(mx, mo);
+        } else {
+          *xslot(X & 1, hf) = mx;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bx);
+          if (!wait_warp<true>(bx, X & 1, abort, F_XCH)) { ok = false; break; }
+          mx = fmaxf(mx, *xslot(X & 1, hf ^ 1));
+        }
         const float m_new = fmaxf(m_used, mx * c);
         const bool resc = m_new > m_used + 8.0f;
         float alpha = 1.f;
@@ -499,7 +541,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         // both tiles form one sequence over all items, t0(0) t1(0) t0(1)
         // t1(1) ... (the longer tile's extra phases last); wait until the
         // other tile has finished every phase before this one in it.
-        {
+        if (AXIS_ATTN_FWD_TOKEN) {
           const int need = A_o + (t == 0 ? min(j, n_o) : min(j + 1, n_o));
           if (need > 0 && !wait_warp<true>(bar_tok(t), (need - 1) & 1, abort, F_TOK)) { ok = false; break; }
         }
@@ -511,8 +553,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         uint32_t pk0[16], pk1[16];
         acc = exp_pairs<0, 16>(v0, cc2, nm2, acc, pk0);
         acc = exp_pairs<0, 8>(v1, cc2, nm2, acc, pk1);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_tok(1 - t));
+        if (AXIS_ATTN_FWD_TOKEN) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_tok(1 - t));
+        }
         acc = exp_pairs<8, 8>(v1, cc2, nm2, acc, pk1);
         float rs_lo, rs_hi;
         f2_unpack(acc, rs_lo, rs_hi);
@@ -539,7 +583,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_pfull(t));
+        if (lane == 0 && !(AXIS_ATTN_TEST_DROP_ARRIVE == 1 && J == 0 && t == 0)) mbar_arrive(bar_pfull(t));
       }
       A_o += n_o;
       if (!ok || n_t == 0) continue;

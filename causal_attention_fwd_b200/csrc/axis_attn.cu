@@ -10,6 +10,8 @@
 
 #include "../../include/axis_attn.h"
 #include "attn_bwd.cuh"
+#include "attn_bwd_dq.cuh"
+#include "attn_decode.cuh"
 #include "attn_fwd.cuh"
 
 namespace axis_attn {
@@ -95,17 +97,16 @@ struct WsLayout {
   int S_pad;
 };
 
-// det: one fp32 dQ slice per 128-key tile ([nkv][B*Hq][S][D]) instead of one
-// shared accumulator.
+// det: no dQ accumulator (the deterministic dQ pass keeps dQ in TMEM), so the
+// workspace is the two row sections only.
 WsLayout ws_layout(int B, int Hq, int S, int D, bool det = false) {
   WsLayout w;
   w.S_pad = (S + 127) / 128 * 128;
   const size_t rows = (size_t)B * Hq * w.S_pad;
-  const size_t slices = det ? (size_t)((S + 127) / 128) : 1;
   w.lse2 = 0;
   w.dr = round256(rows * 4);
   w.dqacc = w.dr + round256(rows * 4);
-  w.total = w.dqacc + round256(slices * B * Hq * S * D * 4);
+  w.total = w.dqacc + (det ? 0 : round256((size_t)B * Hq * S * D * 4));
   return w;
 }
 
@@ -142,6 +143,17 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   // persistent: one CTA per SM (the kernel walks its share of the items)
   const unsigned grid = (unsigned)(a.n_items < sm_count(dev) ? a.n_items : sm_count(dev));
   kern<<<grid, FWD_THREADS, FwdCfg<HD>::SMEM, st>>>(mq, mk, mv, a);
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+template <int HD, bool CAUSAL>
+int launch_bwd_dq(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                  const DqArgs& a, cudaStream_t st, int dev) {
+  auto kern = attn_bwd_dq_kernel<HD, CAUSAL>;
+  static bool done[64];
+  if (int rc = set_smem(kern, DqCfg<HD>::SMEM, dev, done)) return rc;
+  const unsigned grid = (unsigned)((a.S + 127) / 128) * a.B * a.Hq;
+  kern<<<grid, DQ_THREADS, DqCfg<HD>::SMEM, st>>>(mq, mk, mv, mdo, a);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
@@ -236,7 +248,7 @@ int run_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, 
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
-// Stage 2: the main kernel; det stores each key tile's dQ tiles into its slice.
+// Stage 2: the main kernel; det: dK, dV only (no dQ accumulator).
 int run_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int Hq,
              int Hkv, int S, int D, float scale, int causal, const WsLayout& w, const WsPtrs& p, bool det,
              cudaStream_t st, int dev) {
@@ -245,9 +257,8 @@ int run_main(const void* q, const void* k, const void* v, const void* dO, void* 
   if (!make_map(&mq, q, B, S, Hq, D, BM) || !make_map(&mdo, dO, B, S, Hq, D, BM) ||
       !make_map(&mk, k, B, S, Hkv, D, 128) || !make_map(&mv, v, B, S, Hkv, D, 128))
     return AXIS_ATTN_ERR_CUDA;
-  const int nkv = (S + 127) / 128;
-  CUtensorMap mdq;
-  if (!make_dq_map(&mdq, p.dqacc, B * Hq * (det ? nkv : 1), S, D)) return AXIS_ATTN_ERR_CUDA;
+  CUtensorMap mdq = {};  // not read by the kernel in the deterministic mode
+  if (!det && !make_dq_map(&mdq, p.dqacc, B * Hq, S, D)) return AXIS_ATTN_ERR_CUDA;
   BwdArgs a;
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);
@@ -261,7 +272,7 @@ int run_main(const void* q, const void* k, const void* v, const void* dO, void* 
   a.S_pad = w.S_pad;
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
-  a.det = det ? 1 : 0;
+  a.no_dq = det ? 1 : 0;
   if (D == 64)
     return causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, mdq, a, st, dev)
                   : launch_bwd_main<64, false>(mq, mk, mv, mdo, mdq, a, st, dev);
@@ -269,18 +280,12 @@ int run_main(const void* q, const void* k, const void* v, const void* dO, void* 
                 : launch_bwd_main<128, false>(mq, mk, mv, mdo, mdq, a, st, dev);
 }
 
-// Stage 3: dQ to bf16 [B,S,Hq,D] (det: the key-tile slices summed in order).
-int run_finalize(void* dq, int B, int Hq, int S, int D, int causal, const WsPtrs& p, bool det, cudaStream_t st) {
+// Stage 3: dQ to bf16 [B,S,Hq,D].
+int run_finalize(void* dq, int B, int Hq, int S, int D, const WsPtrs& p, cudaStream_t st) {
   const size_t n8 = (size_t)B * S * Hq * D / 8;
   const unsigned grid = (unsigned)((n8 + 255) / 256 < 4096 ? (n8 + 255) / 256 : 4096);
   auto* out = static_cast<__nv_bfloat16*>(dq);
-  const int nkv = (S + 127) / 128;
-  if (det) {
-    if (D == 64)
-      attn_bwd_dq_sum_kernel<64><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, nkv, causal, n8);
-    else
-      attn_bwd_dq_sum_kernel<128><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, nkv, causal, n8);
-  } else if (D == 64) {
+  if (D == 64) {
     attn_bwd_dq_convert_kernel<64><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, n8);
   } else {
     attn_bwd_dq_convert_kernel<128><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, n8);
@@ -326,10 +331,36 @@ extern "C" int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, i
   if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
-  return run_finalize(dq, B, Hq, S, D, 1, ws_ptrs(workspace, w), false, static_cast<cudaStream_t>(stream));
+  return run_finalize(dq, B, Hq, S, D, ws_ptrs(workspace, w), static_cast<cudaStream_t>(stream));
 }
 
 namespace {
+
+// Deterministic mode, stage 3: dQ recomputed per 128-row query tile.
+int run_dq_pass(const void* q, const void* k, const void* v, const void* dO, void* dq, int B, int Hq, int Hkv,
+                int S, int D, float scale, int causal, const WsLayout& w, const WsPtrs& p, cudaStream_t st,
+                int dev) {
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, B, S, Hq, D, 128) || !make_map(&mdo, dO, B, S, Hq, D, 128) ||
+      !make_map(&mk, k, B, S, Hkv, D, 128) || !make_map(&mv, v, B, S, Hkv, D, 128))
+    return AXIS_ATTN_ERR_CUDA;
+  DqArgs a;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.nlse2 = p.lse2;
+  a.ndr = p.dr;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.S = S;
+  a.S_pad = w.S_pad;
+  a.scale = scale;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  if (D == 64)
+    return causal ? launch_bwd_dq<64, true>(mq, mk, mv, mdo, a, st, dev)
+                  : launch_bwd_dq<64, false>(mq, mk, mv, mdo, a, st, dev);
+  return causal ? launch_bwd_dq<128, true>(mq, mk, mv, mdo, a, st, dev)
+                : launch_bwd_dq<128, false>(mq, mk, mv, mdo, a, st, dev);
+}
 
 int run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
             void* dk, void* dv, int B, int Hq, int Hkv, int S, int D, float scale, int causal, void* workspace,
@@ -348,7 +379,8 @@ int run_bwd(const void* q, const void* k, const void* v, const void* o, const vo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (int rc = run_prepare(o, dO, lse, B, Hq, S, D, w, p, !det, st)) return rc;
   if (int rc = run_main(q, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, w, p, det, st, dev)) return rc;
-  return run_finalize(dq, B, Hq, S, D, causal, p, det, st);
+  if (det) return run_dq_pass(q, k, v, dO, dq, B, Hq, Hkv, S, D, scale, causal, w, p, st, dev);
+  return run_finalize(dq, B, Hq, S, D, p, st);
 }
 
 }  // namespace
@@ -420,6 +452,134 @@ extern "C" int axis_attn_bwd_noalloc(const void* q, const void* k, const void* v
                        (size_t)AXIS_ATTN_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+// ----------------------------------------------------------------------------
+// Decode step against a paged KV cache.
+
+namespace axis_attn {
+namespace {
+
+bool pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+
+int check_decode_shape(int B, int Hq, int Hkv, int D, int page_size, int max_pages, int num_pages, float scale) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_pages < 1 || num_pages < 1) return AXIS_ATTN_ERR_SHAPE;
+  if (!(std::isfinite(scale) && scale > 0.f)) return AXIS_ATTN_ERR_SHAPE;
+  if (D != 64 && D != 128) return AXIS_ATTN_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 8 || !pow2_in(page_size, 8, 256)) return AXIS_ATTN_ERR_UNSUPPORTED;
+  if ((long long)max_pages * page_size >= (1LL << 30) || (long long)num_pages * page_size >= (1LL << 31) ||
+      (long long)B * max_pages >= (1LL << 31))
+    return AXIS_ATTN_ERR_SHAPE;
+  return AXIS_ATTN_OK;
+}
+
+// Splits of each sequence: at least one full wave of CTAs (two per SM) when the
+// batch is small, at least 256 keys (8 pieces, 2 per compute warp) per split.
+struct DecSplit {
+  int n_splits, keys_per_split;
+};
+DecSplit decode_split(int B, int Hkv, int page_size, int max_pages) {
+  const long long keys = (long long)max_pages * page_size;
+  const long long units = (long long)B * Hkv;
+  long long n = (296 + units - 1) / units;
+  const long long n_max = (keys + 255) / 256;
+  if (n > n_max) n = n_max;
+  if (n < 1) n = 1;
+  long long kps = ((keys + n - 1) / n + 31) / 32 * 32;
+  n = (keys + kps - 1) / kps;
+  return {(int)n, (int)kps};
+}
+
+size_t decode_ws_bytes(int B, int Hq, int D, const DecSplit& sp) {
+  return sp.n_splits > 1 ? (size_t)B * Hq * sp.n_splits * (D + 2) * 4 : 0;
+}
+
+// 3-D map over a paged cache [num_pages * page_size rows][Hkv][D] (bf16):
+// dims (D, Hkv, rows), box (64, 1, min(page_size, 32)), 128-byte swizzle.
+bool make_cache_map(CUtensorMap* map, const void* ptr, int rows, int Hkv, int D, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int HD, int GM>
+int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev) {
+  auto kern = attn_decode_kernel<HD, GM>;
+  static bool done[64];
+  if (int rc = set_smem(kern, DecCfg<HD>::SMEM, dev, done)) return rc;
+  const unsigned grid = (unsigned)(a.B * a.Hkv * a.n_splits);
+  kern<<<grid, DEC_THREADS, DecCfg<HD>::SMEM, st>>>(mk, mv, a);
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+template <int HD>
+int launch_decode_g(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev) {
+  if (a.G <= 2) return launch_decode<HD, 2>(mk, mv, a, st, dev);
+  if (a.G <= 4) return launch_decode<HD, 4>(mk, mv, a, st, dev);
+  return launch_decode<HD, 8>(mk, mv, a, st, dev);
+}
+
+}  // namespace
+}  // namespace axis_attn
+
+extern "C" size_t axis_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int page_size, int max_pages) {
+  if (check_decode_shape(B, Hq, Hkv, D, page_size, max_pages, 1, 1.f) != AXIS_ATTN_OK) return 0;
+  return decode_ws_bytes(B, Hq, D, decode_split(B, Hkv, page_size, max_pages));
+}
+
+extern "C" int axis_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                                const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
+                                int page_size, int max_pages, int num_pages, float scale, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !o || !lse) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return AXIS_ATTN_ERR_ALIGN;
+  if (int rc = check_decode_shape(B, Hq, Hkv, D, page_size, max_pages, num_pages, scale)) return rc;
+  const DecSplit sp = decode_split(B, Hkv, page_size, max_pages);
+  const size_t need = decode_ws_bytes(B, Hq, D, sp);
+  if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need))
+    return AXIS_ATTN_ERR_WORKSPACE;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  CUtensorMap mk, mv;
+  const int box_rows = page_size < 32 ? page_size : 32;
+  if (!make_cache_map(&mk, k_cache, num_pages * page_size, Hkv, D, box_rows) ||
+      !make_cache_map(&mv, v_cache, num_pages * page_size, Hkv, D, box_rows))
+    return AXIS_ATTN_ERR_CUDA;
+  DecArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.part = static_cast<float*>(workspace);
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = Hq / Hkv;
+  a.page_size = page_size;
+  a.max_pages = max_pages;
+  a.num_pages = num_pages;
+  a.keys_per_split = sp.keys_per_split;
+  a.n_splits = sp.n_splits;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = D == 64 ? launch_decode_g<64>(mk, mv, a, st, dev) : launch_decode_g<128>(mk, mv, a, st, dev);
+  if (rc || sp.n_splits == 1) return rc;
+  const int rows = B * Hq;
+  const unsigned grid = (unsigned)((rows + 7) / 8 < 4096 ? (rows + 7) / 8 : 4096);
+  if (D == 64)
+    attn_decode_combine_kernel<64><<<grid, 256, 0, st>>>(a.part, a.o, lse, rows, sp.n_splits);
+  else
+    attn_decode_combine_kernel<128><<<grid, 256, 0, st>>>(a.part, a.o, lse, rows, sp.n_splits);
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
 static unsigned int g_last_status_word;
 
 extern "C" unsigned int axis_attn_last_status_word(void) { return g_last_status_word; }
@@ -430,7 +590,8 @@ extern "C" int axis_attn_get_status(void* stream) {
   if (cudaMemcpyFromSymbol(&st, g_status, sizeof(st)) != cudaSuccess) return AXIS_ATTN_ERR_CUDA;
   g_last_status_word = st;
   if (st != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return AXIS_ATTN_ERR_CUDA;
-  if (st != 0) return AXIS_ATTN_ERR_TIMEOUT;
+  if (st & 1u) return AXIS_ATTN_ERR_TIMEOUT;
+  if (st & 2u) return AXIS_ATTN_ERR_INDEX;
   return cudaGetLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
@@ -444,6 +605,7 @@ extern "C" const char* axis_attn_strerror(int code) {
     case AXIS_ATTN_ERR_WORKSPACE: return "workspace NULL, not 256-byte aligned, or too small";
     case AXIS_ATTN_ERR_CUDA: return "CUDA runtime or driver error";
     case AXIS_ATTN_ERR_TIMEOUT: return "a device-side wait timed out";
+    case AXIS_ATTN_ERR_INDEX: return "a device-side index (page table entry or sequence length) was out of range";
     default: return "unknown status";
   }
 }

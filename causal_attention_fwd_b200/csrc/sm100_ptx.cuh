@@ -14,35 +14,74 @@
 namespace axis_attn {
 
 // ------------------------------------------------------------------ status
-// Device status word.  Bit 0: a bounded wait ran out.  Bits 8..15: the wait
-// site of the first such event (for debugging).  Read and cleared by
-// axis_attn_get_status().
+// Device status word.  Bit 0: a bounded wait ran out.  Bit 1: a device-side
+// index (a page of the decode step's block table, a sequence length) was out
+// of range and was not used.  Bits 8..15: the wait site of the first timeout
+// (for debugging).  Read and cleared by axis_attn_get_status().
 __device__ unsigned int g_status;
+// Number of bounded waits that have ever run out on this device (never
+// cleared).  A launch snapshots it at entry; a change during the launch means
+// that one of its own CTAs gave up, and the others stop waiting.  A timeout
+// left over from an earlier launch is therefore never mistaken for one of the
+// current launch, whether or not axis_attn_get_status() has been called since.
+__device__ unsigned int g_timeouts;
 
 // Upper bound on any single wait inside a kernel, in SM clock cycles (2^31,
 // about 1.1 s at 1.965 GHz).  No wait in a correct run comes near it: every
-// wait here is on work that the same CTA issued.  Once any CTA has timed out
-// (g_status bit 0), the other CTAs stop waiting at their next status check,
-// so a faulty launch ends quickly instead of timing out CTA by CTA.  The status
-// stays set until axis_attn_get_status() clears it.
+// wait here is on work that the same CTA issued.  Once any CTA of a launch has
+// timed out, the other CTAs of that launch stop waiting at their next check,
+// so a faulty launch ends quickly instead of timing out CTA by CTA.
 //
 // The polling loops below touch only shared memory and the SM's own cycle
-// counter on each pass; the global status word is read about every 2^16
-// cycles.  (Reading global memory or %globaltimer on every pass would make a
-// waiting thread notice a completed barrier up to a global round trip late.)
+// counter on each pass; the global counter is read about every 2^16 cycles.
+// (Reading global memory or %globaltimer on every pass would make a waiting
+// thread notice a completed barrier up to a global round trip late.)
 #ifndef AXIS_ATTN_WAIT_LIMIT_CYCLES
 #define AXIS_ATTN_WAIT_LIMIT_CYCLES (1ull << 31)
 #endif
 #define AXIS_ATTN_STATUS_CHECK_CYCLES (1ull << 16)
 
+// Test-only builds: AXIS_ATTN_TEST_DROP_ARRIVE = 1 makes the softmax warps of
+// the forward's first query tile skip their first "P is in TMEM" arrive, 2
+// makes the backward's compute warps skip their first "P^T, dS^T written"
+// arrive.  The wait for that barrier phase can then never complete (the next
+// arrivals come only after it), and AXIS_ATTN_TEST_SHORT_SITE gives that one
+// wait site a short limit (AXIS_ATTN_TEST_SHORT_LIMIT cycles), so the failure
+// path runs: the waiting MMA issuer records a timeout at its site, the other
+// roles of the CTA stop on the abort flag, the other CTAs on the changed
+// timeout count, copies and MMAs in flight drain, TMEM is freed, the kernel
+// returns.  All three are 0 in every normal build.
+#ifndef AXIS_ATTN_TEST_DROP_ARRIVE
+#define AXIS_ATTN_TEST_DROP_ARRIVE 0
+#endif
+#ifndef AXIS_ATTN_TEST_SHORT_SITE
+#define AXIS_ATTN_TEST_SHORT_SITE 0
+#endif
+#ifndef AXIS_ATTN_TEST_SHORT_LIMIT
+#define AXIS_ATTN_TEST_SHORT_LIMIT (1ull << 22)
+#endif
+
+// Per-CTA wait control in shared memory: `abort` is raised by the first role
+// that gives up (the others see it on their next poll); `epoch` is the
+// launch's snapshot of g_timeouts; `watch` = 0 for drain waits (on TMA copies
+// or MMAs already issued, which complete whatever other CTAs do), which
+// therefore ignore the other CTAs.
+struct WaitCtl {
+  int abort;
+  unsigned int epoch;
+  unsigned int watch;
+};
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ bool other_cta_timed_out() {
-  return (*reinterpret_cast<volatile unsigned int*>(&g_status) & 1u) != 0;
+// Called by one thread while the CTA initialises its barriers.
+__device__ __forceinline__ void wait_ctl_init(volatile WaitCtl* c) {
+  c->abort = 0;
+  c->epoch = *reinterpret_cast<volatile unsigned int*>(&g_timeouts);
+  c->watch = 1;
 }
-
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -76,36 +115,42 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase of `bar` with parity `parity` has completed.  Gives up
-// when `*abort` becomes non-zero (another role of the CTA gave up), when
-// another CTA has timed out, or after AXIS_ATTN_WAIT_LIMIT_CYCLES; in the
-// last case it raises `*abort` and records the failure in g_status.  Returns
+// when `abort->abort` becomes non-zero (another role of the CTA gave up), when
+// another CTA of the launch has timed out (unless abort->watch is 0), or after
+// AXIS_ATTN_WAIT_LIMIT_CYCLES; in the last case it raises `abort->abort` and
+// records the failure in g_status and g_timeouts.  Returns
 // true when the phase completed.  Called by a single thread, or by all lanes
 // of a warp (see wait_warp).  The poll loop reads only the barrier, the
 // 32-bit SM clock and the abort flag; try_wait suspends the thread in
 // hardware between polls.
-__device__ __forceinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, volatile int* abort, int site) {
+__device__ __forceinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, volatile WaitCtl* abort, int site) {
   const uint32_t t0 = (uint32_t)clock();
   uint32_t last = t0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
+    if (abort->abort) return false;
     const uint32_t now = (uint32_t)clock();
     if (now - last > AXIS_ATTN_STATUS_CHECK_CYCLES) {
       last = now;
-      if (other_cta_timed_out()) {  // results are void already: stop waiting
-        *abort = 1;
+      if (abort->watch && *reinterpret_cast<volatile unsigned int*>(&g_timeouts) != abort->epoch) {
+        abort->abort = 1;  // another CTA of this launch gave up: results are void already
         return false;
       }
-      if (now - t0 > AXIS_ATTN_WAIT_LIMIT_CYCLES) {
-        *abort = 1;
-        atomicOr(&g_status, 1u | ((unsigned)(site & 0xff) << 8));
+      const unsigned long long limit = (AXIS_ATTN_TEST_SHORT_SITE != 0 && site == AXIS_ATTN_TEST_SHORT_SITE)
+                                           ? AXIS_ATTN_TEST_SHORT_LIMIT
+                                           : AXIS_ATTN_WAIT_LIMIT_CYCLES;
+      if (now - t0 > limit) {
+        abort->abort = 1;
+        // the first timeout since the report was last cleared names its site
+        if ((atomicOr(&g_status, 1u) & 1u) == 0) atomicOr(&g_status, (unsigned)(site & 0xff) << 8);
+        atomicAdd(&g_timeouts, 1u);
         return false;
       }
     }
   }
 }
 
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort, int site) {
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile WaitCtl* abort, int site) {
   return mbar_wait_loop(bar, parity, abort, site);
 }
 
@@ -113,7 +158,7 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
 // code at each call site, but the compiler saves the caller's live registers
 // around the call) or inline (INL = true: no call, more code).
 template <bool INL = false>
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile WaitCtl* abort,
                                                   int site) {
   if (mbar_try_wait(bar, parity)) return true;
   return INL ? mbar_wait_loop(bar, parity, abort, site) : mbar_wait_slow(bar, parity, abort, site);
@@ -123,7 +168,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 // all lanes saw the phase complete, so warp-collective instructions that
 // follow are never reached by a partial warp.
 template <bool INL = false>
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort,
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile WaitCtl* abort,
                                           int site) {
   const bool ok = mbar_wait_bounded<INL>(bar, parity, abort, site);
   return __all_sync(0xffffffffu, ok);
@@ -144,6 +189,16 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 3-D tiled load (coordinates innermost first), completion counted in bytes on `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
 // L2 prefetch of a 4-D tile (no shared-memory destination, no completion).
 __device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
   asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global [%0, {%1, %2, %3, %4}];" ::"l"(
@@ -157,14 +212,6 @@ __device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int c0, 
 // Completion is tracked by bulk groups of the issuing thread.
 __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
   asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(src), "r"(c0), "r"(c1), "r"(c2)
-               : "memory");
-}
-// 3-D tiled store from shared memory (bulk-group completion).  Elements of
-// the box that lie past the tensor's extent are not written.
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
                "r"(src), "r"(c0), "r"(c1), "r"(c2)
                : "memory");
@@ -375,6 +422,44 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+// Round-to-nearest packed add (explicit .rn: the magic-number rounding below
+// must not be contracted with a neighbouring multiply).
+__device__ __forceinline__ uint64_t f2_add_rn(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of fp32 values on the FP32 and integer pipes instead of the
+// MUFU: x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low
+// mantissa bits) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose
+// coefficients are the fp32-rounded least-maximum-relative-error fit on
+// [-1/2, 1/2] by the Remez exchange (exp2_fit.py in the package reproduces
+// them); n is added to the exponent field with one integer shift-add (the
+// magic number's own bits shift out).  Relative error <= 7.5e-5 for
+// -125 <= x <= 64 (measured on the fp32 evaluation), mean +5e-6.  x is
+// clamped at -126 first, so every smaller x, -inf included, gives 2^-126
+// (1.2e-38) instead of 0: below the fp32 resolution of any sum or product it
+// enters here.
+constexpr float EXP2_C0 = 0.999928057f, EXP2_C1 = 0.693260968f, EXP2_C2 = 0.242611125f,
+                EXP2_C3 = 0.0551716685f;
+__device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t x = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = f2_add_rn(x, f2_pack(12582912.f, 12582912.f));
+  const uint64_t n = f2_add_rn(t, f2_pack(-12582912.f, -12582912.f));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f2_pack(EXP2_C3, EXP2_C3), f, f2_pack(EXP2_C2, EXP2_C2));
+  p = f2_fma(p, f, f2_pack(EXP2_C1, EXP2_C1));
+  p = f2_fma(p, f, f2_pack(EXP2_C0, EXP2_C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

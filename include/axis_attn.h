@@ -57,7 +57,8 @@ typedef enum {
     AXIS_ATTN_ERR_UNSUPPORTED = 4, /* D not in {64,128}, or not a CC 10.0 device */
     AXIS_ATTN_ERR_WORKSPACE = 5,   /* workspace NULL, misaligned or too small */
     AXIS_ATTN_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed */
-    AXIS_ATTN_ERR_TIMEOUT = 7      /* a device-side wait ran out (see above) */
+    AXIS_ATTN_ERR_TIMEOUT = 7,     /* a device-side wait ran out (see above) */
+    AXIS_ATTN_ERR_INDEX = 8        /* a device-side index (decode page table, length) was out of range */
 } axis_attn_status;
 
 /*
@@ -124,19 +125,23 @@ int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, int D, void*
  * the training step; with the ordinary backward, dQ is the one output whose
  * fp32 additions happen in a run-dependent order.
  *
- * How: every 128-key tile writes its dQ contribution into its own fp32 slice
- * of the workspace, and the last stage adds the slices of each row in the
- * fixed order of the key tiles.  dk and dv take no cross-tile additions in
- * either mode.  Results agree with axis_attn_bwd() to rounding (the same
- * products, summed in another order).
+ * How: the main kernel computes dK and dV only (they take no cross-CTA
+ * additions in either mode), and a separate pass recomputes, per 128-row
+ * query tile, S = Q K^T, P and dS = P (dO V^T - Dr) for every key tile the
+ * rows see and accumulates dQ = scale * sum_j dS_j K_j on chip in the fixed
+ * order of the key tiles.  The extra cost is two more MMAs per tile (S and dP
+ * are formed twice); the workspace holds only the per-row LSE and Dr, so
+ * memory stays flat as the sequence grows (the Axis page, feature list).
+ * Results agree with axis_attn_bwd() to rounding (the same products, summed
+ * in another order); dk and dv are bitwise the same as axis_attn_bwd()'s.
  *
- * Arguments, layouts, ownership and errors as for axis_attn_bwd(), with a
- * larger workspace:
- *   axis_attn_bwd_det_workspace_bytes() = the row statistics of
- *   axis_attn_bwd() + 4 * ceil(S / 128) * B * Hq * S * D bytes
- * (about 1.07 GB for B=4, Hq=32, S=2048, D=64; it grows as S^2).  A workspace
- * shorter than that returns AXIS_ATTN_ERR_WORKSPACE and launches nothing.
- * Returns 0 from the size function for invalid sizes.
+ * Arguments, layouts, ownership and errors as for axis_attn_bwd(), with the
+ * smaller workspace
+ *   axis_attn_bwd_det_workspace_bytes() = 2 * round256(4 * B * Hq * S_pad),
+ *   S_pad = ceil(S / 128) * 128
+ * (about 2.1 MB for B=4, Hq=32, S=2048).  A workspace shorter than that
+ * returns AXIS_ATTN_ERR_WORKSPACE and launches nothing.  Returns 0 from the
+ * size function for invalid sizes.
  */
 size_t axis_attn_bwd_det_workspace_bytes(int B, int Hq, int Hkv, int S, int D);
 int axis_attn_bwd_det(const void* q, const void* k, const void* v, const void* o, const void* dO,
@@ -176,9 +181,46 @@ int axis_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
                           void* stream);
 
 /*
+ * Decode step against a paged KV cache: for each sequence b, the new token's
+ * query row attends to every key cached for b (itself included, so no mask is
+ * needed).  This is the per-token step of the axiomlm inference engine
+ * (axiomlm page, PyPI: Key Features, "State-cached Key-Value (KV) decode
+ * engine achieving O(1) step latency"; Quick Start section 4, "the Paged
+ * KV-Cache engine"), with its GQA heads (Key Features, "4-head Grouped-Query
+ * Attention").  For query head h (kv head h / (Hq / Hkv)):
+ *   o[b,h,:] = sum_j P_j V_j,  P = softmax_j(scale * <q[b,h,:], K_j>),  j < seq_lens[b]
+ *   lse[b,h] = ln sum_j exp(scale * <q[b,h,:], K_j>)
+ *
+ *  - q, o: [B, Hq, D] bf16 (one row per sequence); lse: [B, Hq] fp32.
+ *  - k_cache, v_cache: [num_pages, page_size, Hkv, D] bf16, a pool of pages.
+ *    Position j of sequence b is row j % page_size of page
+ *    block_table[b * max_pages + j / page_size].
+ *  - block_table: [B, max_pages] int32; seq_lens: [B] int32, the number of
+ *    cached tokens of each sequence including the new one.  Both are DEVICE
+ *    arrays read by the kernel: an entry outside [0, num_pages) that a
+ *    sequence's length reaches, or a length outside [1, max_pages*page_size],
+ *    is never used for a memory access; the affected keys are left out and
+ *    axis_attn_get_status() reports AXIS_ATTN_ERR_INDEX.
+ *  - Requirements: D in {64, 128}; Hq / Hkv <= 8; page_size a power of two in
+ *    [8, 256]; B, max_pages, num_pages >= 1; scale finite and > 0; 16-byte
+ *    aligned q, caches, o, lse; 4-byte aligned block_table, seq_lens.
+ *  - workspace: axis_attn_decode_workspace_bytes() bytes (0 is possible:
+ *    then workspace may be NULL), 256-byte aligned, caller-owned; long
+ *    sequences at small batch are split over several CTAs whose partial
+ *    results meet there.  Calls that overlap on the GPU must not share it.
+ *  - The kernel is HBM-bound: every cached key and value is read once.
+ */
+size_t axis_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int page_size, int max_pages);
+int axis_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                     const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
+                     int page_size, int max_pages, int num_pages, float scale, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then returns AXIS_ATTN_ERR_TIMEOUT if any kernel of
  * this library on the current device has reported a timed-out device wait since
- * the last call (and clears that report), AXIS_ATTN_ERR_CUDA if the CUDA
+ * the last call, else AXIS_ATTN_ERR_INDEX if a decode step met an out-of-range
+ * device-side index (and clears those reports), AXIS_ATTN_ERR_CUDA if the CUDA
  * context holds an error, else AXIS_ATTN_OK.  For tests and debugging: it
  * blocks the host.  A launch that timed out leaves its outputs undefined; it
  * does not affect later launches, whether or not this function is called in
@@ -189,8 +231,9 @@ int axis_attn_get_status(void* stream);
 /*
  * Diagnostics: the raw device status word that the last axis_attn_get_status()
  * call read before clearing it (0 if none was set).  Bit 0: a wait timed out;
- * bits 8..15: the wait site that first did (1..10: forward kernel, 21..32:
- * backward main kernel).
+ * bit 1: a decode index was out of range; bits 8..15: the wait site that first
+ * timed out (1..13: forward kernel, 21..32: backward main kernel, 41..42:
+ * decode kernel).
  */
 unsigned int axis_attn_last_status_word(void);
 

@@ -41,8 +41,8 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_strerror_covers_every_status(lib):
-    texts = {aa.axis_attn_strerror(c) for c in range(8)}
-    assert len(texts) == 8 and "ok" in texts
+    texts = {aa.axis_attn_strerror(c) for c in range(9)}
+    assert len(texts) == 9 and "ok" in texts
     assert aa.axis_attn_strerror(99) == "unknown status"
 
 
@@ -58,15 +58,16 @@ def test_workspace_bytes(lib):
 
 
 def test_det_workspace_bytes(lib):
-    # the same row sections + one fp32 dQ slice per 128-key tile
+    # only the two row sections: dQ stays on chip in the deterministic pass
     B, Hq, Hkv, S, D = 2, 12, 4, 1000, 64
     rows = B * Hq * 1024
     r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    nkv = (S + 127) // 128
-    assert aa.axis_attn_bwd_det_workspace_bytes(B, Hq, Hkv, S, D) == 2 * r256(rows * 4) + r256(
-        nkv * B * Hq * S * D * 4)
-    # the header's example: B=4, Hq=32, S=2048, D=64 needs about 1.07 GB
-    assert abs(aa.axis_attn_bwd_det_workspace_bytes(4, 32, 8, 2048, 64) / 1.07e9 - 1) < 0.01
+    assert aa.axis_attn_bwd_det_workspace_bytes(B, Hq, Hkv, S, D) == 2 * r256(rows * 4)
+    # the header's example: B=4, Hq=32, S=2048 needs about 2.1 MB, flat in D
+    assert aa.axis_attn_bwd_det_workspace_bytes(4, 32, 8, 2048, 64) == 2 * r256(4 * 32 * 2048 * 4)
+    assert aa.axis_attn_bwd_det_workspace_bytes(4, 32, 8, 2048, 128) == 2 * r256(4 * 32 * 2048 * 4)
+    # the longest workload: 1 x 16 heads x 32768 -> 4 MB (no S^2 term)
+    assert aa.axis_attn_bwd_det_workspace_bytes(1, 16, 16, 32768, 128) == 2 * r256(16 * 32768 * 4)
     assert aa.axis_attn_bwd_det_workspace_bytes(1, 3, 2, 128, 64) == 0
     assert aa.axis_attn_bwd_det_workspace_bytes(1, 1, 1, 128, 96) == 0
 
@@ -114,16 +115,15 @@ def test_bwd_rejects(lib, over, code):
 @pytest.mark.parametrize("over,code", [
     (dict(dO=None), 1), (dict(dq=None), 1), (dict(dk=A + 8), 2), (dict(S=0), 3), (dict(D=80), 4),
     (dict(workspace=None), 5), (dict(workspace=A + 16), 5),
-    # enough for axis_attn_bwd (about 0.5 MB here) but not for the key-tile slices (about 4.1 MB)
-    (dict(S=1000, workspace_bytes=3 << 20), 5),
+    # one byte short of the two row sections
+    (dict(S=1000, workspace_bytes=2 * 1024 * 2 * 4 - 1), 5),
 ])
 def test_bwd_det_rejects(lib, over, code):
     args = dict(q=A, k=A, v=A, o=A, dO=A, lse=A, dq=A, dk=A, dv=A, B=1, Hq=2, Hkv=1, S=128, D=64,
                 scale=0.125, causal=1, workspace=A, workspace_bytes=1 << 30, stream=None)
     args.update(over)
     if "S" in over and over["S"] == 1000:
-        assert aa.axis_attn_bwd_workspace_bytes(1, 2, 1, 1000, 64) < args["workspace_bytes"]
-        assert aa.axis_attn_bwd_det_workspace_bytes(1, 2, 1, 1000, 64) > args["workspace_bytes"]
+        assert aa.axis_attn_bwd_det_workspace_bytes(1, 2, 1, 1000, 64) == args["workspace_bytes"] + 1
     assert aa.axis_attn_bwd_det(*args.values()) == code
 
 
@@ -154,3 +154,32 @@ def test_valid_args_without_gpu_report_cuda_error(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert _fwd() in (4, 6)
+
+
+def _dec(**over):
+    args = dict(q=A, k_cache=A, v_cache=A, block_table=A, seq_lens=A, o=A, lse=A, B=1, Hq=32, Hkv=8, D=128,
+                page_size=64, max_pages=128, num_pages=128, scale=0.088, workspace=A, workspace_bytes=1 << 30,
+                stream=None)
+    args.update(over)
+    return aa.axis_attn_decode(*args.values())
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), 1), (dict(block_table=None), 1), (dict(seq_lens=None), 1), (dict(lse=None), 1),
+    (dict(k_cache=A + 8), 2), (dict(o=A + 2), 2), (dict(block_table=A + 2), 2), (dict(seq_lens=A + 1), 2),
+    (dict(B=0), 3), (dict(Hq=12, Hkv=5), 3), (dict(max_pages=0), 3), (dict(num_pages=0), 3),
+    (dict(scale=0.0), 3), (dict(scale=float("nan")), 3),
+    (dict(D=96), 4), (dict(Hq=72, Hkv=8), 4), (dict(page_size=24), 4), (dict(page_size=4), 4),
+    (dict(page_size=512), 4),
+    (dict(workspace=None), 5), (dict(workspace=A + 16), 5), (dict(workspace_bytes=100), 5),
+])
+def test_decode_rejects(lib, over, code):
+    assert _dec(**over) == code
+
+
+def test_decode_workspace_bytes(lib):
+    # B=1, 8 kv heads, 8192 keys: ceil(296 / 8) = 37 splits wanted, at least 256 keys each -> 32 splits
+    n = aa.axis_attn_decode_workspace_bytes(1, 32, 8, 128, 64, 128)
+    assert n == 1 * 32 * 32 * (128 + 2) * 4
+    assert aa.axis_attn_decode_workspace_bytes(64, 32, 8, 128, 16, 38) == 0  # 512 units: no split
+    assert aa.axis_attn_decode_workspace_bytes(1, 32, 8, 96, 64, 128) == 0

@@ -1,0 +1,124 @@
+"""GPU parity of the decode step (axis_attn_decode) against the oracle.
+
+The oracle reads a contiguous cache [B, Smax, Hkv, D]; the test scatters the
+same rows into a shuffled pool of pages, fills the block table (entries past a
+sequence's last page hold -1, which the kernel must never touch) and compares
+O and LSE with the tolerances of the other tests (O max abs <= 1e-2, LSE max
+abs <= 1e-4).  Cases cover both head dims, GQA groups 1..8 (including 3),
+page sizes 8..256, ragged lengths (1, around page and piece edges), batches
+that take the split-K path and batches that do not, and bad device-side
+indices, which must be reported as AXIS_ATTN_ERR_INDEX without an access.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import causal_attention_fwd_b200 as aa
+
+pytestmark = pytest.mark.gpu
+
+TOL_O, TOL_LSE = 1e-2, 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from causal_attention_fwd_b200 import build
+
+    build.build()
+
+
+def paged(k, v, lens, page_size, seed, extra_pages=3):
+    """Scatter contiguous caches [B, Smax, Hkv, D] into a shuffled page pool."""
+    B, Smax, Hkv, D = k.shape
+    max_pages = (Smax + page_size - 1) // page_size
+    need = [(int(L) + page_size - 1) // page_size for L in lens]
+    num_pages = sum(need) + extra_pages
+    order = np.random.default_rng(seed).permutation(num_pages)
+    kc = torch.zeros((num_pages, page_size, Hkv, D), dtype=k.dtype)
+    vc = torch.zeros_like(kc)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    n = 0
+    for b in range(B):
+        for p in range(need[b]):
+            page = int(order[n])
+            n += 1
+            table[b, p] = page
+            rows = slice(p * page_size, min((p + 1) * page_size, int(lens[b])))
+            cnt = rows.stop - rows.start
+            kc[page, :cnt] = k[b, rows]
+            vc[page, :cnt] = v[b, rows]
+    return kc, vc, table, num_pages
+
+
+def run_case(oracle_mod, B, Hq, Hkv, D, Smax, page_size, lens, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((B, Hq, D), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
+    lens = np.asarray(lens, np.int32)
+    sc = 1.0 / math.sqrt(D)
+    kc, vc, table, num_pages = paged(k, v, lens, page_size, seed)
+    dev = torch.device("cuda:0")
+    o, lse = aa.attention_decode(q.to(dev), kc.to(dev), vc.to(dev), table.to(dev),
+                                 torch.from_numpy(lens).to(dev), scale=sc)
+    aa.check_status()
+    ro, rl = oracle_mod.attn_decode(q, k, v, lens, sc)
+    eo = float((o.cpu().double() - torch.from_numpy(ro)).abs().max())
+    el = float((lse.cpu().double() - torch.from_numpy(rl)).abs().max())
+    return eo, el
+
+
+CASES = [
+    # B, Hq, Hkv, D, Smax, page_size, lens
+    (1, 1, 1, 64, 1, 8, [1]),
+    (3, 4, 4, 64, 100, 16, [1, 31, 100]),
+    (2, 12, 4, 64, 1024, 16, [1024, 517]),           # the axiomlm model's heads and block size
+    (4, 8, 1, 128, 300, 32, [32, 33, 64, 299]),
+    (2, 6, 2, 128, 700, 64, [700, 65]),
+    (5, 16, 2, 64, 257, 256, [256, 257, 1, 128, 200]),
+    (1, 32, 8, 128, 8192, 64, [8192]),               # one long sequence: split-K
+    (2, 24, 8, 64, 5000, 8, [4999, 3]),               # G = 3, small pages, split-K
+    (64, 32, 8, 128, 600, 16, list(range(9, 9 + 64 * 9, 9))),  # many sequences: no split
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D,Smax,ps,lens", CASES)
+def test_decode_matches_oracle(oracle_mod, B, Hq, Hkv, D, Smax, ps, lens):
+    eo, el = run_case(oracle_mod, B, Hq, Hkv, D, Smax, ps, lens, seed=3000 + B + Hq + D + Smax + ps)
+    print(f"B{B} Hq{Hq} Hkv{Hkv} D{D} S{Smax} ps{ps}: O {eo:.2e} LSE {el:.2e}")
+    assert eo <= TOL_O and el <= TOL_LSE
+
+
+def test_decode_workspace_is_split_dependent():
+    # one sequence of 8192 keys over 8 kv heads is split; 64 x 8 units are not
+    assert aa.axis_attn_decode_workspace_bytes(1, 32, 8, 128, 64, 128) > 0
+    assert aa.axis_attn_decode_workspace_bytes(64, 32, 8, 128, 16, 38) == 0
+    assert aa.axis_attn_decode_workspace_bytes(1, 32, 8, 96, 64, 128) == 0  # unsupported D
+
+
+def test_decode_bad_indices_are_reported_not_used(oracle_mod):
+    B, Hq, Hkv, D, Smax, ps = 2, 4, 2, 64, 64, 16
+    g = torch.Generator().manual_seed(9)
+    q = torch.randn((B, Hq, D), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
+    lens = np.array([64, 40], np.int32)
+    kc, vc, table, num_pages = paged(k, v, lens, ps, 9)
+    dev = torch.device("cuda:0")
+    args = [t.to(dev) for t in (q, kc, vc)]
+    bad = table.clone()
+    bad[1, 1] = num_pages + 1000  # inside sequence 1's length
+    aa.attention_decode(*args, bad.to(dev), torch.from_numpy(lens).to(dev), scale=D ** -0.5)
+    assert aa.axis_attn_get_status(aa.binding._stream(None)) == 8  # AXIS_ATTN_ERR_INDEX
+    bad_len = torch.tensor([64, 10 ** 6], dtype=torch.int32)
+    aa.attention_decode(*args, table.to(dev), bad_len.to(dev), scale=D ** -0.5)
+    assert aa.axis_attn_get_status(aa.binding._stream(None)) == 8
+    # the same call with good indices is exact afterwards
+    o, lse = aa.attention_decode(*args, table.to(dev), torch.from_numpy(lens).to(dev), scale=D ** -0.5)
+    aa.check_status()
+    ro, rl = oracle_mod.attn_decode(q, k, v, lens, D ** -0.5)
+    assert float((o.cpu().double() - torch.from_numpy(ro)).abs().max()) <= TOL_O
