@@ -389,6 +389,109 @@ def shard_problem(aa, w, seed: int, dev, det: bool, world: int, rank: int):
     return Problem(aa, wl, seed, dev, det, host=host)
 
 
+def time_rope(aa, w, seed, dev, steps, flush, p_meas):
+    """The headline step with the rotary embedding fused (axis_attn_fwd_rope +
+    axis_attn_bwd_rope): fwd / bwd TFLOP/s counting the same attention FLOPs
+    (the rotations add no MMA work), device time per call with CUDA events."""
+    import torch
+
+    from causal_attention_fwd_b200.synthetic import workload_inputs
+
+    q, k, v, do = (t.to(dev) for t in workload_inputs(w, seed=seed))
+    B, Hq, Hkv, S, D = w.B, w.Hq, w.Hkv, w.S, w.D
+    cs = aa.rope_table(S, D, 10000.0, device=dev)
+    o, lse = torch.empty_like(q), torch.empty((B, Hq, S), device=dev, dtype=torch.float32)
+    k_rot, dq, dk, dv = torch.empty_like(k), torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsb = aa.axis_attn_bwd_rope_workspace_bytes(B, Hq, Hkv, S, D, 0)
+    ws = torch.empty(wsb, device=dev, dtype=torch.uint8)
+    st = torch.cuda.current_stream(dev)
+    import ctypes
+
+    sp = ctypes.c_void_p(st.cuda_stream)
+
+    def fwd():
+        rc = aa.axis_attn_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), cs.data_ptr(), o.data_ptr(),
+                                   lse.data_ptr(), k_rot.data_ptr(), B, Hq, Hkv, S, D, w.scale, int(w.causal), sp)
+        if rc:
+            raise aa.AxisAttnError(rc, "axis_attn_fwd_rope")
+
+    def bwd():
+        rc = aa.axis_attn_bwd_rope(q.data_ptr(), k_rot.data_ptr(), v.data_ptr(), cs.data_ptr(), o.data_ptr(),
+                                   do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq,
+                                   Hkv, S, D, w.scale, int(w.causal), 0, ws.data_ptr(), wsb, sp)
+        if rc:
+            raise aa.AxisAttnError(rc, "axis_attn_bwd_rope")
+
+    ev = []
+    for n in range(3 + steps):
+        flush.fill_(n & 0xFF)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(st)
+        fwd()
+        e[1].record(st)
+        bwd()
+        e[2].record(st)
+        if n >= 3:
+            ev.append(e)
+    torch.cuda.synchronize()
+    aa.check_status(st)
+    f_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev)
+    b_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / len(ev)
+    fwd_tf, bwd_tf = w.fwd_flops / f_ms / 1e9, w.bwd_flops / b_ms / 1e9
+    return {"fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf, "fwd_ms": f_ms, "bwd_ms": b_ms, "steps": steps,
+            "fwd_frac_of_measured": fwd_tf / p_meas, "bwd_frac_of_measured": bwd_tf / p_meas,
+            "note": "fwd: K rotated once by a prologue kernel, Q tiles rotated in shared memory; bwd: Q rotated "
+                    "once into the workspace, the transposed rotation fused into the dQ finalize and the dK "
+                    "epilogue; times include the rotations"}
+
+
+# Decode workloads: one new token per sequence against a paged KV cache of
+# `ctx` tokens (the axiomlm model's heads and block size; an 8B-class model).
+DECODE = {
+    "decode_gpt2s_gqa": dict(B=256, Hq=12, Hkv=4, D=64, ctx=1024, page=16),
+    "decode_llm8b_gqa": dict(B=32, Hq=32, Hkv=8, D=128, ctx=8192, page=64),
+}
+
+
+def time_decode(aa, name, dev, steps, flush, hbm_gbs):
+    """Decode step timing: HBM GB/s of the cache bytes every call must read
+    (K and V of every cached token, plus q and o), against the measured copy
+    bandwidth."""
+    import torch
+
+    c = DECODE[name]
+    B, Hq, Hkv, D, ctx, page = c["B"], c["Hq"], c["Hkv"], c["D"], c["ctx"], c["page"]
+    g = torch.Generator().manual_seed(4000)
+    max_pages = ctx // page
+    num_pages = B * max_pages
+    q = torch.randn((B, Hq, D), generator=g).to(torch.bfloat16).to(dev)
+    kc = torch.randn((num_pages, page, Hkv, D), generator=g).to(torch.bfloat16).to(dev)
+    vc = torch.randn((num_pages, page, Hkv, D), generator=g).to(torch.bfloat16).to(dev)
+    table = torch.randperm(num_pages, generator=g).to(torch.int32).reshape(B, max_pages).to(dev)
+    lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+    o, lse = torch.empty_like(q), torch.empty((B, Hq), device=dev, dtype=torch.float32)
+    need = aa.axis_attn_decode_workspace_bytes(B, Hq, Hkv, D, page, max_pages)
+    ws = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
+    st = torch.cuda.current_stream(dev)
+    ev = []
+    for n in range(3 + steps):
+        flush.fill_(n & 0xFF)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(st)
+        aa.attention_decode(q, kc, vc, table, lens, out=o, lse=lse, workspace=ws)
+        e[1].record(st)
+        if n >= 3:
+            ev.append(e)
+    torch.cuda.synchronize()
+    aa.check_status(st)
+    ms = sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev)
+    nbytes = B * ctx * Hkv * D * 2 * 2 + 2 * B * Hq * D * 2
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"config": f"B={B} Hq={Hq} Hkv={Hkv} D={D} context={ctx} page_size={page} (bf16 paged cache, "
+                      f"random page order)", "ms": ms, "steps": steps, "algorithmic_bytes": nbytes,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs}}
+
+
 def summarize(w, total_ms, stage_totals, steps, world, p_meas, det):
     """Per-workload figures: fwd / bwd TFLOP/s and fractions of the peaks."""
     avg = [float(t) / steps for t in stage_totals]
@@ -536,6 +639,15 @@ def main():
         summ["gpu_launches"] = 4 * ko
         del po
         torch.cuda.empty_cache()
+    # ---- the headline workload with RoPE fused, and the decode step
+    rope = None
+    decode = {}
+    if not sharded and not det:
+        rope = time_rope(aa, w, rank_seed(WORKLOAD_SEED[w.name], rank), dev, args.other_steps, flush, p_meas)
+        torch.cuda.empty_cache()
+        for name in DECODE:
+            decode[name] = time_decode(aa, name, dev, args.other_steps, flush, pk["hbm_gbs"])
+            torch.cuda.empty_cache()
     sampler.stop()
 
     cpu = None
@@ -563,7 +675,7 @@ def main():
             "bwd_mode": "deterministic (axis_attn_bwd_det)" if det else "ordinary (axis_attn_bwd stages)",
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": 4 * K, "clocks": clocks,
-            "workloads": others,
+            "workloads": others, "rope": rope, "decode": decode,
         }
         print(json.dumps(line))
     if world > 1:

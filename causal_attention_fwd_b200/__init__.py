@@ -9,8 +9,10 @@ from .binding import (  # noqa: F401
     EXPORTS,
     AxisAttnError,
     attention_backward,
+    attention_backward_rope,
     attention_decode,
     attention_forward,
+    attention_forward_rope,
     axis_attn_bwd,
     axis_attn_bwd_det,
     axis_attn_bwd_det_workspace_bytes,
@@ -18,14 +20,20 @@ from .binding import (  # noqa: F401
     axis_attn_bwd_main,
     axis_attn_bwd_noalloc,
     axis_attn_bwd_prepare,
+    axis_attn_bwd_rope,
+    axis_attn_bwd_rope_workspace_bytes,
     axis_attn_bwd_workspace_bytes,
     axis_attn_decode,
     axis_attn_decode_workspace_bytes,
     axis_attn_fwd,
+    axis_attn_fwd_rope,
     axis_attn_get_status,
     axis_attn_last_status_word,
+    axis_attn_rope,
+    axis_attn_rope_table,
     axis_attn_strerror,
     check_status,
     library_path,
     load,
+    rope_table,
 )

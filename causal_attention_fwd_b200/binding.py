@@ -28,6 +28,11 @@ EXPORTS = (
     "axis_attn_bwd_noalloc",
     "axis_attn_bwd_det_workspace_bytes",
     "axis_attn_bwd_det",
+    "axis_attn_rope_table",
+    "axis_attn_rope",
+    "axis_attn_fwd_rope",
+    "axis_attn_bwd_rope_workspace_bytes",
+    "axis_attn_bwd_rope",
     "axis_attn_decode_workspace_bytes",
     "axis_attn_decode",
     "axis_attn_get_status",
@@ -90,6 +95,16 @@ def load():
             lib.axis_attn_bwd_det_workspace_bytes.restype = sz
             lib.axis_attn_bwd_det.argtypes = [vp] * 9 + [i] * 5 + [f, i, vp, sz, vp]
             lib.axis_attn_bwd_det.restype = i
+            lib.axis_attn_rope_table.argtypes = [vp, i, i, ctypes.c_double, vp]
+            lib.axis_attn_rope_table.restype = i
+            lib.axis_attn_rope.argtypes = [vp] * 3 + [i] * 5 + [vp]
+            lib.axis_attn_rope.restype = i
+            lib.axis_attn_fwd_rope.argtypes = [vp] * 7 + [i] * 5 + [f, i, vp]
+            lib.axis_attn_fwd_rope.restype = i
+            lib.axis_attn_bwd_rope_workspace_bytes.argtypes = [i] * 6
+            lib.axis_attn_bwd_rope_workspace_bytes.restype = sz
+            lib.axis_attn_bwd_rope.argtypes = [vp] * 10 + [i] * 5 + [f, i, i, vp, sz, vp]
+            lib.axis_attn_bwd_rope.restype = i
             lib.axis_attn_decode_workspace_bytes.argtypes = [i] * 6
             lib.axis_attn_decode_workspace_bytes.restype = sz
             lib.axis_attn_decode.argtypes = [vp] * 7 + [i] * 7 + [f, vp, sz, vp]
@@ -151,6 +166,28 @@ def axis_attn_bwd_det(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, 
     the key tiles in a fixed order; see include/axis_attn.h)."""
     return load().axis_attn_bwd_det(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
                                     workspace, workspace_bytes, stream)
+
+
+def axis_attn_rope_table(cs, S, D, base, stream) -> int:
+    return load().axis_attn_rope_table(cs, S, D, base, stream)
+
+
+def axis_attn_rope(x, y, cs, B, S, H, D, inverse, stream) -> int:
+    return load().axis_attn_rope(x, y, cs, B, S, H, D, inverse, stream)
+
+
+def axis_attn_fwd_rope(q, k, v, cs, o, lse, k_rot, B, Hq, Hkv, S, D, scale, causal, stream) -> int:
+    return load().axis_attn_fwd_rope(q, k, v, cs, o, lse, k_rot, B, Hq, Hkv, S, D, scale, causal, stream)
+
+
+def axis_attn_bwd_rope_workspace_bytes(B, Hq, Hkv, S, D, deterministic) -> int:
+    return int(load().axis_attn_bwd_rope_workspace_bytes(B, Hq, Hkv, S, D, deterministic))
+
+
+def axis_attn_bwd_rope(q, k_rot, v, cs, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, deterministic,
+                       workspace, workspace_bytes, stream) -> int:
+    return load().axis_attn_bwd_rope(q, k_rot, v, cs, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
+                                     deterministic, workspace, workspace_bytes, stream)
 
 
 def axis_attn_decode_workspace_bytes(B, Hq, Hkv, D, page_size, max_pages) -> int:
@@ -301,6 +338,75 @@ def attention_backward(q, k, v, o, lse, dout, causal: bool = True, scale: float 
                   workspace.numel() * workspace.element_size(), _stream(stream, dev))
     if rc:
         raise AxisAttnError(rc, name)
+    return dq, dk, dv
+
+
+def rope_table(S: int, D: int, base: float = 10000.0, device=None, stream=None):
+    """The (cos, sin) table [S, D/2, 2] fp64 of the rotary embedding (freqs_cis)."""
+    import torch
+
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    cs = torch.empty((S, D // 2, 2), device=dev, dtype=torch.float64)
+    with torch.cuda.device(dev):
+        rc = axis_attn_rope_table(cs.data_ptr(), S, D, base, _stream(stream, dev))
+    if rc:
+        raise AxisAttnError(rc, "axis_attn_rope_table")
+    return cs
+
+
+def _check_cs(cs, S, D, where):
+    import torch
+
+    _require(isinstance(cs, torch.Tensor) and cs.dim() == 3 and cs.shape[0] >= S and cs.shape[1:] == (D // 2, 2),
+             ERR_SHAPE, where, f"the RoPE table must be [>= {S}, {D // 2}, 2]")
+    _check_tensor(cs[:S], "cs", (S, D // 2, 2), torch.float64, where)
+
+
+def attention_forward_rope(q, k, v, cs, causal: bool = True, scale: float | None = None, stream=None):
+    """Forward with RoPE fused: (o, lse, k_rot) for unrotated bf16 q, k and the
+    table cs of rope_table(); k_rot (the rotated keys) feeds attention_backward_rope."""
+    import torch
+
+    where = "attention_forward_rope"
+    B, Hq, Hkv, S, D = _dims(q, k, v, where)
+    _check_cs(cs, S, D, where)
+    dev = _check_device({"q": q, "k": k, "v": v, "cs": cs}, where)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    with torch.cuda.device(dev):
+        o = torch.empty_like(q)
+        l = torch.empty((B, Hq, S), device=dev, dtype=torch.float32)
+        k_rot = torch.empty_like(k)
+        rc = axis_attn_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), cs.data_ptr(), o.data_ptr(), l.data_ptr(),
+                                k_rot.data_ptr(), B, Hq, Hkv, S, D, scale, int(causal), _stream(stream, dev))
+    if rc:
+        raise AxisAttnError(rc, "axis_attn_fwd_rope")
+    return o, l, k_rot
+
+
+def attention_backward_rope(q, k_rot, v, cs, o, lse, dout, causal: bool = True, scale: float | None = None,
+                            deterministic: bool = False, stream=None):
+    """Gradients (dq, dk, dv) with respect to the unrotated q, k of
+    attention_forward_rope (k_rot is its third output)."""
+    import torch
+
+    where = "attention_backward_rope"
+    B, Hq, Hkv, S, D = _dims(q, k_rot, v, where)
+    _check_cs(cs, S, D, where)
+    _check_tensor(o, "o", (B, S, Hq, D), torch.bfloat16, where)
+    _check_tensor(dout, "dout", (B, S, Hq, D), torch.bfloat16, where)
+    _check_tensor(lse, "lse", (B, Hq, S), torch.float32, where)
+    dev = _check_device({"q": q, "k_rot": k_rot, "v": v, "cs": cs, "o": o, "lse": lse, "dout": dout}, where)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    need = axis_attn_bwd_rope_workspace_bytes(B, Hq, Hkv, S, D, int(deterministic))
+    with torch.cuda.device(dev):
+        ws = torch.empty(need, device=dev, dtype=torch.uint8)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k_rot), torch.empty_like(v)
+        rc = axis_attn_bwd_rope(q.data_ptr(), k_rot.data_ptr(), v.data_ptr(), cs.data_ptr(), o.data_ptr(),
+                                dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                B, Hq, Hkv, S, D, scale, int(causal), int(deterministic), ws.data_ptr(), need,
+                                _stream(stream, dev))
+    if rc:
+        raise AxisAttnError(rc, "axis_attn_bwd_rope")
     return dq, dk, dv
 
 

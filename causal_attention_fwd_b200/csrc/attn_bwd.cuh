@@ -30,9 +30,22 @@
 // lane = feature), so every MMA has M = 128.
 #pragma once
 
+#include "attn_rope.cuh"
 #include "sm100_ptx.cuh"
 
 namespace axis_attn {
+
+// Compute warps (P^T, dS^T): 8 (two per SM sub-partition, each thread a key
+// row and half the query columns, in 32-column chunks) or 16 (four per
+// sub-partition, a quarter of the columns, in 16-column chunks; more warps to
+// hide the TMEM, MUFU and barrier latencies of each step).
+#ifndef AXIS_ATTN_BWD_CW
+#define AXIS_ATTN_BWD_CW 8
+#endif
+// Unroll factor of the per-step loop over a compute thread's TMEM chunks.
+#ifndef AXIS_ATTN_BWD_CC_UNROLL
+#define AXIS_ATTN_BWD_CC_UNROLL 4
+#endif
 
 struct BwdArgs {
   __nv_bfloat16* dk;
@@ -43,6 +56,7 @@ struct BwdArgs {
   int B, Hq, Hkv, S, S_pad;
   float scale, scale_log2;
   int no_dq;           // 1: dK, dV only (deterministic mode: attn_bwd_dq_kernel computes dQ)
+  const double2* rope_cs;  // RoPE: (cos, sin) table [S][HD/2], fp64; dK leaves through the transposed rotation
 };
 
 template <int HD>
@@ -56,8 +70,9 @@ struct BwdCfg {
   static constexpr uint32_t QTILE = NSLAB * QSLAB;
   static constexpr uint32_t PS_BYTES = (BM / 64) * 128 * 128;  // dS^T: 128 keys x BM bf16
   static constexpr int ST = 3;                     // Q / dO / LSE / Dr ring depth
-  static constexpr int HALF = BM / 2;              // query columns per compute warpgroup
-  static constexpr int NCH = HALF / 32;            // 32-column chunks per compute thread
+  static constexpr int COLS = BM / (AXIS_ATTN_BWD_CW / 4);  // query columns per compute thread
+  static constexpr int SUBW = AXIS_ATTN_BWD_CW == 16 ? 16 : 32;  // columns per TMEM load
+  static constexpr int NSUB = COLS / SUBW;                       // loads per step
   // dQ tile staged for the TMA reduce-add: fp32, four 128B-swizzled boxes of
   // 32 columns x 64 rows (D = 64: rows = queries, columns = features; D = 128:
   // the tile is 64 queries x 128 features, one box per 32 features)
@@ -88,18 +103,20 @@ struct BwdCfg {
 #define AXIS_ATTN_BWD_POLY_MASK 0x0000
 #endif
 
-// Warps 0-7: P^T / dS^T (thread = key row, half the query columns each);
-// warp 8 loads; warp 9 issues the score MMAs and owns TMEM; warp 10 issues
-// the TMA reduce-adds of the dQ tiles into the fp32 accumulator; warp 11
-// issues the gradient MMAs; warps 12-15 copy each dQ tile from TMEM into the
-// swizzled staging tile (one TMEM lane quarter each), off the compute warps'
-// critical path.  512 threads: up to 128 registers each.
-constexpr int BWD_THREADS = 512;
-constexpr int BWD_WARP_LOAD = 8;
-constexpr int BWD_WARP_MMA = 9;
-constexpr int BWD_WARP_RED = 10;
-constexpr int BWD_WARP_GRAD = 11;
-constexpr int BWD_WARP_DQ0 = 12;
+// Warps 0 .. CW-1: P^T / dS^T (thread = key row); CW loads; CW+1 issues the
+// score MMAs and owns TMEM; CW+2 issues the TMA reduce-adds of the dQ tiles
+// into the fp32 accumulator; CW+3 issues the gradient MMAs; CW+4 .. CW+7 copy
+// each dQ tile from TMEM into the swizzled staging tile (one TMEM lane quarter
+// each), off the compute warps' critical path.
+constexpr int BWD_CW = AXIS_ATTN_BWD_CW;
+constexpr int BWD_CC_UNROLL = AXIS_ATTN_BWD_CC_UNROLL;
+static_assert(BWD_CW == 8 || BWD_CW == 16, "8 or 16 compute warps");
+constexpr int BWD_THREADS = (BWD_CW + 8) * 32;
+constexpr int BWD_WARP_LOAD = BWD_CW;
+constexpr int BWD_WARP_MMA = BWD_CW + 1;
+constexpr int BWD_WARP_RED = BWD_CW + 2;
+constexpr int BWD_WARP_GRAD = BWD_CW + 3;
+constexpr int BWD_WARP_DQ0 = BWD_CW + 4;
 
 enum BwdSite { B_KV = 21, B_QEMPTY, B_QFULL, B_SPFREE, B_PDSFULL, B_DQFREE, B_SPFULL, B_DQFULL, B_FIN, B_PDSFREE,
                B_STGFULL, B_STGFREE };
@@ -146,7 +163,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
   using C = BwdCfg<HD>;
-  constexpr int BM = C::BM, ST = C::ST, HALF = C::HALF, NCH = C::NCH;
+  constexpr int BM = C::BM, ST = C::ST, COLS = C::COLS, SUBW = C::SUBW, NSUB = C::NSUB;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -196,8 +213,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mbar_init(bar_qempty(s), 2);  // one commit from each MMA issuer
     }
     mbar_init(bar_spfull, 1);
-    mbar_init(bar_spfree, 8);
-    mbar_init(bar_pdsfull, 8);
+    mbar_init(bar_spfree, BWD_CW);
+    mbar_init(bar_pdsfull, BWD_CW);
     mbar_init(bar_ptfree, 1);
     mbar_init(bar_dqfull, 1);
     mbar_init(bar_dqfree, 4);
@@ -376,25 +393,27 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const float sc = a.scale;
       for (int t = 0; t < n_it; ++t) {
         if (!wait_warp(bar_dqfull, t & 1, abort, B_DQFULL)) break;
-        tc_fence_after();
-        uint32_t v[2][32];
-        tmem_ld32(tmem + lane_off + C::T_DQ, v[0]);
-        tmem_ld32(tmem + lane_off + C::T_DQ + 32, v[1]);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_dqfree);
         if (t > 0 && !wait_warp(bar_stgfree, (t - 1) & 1, abort, B_STGFREE)) break;
+        tc_fence_after();
+        // one 32-column half at a time (32 registers); TMEM is released after the second load
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + C::T_DQ + 32 * ch, v);
+          tmem_wait_ld();
+          if (ch == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_dqfree);
+          }
           if (C::QLANE) {
             // lane = query row kr, columns = features [32 ch, 32 ch + 32): one 128-byte box row
             const uint32_t row = sSTG + ((kr >> 6) * 2 + ch) * C::DQ_BOX + (kr & 63) * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
               asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(row + ((c ^ (kr & 7)) << 4)),
-                           "f"(__uint_as_float(v[ch][4 * c]) * sc), "f"(__uint_as_float(v[ch][4 * c + 1]) * sc),
-                           "f"(__uint_as_float(v[ch][4 * c + 2]) * sc), "f"(__uint_as_float(v[ch][4 * c + 3]) * sc)
+                           "f"(__uint_as_float(v[4 * c]) * sc), "f"(__uint_as_float(v[4 * c + 1]) * sc),
+                           "f"(__uint_as_float(v[4 * c + 2]) * sc), "f"(__uint_as_float(v[4 * c + 3]) * sc)
                            : "memory");
           } else {
             // lane = feature kr (box kr / 32, column kr % 32), columns = query rows 32 ch + e
@@ -403,7 +422,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             for (int e = 0; e < 32; ++e) {
               const int q = 32 * ch + e;
               asm volatile("st.shared.f32 [%0], %1;" ::"r"(boxb + q * 128 + (((lane >> 2) ^ (q & 7)) << 4)),
-                           "f"(__uint_as_float(v[ch][e]) * sc)
+                           "f"(__uint_as_float(v[e]) * sc)
                            : "memory");
             }
           }
@@ -413,13 +432,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         if (lane == 0) mbar_arrive(bar_stgfull);
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < BWD_CW) {
     // ===================================================== P^T, dS^T (thread = key row)
-    const int wq = warp & 3, ch = warp >> 2;
+    const int wq = warp & 3, ch = warp >> 2;  // lane quarter, column group
     const int kr = wq * 32 + lane;
     const int key = 128 * j + kr;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const int c0 = ch * HALF;
+    const int c0 = ch * COLS;
     const uint64_t cc2 = f2_pack(a.scale_log2, a.scale_log2);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
@@ -435,23 +454,28 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const bool need_mask = (CAUSAL && q0 < 128 * j + 127) || (128 * j + 128 > a.S);
       const float* lse_t = lse_s + s * BM + c0;
       const float* dr_t = dr_s + s * BM + c0;
-#pragma unroll
-      for (int cc = 0; cc < NCH; ++cc) {
-        uint32_t sv[32], dpv[32];
-        tmem_ld32(tmem + lane_off + C::T_S + c0 + 32 * cc, sv);
-        tmem_ld32(tmem + lane_off + C::T_DP + c0 + 32 * cc, dpv);
+#pragma unroll BWD_CC_UNROLL
+      for (int cc = 0; cc < NSUB; ++cc) {
+        uint32_t sv[SUBW], dpv[SUBW];
+        if constexpr (SUBW == 32) {
+          tmem_ld32(tmem + lane_off + C::T_S + c0 + SUBW * cc, sv);
+          tmem_ld32(tmem + lane_off + C::T_DP + c0 + SUBW * cc, dpv);
+        } else {
+          tmem_ld16(tmem + lane_off + C::T_S + c0 + SUBW * cc, sv);
+          tmem_ld16(tmem + lane_off + C::T_DP + c0 + SUBW * cc, dpv);
+        }
         tmem_wait_ld();
-        if (cc == NCH - 1) {
+        if (cc == NSUB - 1) {
           // all of this thread's S^T, dP^T are in registers: TMEM may take the next step's
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar_spfree);
         }
-        uint32_t pk[16], dk[16];
+        uint32_t pk[SUBW / 2], dk[SUBW / 2];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse_t + 32 * cc + e);
-          const float4 d4 = *reinterpret_cast<const float4*>(dr_t + 32 * cc + e);
+        for (int e = 0; e < SUBW; e += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_t + SUBW * cc + e);
+          const float4 d4 = *reinterpret_cast<const float4*>(dr_t + SUBW * cc + e);
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int ee = e + 2 * h2;
@@ -468,7 +492,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
               p1 = ex2_approx(x1);
             }
             if (need_mask) {
-              const int q = q0 + c0 + 32 * cc + ee;
+              const int q = q0 + c0 + SUBW * cc + ee;
               if ((CAUSAL && key > q) || key >= a.S) p0 = 0.f;
               if ((CAUSAL && key > q + 1) || key >= a.S) p1 = 0.f;
             }
@@ -484,14 +508,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           ok = false;
           break;
         }
-        tmem_st16(tmem + lane_off + C::T_P + (c0 >> 1) + 16 * cc, pk);
+        if constexpr (SUBW == 32)
+          tmem_st16(tmem + lane_off + C::T_P + (c0 >> 1) + (SUBW / 2) * cc, pk);
+        else
+          tmem_st8(tmem + lane_off + C::T_P + (c0 >> 1) + (SUBW / 2) * cc, pk);
         // ... and the previous step's dK, dQ with dS^T
         if (cc == 0 && it > 0 && !wait_warp(bar_dstfree, (it - 1) & 1, abort, B_PDSFREE)) {
           ok = false;
           break;
         }
-        store_row16(sDST, kr, c0 + 32 * cc, &dk[0]);
-        store_row16(sDST, kr, c0 + 32 * cc + 16, &dk[8]);
+#pragma unroll
+        for (int x = 0; x < SUBW / 16; ++x) store_row16(sDST, kr, c0 + SUBW * cc + 16 * x, &dk[8 * x]);
       }
       if (!ok) break;
       tmem_wait_st();
@@ -500,21 +527,36 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       __syncwarp();
       if (lane == 0 && !(AXIS_ATTN_TEST_DROP_ARRIVE == 2 && it == 0)) mbar_arrive(bar_pdsfull);
     }
-    // epilogue: warps 0-3 write dV, warps 4-7 write dK (x scale)
+    // epilogue: the first half of the column groups writes dV, the second dK
+    // (x scale); with 16 warps each group takes half of the features
+    constexpr int NG = BWD_CW / 4, GPT = NG / 2;  // column groups, groups per tensor
     if (ok && wait_warp(bar_fin, 0, abort, B_FIN)) {
       tc_fence_after();
-      const uint32_t tcol = ch == 0 ? C::T_DV : C::T_DK;
-      const float mul = ch == 0 ? 1.f : a.scale;
-      __nv_bfloat16* dst_row = (ch == 0 ? a.dv : a.dk) + (((size_t)b * a.S + key) * a.Hkv + kvh) * HD;
+      const bool is_dv = ch < GPT;
+      const int f0 = (ch % GPT) * (HD / GPT);  // first feature of this group
+      const uint32_t tcol = (is_dv ? C::T_DV : C::T_DK) + f0;
+      const float mul = is_dv ? 1.f : a.scale;
+      __nv_bfloat16* dst_row = (is_dv ? a.dv : a.dk) + (((size_t)b * a.S + key) * a.Hkv + kvh) * HD + f0;
 #pragma unroll 1
-      for (int cc = 0; cc < HD / 32; ++cc) {
+      for (int cc = 0; cc < HD / GPT / 32; ++cc) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + tcol + cc * 32, v);
         tmem_wait_ld();
         uint32_t pk2[16];
+        if (a.rope_cs != nullptr && !is_dv && key < a.S) {
+          // dK = R(key)^T dK': pairs of features f0 + 32 cc + 2 i
+          const double2* t = a.rope_cs + (size_t)key * (HD / 2) + (f0 + 32 * cc) / 2;
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk2[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+          for (int i = 0; i < 16; ++i) {
+            float g0 = __uint_as_float(v[2 * i]) * mul, g1 = __uint_as_float(v[2 * i + 1]) * mul;
+            rope_back(g0, g1, t[i]);
+            pk2[i] = pack_bf16x2(g0, g1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk2[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+        }
         if (key < a.S) {
           uint4* dst = reinterpret_cast<uint4*>(dst_row + cc * 32);
 #pragma unroll
@@ -590,11 +632,13 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
   for (size_t k = gtid; k < dq_vec4; k += nthreads) dqacc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dq[b,i,h,:] = bf16(dqacc[b,h,i,:]); 8 features per thread.
+// dq[b,i,h,:] = bf16(dqacc[b,h,i,:]); 8 features per thread.  With a RoPE
+// table the row leaves through the transposed rotation of position i.
 template <int HD>
 __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* __restrict__ dqacc,
                                                                   __nv_bfloat16* __restrict__ dq, int Hq,
-                                                                  int S, size_t n8) {
+                                                                  int S, size_t n8,
+                                                                  const double2* __restrict__ rope_cs) {
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < n8; k += stride) {
     const int c8 = (int)(k % (HD / 8));
@@ -604,7 +648,14 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
     const int i = (int)(bi % S);
     const size_t b = bi / S;
     const float4* src = reinterpret_cast<const float4*>(dqacc + (((b * Hq + h) * S + i) * HD) + 8 * c8);
-    const float4 x = src[0], y = src[1];
+    float4 x = src[0], y = src[1];
+    if (rope_cs != nullptr) {  // pairs 4 c8 .. 4 c8 + 3 at position i, transposed rotation
+      const double2* t = rope_cs + (size_t)i * (HD / 2) + 4 * c8;
+      rope_back(x.x, x.y, t[0]);
+      rope_back(x.z, x.w, t[1]);
+      rope_back(y.x, y.y, t[2]);
+      rope_back(y.z, y.w, t[3]);
+    }
     uint4 out;
     out.x = pack_bf16x2(x.x, x.y);
     out.y = pack_bf16x2(x.z, x.w);

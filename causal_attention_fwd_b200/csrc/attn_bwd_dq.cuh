@@ -19,6 +19,7 @@
 // dP [128,256), dQ [256, 256 + HD).
 #pragma once
 
+#include "attn_rope.cuh"
 #include "sm100_ptx.cuh"
 
 namespace axis_attn {
@@ -29,6 +30,7 @@ struct DqArgs {
   const float* ndr;    // [B*Hq][S_pad]  -rowsum(dO * O); 0 on padding rows
   int B, Hq, Hkv, S, S_pad;
   float scale, scale_log2;
+  const double2* rope_cs;  // RoPE: (cos, sin) table [S][HD/2], fp64; dQ leaves through the transposed rotation
 };
 
 template <int HD>
@@ -275,6 +277,17 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         for (int i = 0; i < 16; ++i) v[i] = v16[i];
       }
       tmem_wait_ld();
+      if (row_g < a.S && a.rope_cs != nullptr) {
+        // dQ = R(row)^T dQ': pairs of features NC qc + 2 i
+        const double2* t = a.rope_cs + (size_t)row_g * (HD / 2) + NC * qc / 2;
+#pragma unroll
+        for (int i = 0; i < NC / 2; ++i) {
+          float g0 = __uint_as_float(v[2 * i]), g1 = __uint_as_float(v[2 * i + 1]);
+          rope_back(g0, g1, t[i]);
+          v[2 * i] = __float_as_uint(g0);
+          v[2 * i + 1] = __float_as_uint(g1);
+        }
+      }
       if (row_g < a.S) {
         uint4* dst = reinterpret_cast<uint4*>(a.dq + (((size_t)b * a.S + row_g) * a.Hq + h) * HD + NC * qc);
 #pragma unroll

@@ -40,6 +40,7 @@
 // take turns) P0 [128,192) P1 [192,256) O0 [256,384) O1 [384,512).
 #pragma once
 
+#include "attn_rope.cuh"
 #include "sm100_ptx.cuh"
 
 namespace axis_attn {
@@ -51,6 +52,7 @@ struct FwdArgs {
   float scale_log2;  // scale * log2(e)
   int n_qblocks;     // ceil(S / 256)
   int n_items;       // n_qblocks * B * Hq
+  const double2* rope_cs;  // RoPE kernel only: (cos, sin) table [S][HD/2], fp64
 };
 
 // The it-th item of this CTA: snake order over the grid (even passes left to
@@ -102,7 +104,7 @@ struct FwdCfg {
   static constexpr bool SHARED_S = HD == 128;
   static constexpr uint32_t T_P = SHARED_S ? 128 : 384, T_O = 256;
   static __host__ __device__ constexpr uint32_t t_s(int t) { return SHARED_S ? 0u : 128u * t; }
-  static constexpr int NBAR = 23 + 2 * KST + 2 * VST;
+  static constexpr int NBAR = 24 + 2 * KST + 2 * VST;
   static constexpr uint32_t XCH_OFF = (2 + KST + VST) * TILE;  // row-max / row-sum exchange
   static constexpr uint32_t XCH_BYTES = 2 * 2 * 2 * 128 * 4;   // [parity][tile][half][row] fp32
   static constexpr uint32_t BAR_OFF = XCH_OFF + XCH_BYTES;
@@ -205,6 +207,10 @@ __device__ __forceinline__ void xpose_chunks(uint32_t (&c)[4 * N], int lane) {
 // owner), 18 TMA producer of V, 19 P V issuer.  Five warps per SM
 // sub-partition leave 96 registers a thread: half a row of scores (64) plus
 // its packed probabilities.
+// With RoPE fused (ROPE = true) the whole V-producer warp also rotates each
+// item's Q tiles in shared memory after they land and before the S issuer
+// reads them (a 21st warp would put six warps on one SM sub-partition and
+// cut every thread to 80 registers).
 constexpr int FWD_THREADS = 640;
 constexpr int FWD_SOFTMAX_WARPS = 16;
 constexpr int FWD_WARP_LOAD = 16;
@@ -212,7 +218,7 @@ constexpr int FWD_WARP_MMA = 17;
 constexpr int FWD_WARP_LOADV = 18;
 constexpr int FWD_WARP_PV = 19;
 
-template <int HD, bool CAUSAL>
+template <int HD, bool CAUSAL, bool ROPE>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
@@ -245,6 +251,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   auto bar_xch = [&](int t, int wq) { return bars + 8u * (B2 + 11 + 4 * t + wq); };
   // O_t has been read out by the epilogue: the next item may overwrite it
   auto bar_ofree = [&](int t) { return bars + 8u * (B2 + 19 + t); };
+  // RoPE kernel: the Q copies land here; the rope warp then completes bar_q
+  const uint32_t bar_qraw = bars + 8u * (B2 + 21);
   float* xch = reinterpret_cast<float*>(gbase + C::XCH_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::BAR_OFF + 8 * C::NBAR);
   volatile WaitCtl* abort = reinterpret_cast<volatile WaitCtl*>(gbase + C::BAR_OFF + 8 * C::NBAR + 4);
@@ -273,6 +281,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       for (int wq = 0; wq < 4; ++wq) mbar_init(bar_xch(t, wq), 2);
     }
     mbar_init(bar_fin, 2);  // one commit from each MMA issuer
+    mbar_init(bar_qraw, 1);
     wait_ctl_init(abort);
     fence_barrier_init();
   }
@@ -285,7 +294,46 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == FWD_WARP_LOAD || warp == FWD_WARP_LOADV) {
+  if (ROPE && warp == FWD_WARP_LOADV) {
+    // ===================================================== V producer + RoPE of Q
+    // Per item, the whole warp waits for the Q copies, rotates every Q row by
+    // its sequence position in shared memory, makes the generic-proxy writes
+    // visible to the tensor cores and releases Q to the S issuer (bar_q);
+    // then lane 0 streams the item's V tiles as the plain V producer does.
+    if (lane == 0) tma_prefetch_desc(&tm_v);
+    int g = 0;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      const int w = fwd_item(it);
+      if (w >= a.n_items) break;
+      const FwdItem I = fwd_decode(a, w, CAUSAL);
+      if (!(ok = wait_warp<true>(bar_qraw, it & 1, abort, F_Q))) break;
+      rope_tile_smem<HD>(sQ, SLAB, 128, 256 * I.m, a.S, a.rope_cs, lane);
+      if (I.has1) rope_tile_smem<HD>(sQ + TILE, SLAB, 128, 256 * I.m + 128, a.S, a.rope_cs, lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar_q);
+        for (int j = 0; j < I.nmax; ++j, ++g) {
+          const int s = g % VST;
+          if (g >= VST && !mbar_wait_bounded<true>(bar_vempty(s), ((g / VST) & 1) ^ 1, abort, F_EMPTY)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_vfull(s), TILE);
+          for (int sl = 0; sl < C::NSLAB; ++sl)
+            tma_load_4d(sV + s * TILE + sl * SLAB, &tm_v, bar_vfull(s), 64 * sl, I.kvh, 128 * j, I.b);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    // Drain (lane 0): every V copy started has landed before the CTA exits.
+    if (lane == 0) {
+      volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
+      for (int x = g - VST > 0 ? g - VST : 0; x < g; ++x)
+        mbar_wait_bounded<true>(bar_vfull(x % VST), (x / VST) & 1, &never, F_VFULL);
+    }
+  } else if (warp == FWD_WARP_LOAD || warp == FWD_WARP_LOADV) {
     // ===================================================== TMA producers
     // warp 16: per item Q (once the previous item's S products are done with
     // it), then the K ring (with an L2 prefetch of K and V PF tiles ahead);
@@ -308,12 +356,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         const FwdItem I = fwd_decode(a, w, CAUSAL);
         if (is_k) {
           if (it > 0 && !mbar_wait_bounded<true>(bar_qempty, (it - 1) & 1, abort, F_QEMPTY)) break;
-          mbar_arrive_expect_tx(bar_q, (I.has1 ? 2u : 1u) * TILE);
+          const uint32_t bq = ROPE ? bar_qraw : bar_q;
+          mbar_arrive_expect_tx(bq, (I.has1 ? 2u : 1u) * TILE);
           for (int sl = 0; sl < C::NSLAB; ++sl)
-            tma_load_4d(sQ + sl * SLAB, &tm_q, bar_q, 64 * sl, I.h, 256 * I.m, I.b);
+            tma_load_4d(sQ + sl * SLAB, &tm_q, bq, 64 * sl, I.h, 256 * I.m, I.b);
           if (I.has1)
             for (int sl = 0; sl < C::NSLAB; ++sl)
-              tma_load_4d(sQ + TILE + sl * SLAB, &tm_q, bar_q, 64 * sl, I.h, 256 * I.m + 128, I.b);
+              tma_load_4d(sQ + TILE + sl * SLAB, &tm_q, bq, 64 * sl, I.h, 256 * I.m + 128, I.b);
           ++nq;
           constexpr int PF = 4;
           auto prefetch = [&](int j) {
@@ -351,7 +400,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       // (each stage's most recent phase; nothing newer can have started).
       volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
       const int NS = is_k ? KST : VST;
-      if (is_k && nq > 0) mbar_wait_bounded<true>(bar_q, (nq - 1) & 1, &never, F_Q);
+      if (is_k && nq > 0) mbar_wait_bounded<true>(ROPE ? bar_qraw : bar_q, (nq - 1) & 1, &never, F_Q);
       for (int x = g - NS > 0 ? g - NS : 0; x < g; ++x)
         mbar_wait_bounded<true>(is_k ? bar_kfull(x % KST) : bar_vfull(x % VST), (x / NS) & 1, &never,
                           is_k ? F_KFULL : F_VFULL);

@@ -13,6 +13,7 @@
 #include "attn_bwd_dq.cuh"
 #include "attn_decode.cuh"
 #include "attn_fwd.cuh"
+#include "attn_rope.cuh"
 
 namespace axis_attn {
 namespace {
@@ -93,20 +94,22 @@ bool make_dq_map(CUtensorMap* map, const float* ptr, int BH, int S, int D) {
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct WsLayout {
-  size_t lse2, dr, dqacc, total;
+  size_t lse2, dr, dqacc, qrot, total;
   int S_pad;
 };
 
 // det: no dQ accumulator (the deterministic dQ pass keeps dQ in TMEM), so the
-// workspace is the two row sections only.
-WsLayout ws_layout(int B, int Hq, int S, int D, bool det = false) {
+// workspace is the two row sections only.  rope: plus the rotated Q (bf16
+// [B, S, Hq, D]) that the backward's kernels read in place of Q.
+WsLayout ws_layout(int B, int Hq, int S, int D, bool det = false, bool rope = false) {
   WsLayout w;
   w.S_pad = (S + 127) / 128 * 128;
   const size_t rows = (size_t)B * Hq * w.S_pad;
   w.lse2 = 0;
   w.dr = round256(rows * 4);
   w.dqacc = w.dr + round256(rows * 4);
-  w.total = w.dqacc + (det ? 0 : round256((size_t)B * Hq * S * D * 4));
+  w.qrot = w.dqacc + (det ? 0 : round256((size_t)B * Hq * S * D * 4));
+  w.total = w.qrot + (rope ? round256((size_t)B * S * Hq * D * 2) : 0);
   return w;
 }
 
@@ -134,15 +137,61 @@ int set_smem(K kernel, uint32_t bytes, int dev, bool (&done)[64]) {
   return AXIS_ATTN_OK;
 }
 
-template <int HD, bool CAUSAL>
+template <int HD, bool CAUSAL, bool ROPE>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
                cudaStream_t st, int dev) {
-  auto kern = attn_fwd_kernel<HD, CAUSAL>;
+  auto kern = attn_fwd_kernel<HD, CAUSAL, ROPE>;
   static bool done[64];
   if (int rc = set_smem(kern, FwdCfg<HD>::SMEM, dev, done)) return rc;
   // persistent: one CTA per SM (the kernel walks its share of the items)
   const unsigned grid = (unsigned)(a.n_items < sm_count(dev) ? a.n_items : sm_count(dev));
   kern<<<grid, FWD_THREADS, FwdCfg<HD>::SMEM, st>>>(mq, mk, mv, a);
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+// The forward kernel over (q, k, v); with a table, Q tiles are rotated in
+// shared memory (k must then hold the rotated keys already).
+int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int S, int D,
+            float scale, int causal, const double* rope_cs, cudaStream_t st, int dev) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, B, S, Hq, D, 128) || !make_map(&mk, k, B, S, Hkv, D, 128) ||
+      !make_map(&mv, v, B, S, Hkv, D, 128))
+    return AXIS_ATTN_ERR_CUDA;
+  FwdArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.S = S;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  a.n_qblocks = (S + 255) / 256;
+  a.n_items = a.n_qblocks * B * Hq;
+  a.rope_cs = reinterpret_cast<const double2*>(rope_cs);
+  if (rope_cs) {
+    if (D == 64)
+      return causal ? launch_fwd<64, true, true>(mq, mk, mv, a, st, dev)
+                    : launch_fwd<64, false, true>(mq, mk, mv, a, st, dev);
+    return causal ? launch_fwd<128, true, true>(mq, mk, mv, a, st, dev)
+                  : launch_fwd<128, false, true>(mq, mk, mv, a, st, dev);
+  }
+  if (D == 64)
+    return causal ? launch_fwd<64, true, false>(mq, mk, mv, a, st, dev)
+                  : launch_fwd<64, false, false>(mq, mk, mv, a, st, dev);
+  return causal ? launch_fwd<128, true, false>(mq, mk, mv, a, st, dev)
+                : launch_fwd<128, false, false>(mq, mk, mv, a, st, dev);
+}
+
+// y = R x (inverse: R^T x) for x, y [B, S, H, D] bf16 with the table cs [S][D/2].
+int run_rope(const void* x, void* y, const double* cs, int B, int S, int H, int D, int inverse, cudaStream_t st) {
+  const long long n16 = (long long)B * S * H * D / 8;
+  const unsigned grid = (unsigned)((n16 + 255) / 256 < 148 * 16 ? (n16 + 255) / 256 : 148 * 16);
+  const auto* t = reinterpret_cast<const double2*>(cs);
+  if (inverse)
+    rope_apply_back_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y), t, n16, S,
+                                                 H, D);
+  else
+    rope_apply_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y), t, n16, S, H, D);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
@@ -181,24 +230,8 @@ extern "C" int axis_attn_fwd(const void* q, const void* k, const void* v, void* 
   if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, B, S, Hq, D, 128) || !make_map(&mk, k, B, S, Hkv, D, 128) ||
-      !make_map(&mv, v, B, S, Hkv, D, 128))
-    return AXIS_ATTN_ERR_CUDA;
-  FwdArgs a;
-  a.o = static_cast<__nv_bfloat16*>(o);
-  a.lse = lse;
-  a.B = B;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.S = S;
-  a.scale_log2 = (float)((double)scale * 1.4426950408889634);
-  a.n_qblocks = (S + 255) / 256;
-  a.n_items = a.n_qblocks * B * Hq;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 64)
-    return causal ? launch_fwd<64, true>(mq, mk, mv, a, st, dev) : launch_fwd<64, false>(mq, mk, mv, a, st, dev);
-  return causal ? launch_fwd<128, true>(mq, mk, mv, a, st, dev) : launch_fwd<128, false>(mq, mk, mv, a, st, dev);
+  return run_fwd(q, k, v, o, lse, B, Hq, Hkv, S, D, scale, causal, nullptr, static_cast<cudaStream_t>(stream),
+                 dev);
 }
 
 extern "C" size_t axis_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
@@ -251,7 +284,7 @@ int run_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, 
 // Stage 2: the main kernel; det: dK, dV only (no dQ accumulator).
 int run_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int Hq,
              int Hkv, int S, int D, float scale, int causal, const WsLayout& w, const WsPtrs& p, bool det,
-             cudaStream_t st, int dev) {
+             cudaStream_t st, int dev, const double* rope_cs = nullptr) {
   const int BM = D == 64 ? BwdCfg<64>::BM : BwdCfg<128>::BM;
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, q, B, S, Hq, D, BM) || !make_map(&mdo, dO, B, S, Hq, D, BM) ||
@@ -273,6 +306,7 @@ int run_main(const void* q, const void* k, const void* v, const void* dO, void* 
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
   a.no_dq = det ? 1 : 0;
+  a.rope_cs = reinterpret_cast<const double2*>(rope_cs);
   if (D == 64)
     return causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, mdq, a, st, dev)
                   : launch_bwd_main<64, false>(mq, mk, mv, mdo, mdq, a, st, dev);
@@ -281,14 +315,16 @@ int run_main(const void* q, const void* k, const void* v, const void* dO, void* 
 }
 
 // Stage 3: dQ to bf16 [B,S,Hq,D].
-int run_finalize(void* dq, int B, int Hq, int S, int D, const WsPtrs& p, cudaStream_t st) {
+int run_finalize(void* dq, int B, int Hq, int S, int D, const WsPtrs& p, cudaStream_t st,
+                 const double* rope_cs = nullptr) {
   const size_t n8 = (size_t)B * S * Hq * D / 8;
   const unsigned grid = (unsigned)((n8 + 255) / 256 < 4096 ? (n8 + 255) / 256 : 4096);
   auto* out = static_cast<__nv_bfloat16*>(dq);
+  const double2* cs = reinterpret_cast<const double2*>(rope_cs);
   if (D == 64) {
-    attn_bwd_dq_convert_kernel<64><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, n8);
+    attn_bwd_dq_convert_kernel<64><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, n8, cs);
   } else {
-    attn_bwd_dq_convert_kernel<128><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, n8);
+    attn_bwd_dq_convert_kernel<128><<<grid, 256, 0, st>>>(p.dqacc, out, Hq, S, n8, cs);
   }
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
@@ -339,7 +375,7 @@ namespace {
 // Deterministic mode, stage 3: dQ recomputed per 128-row query tile.
 int run_dq_pass(const void* q, const void* k, const void* v, const void* dO, void* dq, int B, int Hq, int Hkv,
                 int S, int D, float scale, int causal, const WsLayout& w, const WsPtrs& p, cudaStream_t st,
-                int dev) {
+                int dev, const double* rope_cs = nullptr) {
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, q, B, S, Hq, D, 128) || !make_map(&mdo, dO, B, S, Hq, D, 128) ||
       !make_map(&mk, k, B, S, Hkv, D, 128) || !make_map(&mv, v, B, S, Hkv, D, 128))
@@ -355,6 +391,7 @@ int run_dq_pass(const void* q, const void* k, const void* v, const void* dO, voi
   a.S_pad = w.S_pad;
   a.scale = scale;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  a.rope_cs = reinterpret_cast<const double2*>(rope_cs);
   if (D == 64)
     return causal ? launch_bwd_dq<64, true>(mq, mk, mv, mdo, a, st, dev)
                   : launch_bwd_dq<64, false>(mq, mk, mv, mdo, a, st, dev);
@@ -362,25 +399,34 @@ int run_dq_pass(const void* q, const void* k, const void* v, const void* dO, voi
                 : launch_bwd_dq<128, false>(mq, mk, mv, mdo, a, st, dev);
 }
 
+// The backward; with a RoPE table, k holds the rotated keys, q is rotated into
+// the workspace first, and dQ, dK leave through the transposed rotation.
 int run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
             void* dk, void* dv, int B, int Hq, int Hkv, int S, int D, float scale, int causal, void* workspace,
-            size_t workspace_bytes, void* stream, bool det) {
+            size_t workspace_bytes, void* stream, bool det, const double* rope_cs = nullptr) {
   // Validate everything first so that no stage runs when a later one would fail.
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return AXIS_ATTN_ERR_NULL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(lse) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (rope_cs && !aligned16(rope_cs)))
     return AXIS_ATTN_ERR_ALIGN;
   if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
-  const WsLayout w = ws_layout(B, Hq, S, D, det);
+  const WsLayout w = ws_layout(B, Hq, S, D, det, rope_cs != nullptr);
   if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
   const WsPtrs p = ws_ptrs(workspace, w);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const void* qk = q;  // the queries the kernels read
+  if (rope_cs) {
+    void* qrot = static_cast<char*>(workspace) + w.qrot;
+    if (int rc = run_rope(q, qrot, rope_cs, B, S, Hq, D, 0, st)) return rc;
+    qk = qrot;
+  }
   if (int rc = run_prepare(o, dO, lse, B, Hq, S, D, w, p, !det, st)) return rc;
-  if (int rc = run_main(q, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, w, p, det, st, dev)) return rc;
-  if (det) return run_dq_pass(q, k, v, dO, dq, B, Hq, Hkv, S, D, scale, causal, w, p, st, dev);
-  return run_finalize(dq, B, Hq, S, D, p, st);
+  if (int rc = run_main(qk, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, w, p, det, st, dev, rope_cs))
+    return rc;
+  if (det) return run_dq_pass(qk, k, v, dO, dq, B, Hq, Hkv, S, D, scale, causal, w, p, st, dev, rope_cs);
+  return run_finalize(dq, B, Hq, S, D, p, st, rope_cs);
 }
 
 }  // namespace
@@ -403,6 +449,62 @@ extern "C" int axis_attn_bwd_det(const void* q, const void* k, const void* v, co
                                  void* stream) {
   return run_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, workspace, workspace_bytes,
                  stream, true);
+}
+
+// ----------------------------------------------------------------------------
+// Rotary position embedding (RoPE) of Q and K, fused with the attention.
+
+extern "C" int axis_attn_rope_table(double* cs, int S, int D, double base, void* stream) {
+  if (!cs) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(cs)) return AXIS_ATTN_ERR_ALIGN;
+  if (S < 1 || D < 8 || D % 8 != 0 || !(std::isfinite(base) && base > 1.0)) return AXIS_ATTN_ERR_SHAPE;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  const long long n = (long long)S * (D / 2);
+  const unsigned grid = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  rope_table_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<double2*>(cs), n, D / 2,
+                                                                         std::log2(base));
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+extern "C" int axis_attn_rope(const void* x, void* y, const double* cs, int B, int S, int H, int D, int inverse,
+                              void* stream) {
+  if (!x || !y || !cs) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(cs)) return AXIS_ATTN_ERR_ALIGN;
+  if (B < 1 || S < 1 || H < 1 || D < 8 || D % 8 != 0 || (long long)B * S * H * D >= (1LL << 40))
+    return AXIS_ATTN_ERR_SHAPE;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  return run_rope(x, y, cs, B, S, H, D, inverse, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int axis_attn_fwd_rope(const void* q, const void* k, const void* v, const double* cs, void* o, float* lse,
+                                  void* k_rot, int B, int Hq, int Hkv, int S, int D, float scale, int causal,
+                                  void* stream) {
+  if (!q || !k || !v || !cs || !o || !lse || !k_rot) return AXIS_ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(cs) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(k_rot))
+    return AXIS_ATTN_ERR_ALIGN;
+  if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
+  int dev = 0;
+  if (int rc = check_device(&dev)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (int rc = run_rope(k, k_rot, cs, B, S, Hkv, D, 0, st)) return rc;
+  return run_fwd(q, k_rot, v, o, lse, B, Hq, Hkv, S, D, scale, causal, cs, st, dev);
+}
+
+extern "C" size_t axis_attn_bwd_rope_workspace_bytes(int B, int Hq, int Hkv, int S, int D, int deterministic) {
+  if (check_shape(B, Hq, Hkv, S, D, 1.f) != AXIS_ATTN_OK) return 0;
+  return ws_layout(B, Hq, S, D, deterministic != 0, true).total;
+}
+
+extern "C" int axis_attn_bwd_rope(const void* q, const void* k_rot, const void* v, const double* cs, const void* o,
+                                  const void* dO, const float* lse, void* dq, void* dk, void* dv, int B, int Hq,
+                                  int Hkv, int S, int D, float scale, int causal, int deterministic,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!cs) return AXIS_ATTN_ERR_NULL;
+  return run_bwd(q, k_rot, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, workspace, workspace_bytes,
+                 stream, deterministic != 0, cs);
 }
 
 // ----------------------------------------------------------------------------

@@ -181,6 +181,53 @@ int axis_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
                           void* stream);
 
 /*
+ * Rotary position embedding (RoPE) of Q and K, fused with the attention.  The
+ * axiomlm page (PyPI) lists RoPE among its Key Features, and its Quick Start
+ * (section 8) computes precompute_rope_frequencies(dim, end) and then
+ * apply_rope(q, k, freqs_cis) before attention; it gives no formula.  The
+ * reading taken (the complex-pair form the name freqs_cis points to): in the
+ * row at sequence position s the pair (x[2p], x[2p+1]) is turned by the angle
+ * s * theta_p, theta_p = base^(-2p/D):
+ *   x'[2p] = x[2p] cos - x[2p+1] sin,   x'[2p+1] = x[2p] sin + x[2p+1] cos.
+ *
+ * axis_attn_rope_table: cs[s * D/2 + p] = (cos, sin)(s * theta_p) as fp64
+ *   pairs, [S][D/2][2] (the page's freqs_cis).  fp64 because the rotated q and
+ *   k are stored in bf16: the rotation is computed in fp64 and rounded once,
+ *   so the stored values are the correctly rounded rotation.
+ *   Requirements: 8 <= D, D % 8 == 0, base finite and > 1, cs 16-byte aligned.
+ * axis_attn_rope: y = the rotation of x (inverse != 0: the transposed rotation,
+ *   which carries gradients back), x, y [B, S, H, D] bf16 (y may be x), cs
+ *   from axis_attn_rope_table for at least S positions.  HBM-bound.
+ * axis_attn_fwd_rope: the forward of axis_attn_fwd() on the rotated q and k:
+ *   o, lse as for softmax(scale * (R q)(R k)^T) V.  q and k are the caller's
+ *   unrotated tensors.  The call rotates K once into k_rot (caller-owned,
+ *   [B, S, Hkv, D] bf16; the backward reads it), and the kernel rotates each
+ *   Q tile in shared memory right after its TMA load, so the rotated Q never
+ *   reaches device memory.  (K tiles are re-read by every query block; turning
+ *   them once up front costs less than turning them at every load.)
+ * axis_attn_bwd_rope: the gradients with respect to the UNROTATED q and k (and
+ *   v) of that forward: it takes k_rot from the forward, rotates q once into
+ *   the workspace, runs the backward of axis_attn_bwd() (deterministic != 0:
+ *   that of axis_attn_bwd_det()) and applies the transposed rotation to dQ in
+ *   the finalize step and to dK in the main kernel's epilogue.  Workspace:
+ *   axis_attn_bwd_rope_workspace_bytes() (the plain backward's plus the
+ *   rotated q).
+ * Arguments, layouts, requirements and errors otherwise as for axis_attn_fwd()
+ * and axis_attn_bwd(); cs must be 16-byte aligned and cover S positions of D.
+ */
+int axis_attn_rope_table(double* cs, int S, int D, double base, void* stream);
+int axis_attn_rope(const void* x, void* y, const double* cs, int B, int S, int H, int D, int inverse,
+                   void* stream);
+int axis_attn_fwd_rope(const void* q, const void* k, const void* v, const double* cs, void* o,
+                       float* lse, void* k_rot, int B, int Hq, int Hkv, int S, int D, float scale,
+                       int causal, void* stream);
+size_t axis_attn_bwd_rope_workspace_bytes(int B, int Hq, int Hkv, int S, int D, int deterministic);
+int axis_attn_bwd_rope(const void* q, const void* k_rot, const void* v, const double* cs,
+                       const void* o, const void* dO, const float* lse, void* dq, void* dk,
+                       void* dv, int B, int Hq, int Hkv, int S, int D, float scale, int causal,
+                       int deterministic, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Decode step against a paged KV cache: for each sequence b, the new token's
  * query row attends to every key cached for b (itself included, so no mask is
  * needed).  This is the per-token step of the axiomlm inference engine

@@ -64,3 +64,25 @@ def assert_close(o, lse, dq, dk, dv, ro, rlse, rdq, rdk, rdv, tag="", S=None):
     assert eo <= TOL_O and el <= TOL_LSE, msg
     assert eq <= tg and ek <= tg and ev <= tg, msg
     return msg
+
+
+def bf16_rn_from_f64(x):
+    """Round float64 values to bf16 directly (round to nearest, ties to even:
+    one rounding, from the fp64 value), returned as a torch bf16 tensor.  The
+    rotated attention inputs are stored in bf16, so the oracle's fp64 rotation
+    is rounded this way before it enters the oracle's attention.  Normal-range
+    values only (the attention inputs); smaller magnitudes flush to zero."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    u = x.view(np.uint64)
+    sign = ((u >> np.uint64(63)) << np.uint64(15)).astype(np.int64)
+    e = ((u >> np.uint64(52)) & np.uint64(0x7FF)).astype(np.int64) - 1023 + 127
+    keep = ((u >> np.uint64(45)) & np.uint64(0x7F)).astype(np.int64)
+    rest = u & np.uint64((1 << 45) - 1)
+    half = np.uint64(1 << 44)
+    up = (rest > half) | ((rest == half) & ((keep & 1) == 1))
+    keep = keep + up.astype(np.int64)
+    carry = keep == 0x80
+    keep = np.where(carry, 0, keep)
+    e = e + carry.astype(np.int64)
+    bits = np.where(e <= 0, sign, sign | (e << 7) | keep)
+    return torch.from_numpy(bits.astype(np.uint16).view(np.int16).copy()).view(torch.bfloat16)
