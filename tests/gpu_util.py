@@ -44,24 +44,43 @@ def max_abs(got, ref) -> float:
     return float(np.abs(f64(got) - f64(ref)).max()) if np.size(ref) else 0.0
 
 
-# Sequences shorter than this carry the whole gradient norm in one or two dS
-# entries.  Each inherits the bf16 rounding of O through Dr = rowsum(dO * O)
-# (the kernel reads the stored bf16 O, the oracle its fp64 O): the absolute
-# error of Dr is about 2^-9 sqrt(D) |dO| |O|, while |dP_ij - Dr_i| can be of
-# order one, so a single entry can be off by a few 1e-2 relatively.  With
-# S >= 16 the error averages over rows and stays near 3e-3.  Short sequences
-# are checked with this looser relative bound instead.
-SHORT_S = 16
-TOL_GRAD_SHORT = 6e-2
+# Short sequences carry the whole gradient norm in a few dS entries.  Each
+# inherits the bf16 rounding of O through Dr = rowsum(dO * O) (the kernel reads
+# the stored bf16 O, the oracle its fp64 O): the absolute error of Dr is about
+# 2^-9 sqrt(D) |dO| |O|, while |dP_ij - Dr_i| can be of order one, so with one
+# or two visible keys a single entry can be off by a few 1e-3 to 1e-2.  The
+# bounds below are the worst relative L2 error measured on a B200 over 12 seeds
+# x 5 shapes per S (B=1; (Hq, Hkv, D, causal) in (1,1,64,c), (4,2,64,c),
+# (2,1,128,c), (4,4,64,nc), (8,2,128,nc)), times 1.5: S=1 2.2e-3, S=2 2.09e-2,
+# S=3 8.4e-3, S=4 1.01e-2, S=5 8.7e-3, S=6 8.8e-3; from S=7 on <= 4.8e-3.
+GRAD_TOL_SHORT = {2: 3.2e-2, 3: 1.3e-2, 4: 1.6e-2, 5: 1.4e-2, 6: 1.4e-2}
+
+
+def grad_tol(S):
+    return GRAD_TOL_SHORT.get(S, TOL_GRAD) if S is not None else TOL_GRAD
+
+
+# O is stored in bf16, whose rounding alone reaches half an ulp, up to
+# 2^-8 |O|: above |O| = 2.56 that exceeds 1e-2 (rows with few visible keys
+# can have |O| > 4).  The O check is therefore max(1e-2, one bf16 ulp of the
+# reference, 2^-7 |O_ref|) element by element: 1e-2 wherever |O_ref| < 1.28.
+def o_excess(o, ro):
+    """max over elements of |o - ro| / max(TOL_O, 2^-7 |ro|): <= 1 passes."""
+    o, ro = f64(o), f64(ro)
+    if not np.size(ro):
+        return 0.0
+    return float((np.abs(o - ro) / np.maximum(TOL_O, np.abs(ro) * 2.0 ** -7)).max())
 
 
 def assert_close(o, lse, dq, dk, dv, ro, rlse, rdq, rdk, rdv, tag="", S=None):
     eo, el = max_abs(o, ro), max_abs(lse, rlse)
     eq, ek, ev = rel_l2(dq, rdq), rel_l2(dk, rdk), rel_l2(dv, rdv)
-    tg = TOL_GRAD_SHORT if (S is not None and S < SHORT_S) else TOL_GRAD
-    msg = f"{tag}: O {eo:.2e} LSE {el:.2e} dQ {eq:.2e} dK {ek:.2e} dV {ev:.2e} (grad tol {tg:g})"
+    tg = grad_tol(S)
+    xo = o_excess(o, ro)
+    msg = (f"{tag}: O {eo:.2e} (bound use {xo:.2f}) LSE {el:.2e} dQ {eq:.2e} dK {ek:.2e} dV {ev:.2e} "
+           f"(grad tol {tg:g})")
     assert np.isfinite([eo, el, eq, ek, ev]).all(), msg
-    assert eo <= TOL_O and el <= TOL_LSE, msg
+    assert xo <= 1.0 and el <= TOL_LSE, msg
     assert eq <= tg and ek <= tg and ev <= tg, msg
     return msg
 

@@ -135,3 +135,19 @@ def test_prefix_mean_property_at_scale():
     s_all = w.scale * torch.einsum("bshd,bhd->bhs", q.double(), k.double()[:, 0].repeat_interleave(G, 1))
     ref_lse = s_all + torch.log(torch.arange(1, w.S + 1, dtype=torch.float64))
     assert (lse.cpu().double() - ref_lse).abs().max() <= TOL_LSE
+
+
+@pytest.mark.parametrize("S", list(range(1, 17)))
+def test_short_sequences_over_seeds(oracle_mod, S):
+    """Every short length, several seeds and shapes, against the per-S bounds
+    (the measured worst case x 1.5; see gpu_util.GRAD_TOL_SHORT)."""
+    for seed in range(3):
+        for Hq, Hkv, D, causal in ((1, 1, 64, True), (4, 2, 64, True), (2, 1, 128, True), (4, 4, 64, False),
+                                   (8, 2, 128, False)):
+            q, k, v, do = make_inputs(1, Hq, Hkv, S, D, 7000 + 97 * seed + S)
+            sc = 1.0 / math.sqrt(D)
+            got = run_gpu(q, k, v, do, causal, sc)
+            ro, rl = oracle_mod.attn_fwd(q, k, v, sc, causal)
+            rdq, rdk, rdv, _ = oracle_mod.attn_bwd(q, k, v, do, sc, causal)
+            assert_close(*got, ro, rl, rdq, rdk, rdv, tag=f"S{S} seed{seed} Hq{Hq} Hkv{Hkv} D{D} c{int(causal)}",
+                         S=S)
