@@ -401,8 +401,9 @@ def time_rope(aa, w, seed, dev, steps, flush, p_meas):
     B, Hq, Hkv, S, D = w.B, w.Hq, w.Hkv, w.S, w.D
     cs = aa.rope_table(S, D, 10000.0, device=dev)
     o, lse = torch.empty_like(q), torch.empty((B, Hq, S), device=dev, dtype=torch.float32)
-    k_rot, dq, dk, dv = torch.empty_like(k), torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    wsb = aa.axis_attn_bwd_rope_workspace_bytes(B, Hq, Hkv, S, D, 0)
+    q_rot, k_rot = torch.empty_like(q), torch.empty_like(k)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsb = aa.axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D)
     ws = torch.empty(wsb, device=dev, dtype=torch.uint8)
     st = torch.cuda.current_stream(dev)
     import ctypes
@@ -411,12 +412,13 @@ def time_rope(aa, w, seed, dev, steps, flush, p_meas):
 
     def fwd():
         rc = aa.axis_attn_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), cs.data_ptr(), o.data_ptr(),
-                                   lse.data_ptr(), k_rot.data_ptr(), B, Hq, Hkv, S, D, w.scale, int(w.causal), sp)
+                                   lse.data_ptr(), q_rot.data_ptr(), k_rot.data_ptr(), B, Hq, Hkv, S, D, w.scale,
+                                   int(w.causal), sp)
         if rc:
             raise aa.AxisAttnError(rc, "axis_attn_fwd_rope")
 
     def bwd():
-        rc = aa.axis_attn_bwd_rope(q.data_ptr(), k_rot.data_ptr(), v.data_ptr(), cs.data_ptr(), o.data_ptr(),
+        rc = aa.axis_attn_bwd_rope(q_rot.data_ptr(), k_rot.data_ptr(), v.data_ptr(), cs.data_ptr(), o.data_ptr(),
                                    do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq,
                                    Hkv, S, D, w.scale, int(w.causal), 0, ws.data_ptr(), wsb, sp)
         if rc:
@@ -440,9 +442,9 @@ def time_rope(aa, w, seed, dev, steps, flush, p_meas):
     fwd_tf, bwd_tf = w.fwd_flops / f_ms / 1e9, w.bwd_flops / b_ms / 1e9
     return {"fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf, "fwd_ms": f_ms, "bwd_ms": b_ms, "steps": steps,
             "fwd_frac_of_measured": fwd_tf / p_meas, "bwd_frac_of_measured": bwd_tf / p_meas,
-            "note": "fwd: K rotated once by a prologue kernel, Q tiles rotated in shared memory; bwd: Q rotated "
-                    "once into the workspace, the transposed rotation fused into the dQ finalize and the dK "
-                    "epilogue; times include the rotations"}
+            "note": "fwd: Q and K rotated once by an HBM-bound prologue pass, then the forward kernel; bwd: the "
+                    "transposed rotation fused into the dQ finalize and the dK epilogue; times include the "
+                    "rotations"}
 
 
 # Decode workloads: one new token per sequence against a paged KV cache of

@@ -31,7 +31,6 @@ EXPORTS = (
     "axis_attn_rope_table",
     "axis_attn_rope",
     "axis_attn_fwd_rope",
-    "axis_attn_bwd_rope_workspace_bytes",
     "axis_attn_bwd_rope",
     "axis_attn_decode_workspace_bytes",
     "axis_attn_decode",
@@ -99,10 +98,8 @@ def load():
             lib.axis_attn_rope_table.restype = i
             lib.axis_attn_rope.argtypes = [vp] * 3 + [i] * 5 + [vp]
             lib.axis_attn_rope.restype = i
-            lib.axis_attn_fwd_rope.argtypes = [vp] * 7 + [i] * 5 + [f, i, vp]
+            lib.axis_attn_fwd_rope.argtypes = [vp] * 8 + [i] * 5 + [f, i, vp]
             lib.axis_attn_fwd_rope.restype = i
-            lib.axis_attn_bwd_rope_workspace_bytes.argtypes = [i] * 6
-            lib.axis_attn_bwd_rope_workspace_bytes.restype = sz
             lib.axis_attn_bwd_rope.argtypes = [vp] * 10 + [i] * 5 + [f, i, i, vp, sz, vp]
             lib.axis_attn_bwd_rope.restype = i
             lib.axis_attn_decode_workspace_bytes.argtypes = [i] * 6
@@ -176,17 +173,13 @@ def axis_attn_rope(x, y, cs, B, S, H, D, inverse, stream) -> int:
     return load().axis_attn_rope(x, y, cs, B, S, H, D, inverse, stream)
 
 
-def axis_attn_fwd_rope(q, k, v, cs, o, lse, k_rot, B, Hq, Hkv, S, D, scale, causal, stream) -> int:
-    return load().axis_attn_fwd_rope(q, k, v, cs, o, lse, k_rot, B, Hq, Hkv, S, D, scale, causal, stream)
+def axis_attn_fwd_rope(q, k, v, cs, o, lse, q_rot, k_rot, B, Hq, Hkv, S, D, scale, causal, stream) -> int:
+    return load().axis_attn_fwd_rope(q, k, v, cs, o, lse, q_rot, k_rot, B, Hq, Hkv, S, D, scale, causal, stream)
 
 
-def axis_attn_bwd_rope_workspace_bytes(B, Hq, Hkv, S, D, deterministic) -> int:
-    return int(load().axis_attn_bwd_rope_workspace_bytes(B, Hq, Hkv, S, D, deterministic))
-
-
-def axis_attn_bwd_rope(q, k_rot, v, cs, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, deterministic,
+def axis_attn_bwd_rope(q_rot, k_rot, v, cs, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, deterministic,
                        workspace, workspace_bytes, stream) -> int:
-    return load().axis_attn_bwd_rope(q, k_rot, v, cs, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
+    return load().axis_attn_bwd_rope(q_rot, k_rot, v, cs, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,
                                      deterministic, workspace, workspace_bytes, stream)
 
 
@@ -363,8 +356,9 @@ def _check_cs(cs, S, D, where):
 
 
 def attention_forward_rope(q, k, v, cs, causal: bool = True, scale: float | None = None, stream=None):
-    """Forward with RoPE fused: (o, lse, k_rot) for unrotated bf16 q, k and the
-    table cs of rope_table(); k_rot (the rotated keys) feeds attention_backward_rope."""
+    """Forward with RoPE: (o, lse, q_rot, k_rot) for unrotated bf16 q, k and the
+    table cs of rope_table(); q_rot, k_rot (the rotated inputs) feed
+    attention_backward_rope."""
     import torch
 
     where = "attention_forward_rope"
@@ -375,21 +369,23 @@ def attention_forward_rope(q, k, v, cs, causal: bool = True, scale: float | None
     with torch.cuda.device(dev):
         o = torch.empty_like(q)
         l = torch.empty((B, Hq, S), device=dev, dtype=torch.float32)
-        k_rot = torch.empty_like(k)
+        q_rot, k_rot = torch.empty_like(q), torch.empty_like(k)
         rc = axis_attn_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), cs.data_ptr(), o.data_ptr(), l.data_ptr(),
-                                k_rot.data_ptr(), B, Hq, Hkv, S, D, scale, int(causal), _stream(stream, dev))
+                                q_rot.data_ptr(), k_rot.data_ptr(), B, Hq, Hkv, S, D, scale, int(causal),
+                                _stream(stream, dev))
     if rc:
         raise AxisAttnError(rc, "axis_attn_fwd_rope")
-    return o, l, k_rot
+    return o, l, q_rot, k_rot
 
 
-def attention_backward_rope(q, k_rot, v, cs, o, lse, dout, causal: bool = True, scale: float | None = None,
+def attention_backward_rope(q_rot, k_rot, v, cs, o, lse, dout, causal: bool = True, scale: float | None = None,
                             deterministic: bool = False, stream=None):
     """Gradients (dq, dk, dv) with respect to the unrotated q, k of
-    attention_forward_rope (k_rot is its third output)."""
+    attention_forward_rope, from its rotated inputs q_rot, k_rot."""
     import torch
 
     where = "attention_backward_rope"
+    q = q_rot
     B, Hq, Hkv, S, D = _dims(q, k_rot, v, where)
     _check_cs(cs, S, D, where)
     _check_tensor(o, "o", (B, S, Hq, D), torch.bfloat16, where)
@@ -397,7 +393,7 @@ def attention_backward_rope(q, k_rot, v, cs, o, lse, dout, causal: bool = True, 
     _check_tensor(lse, "lse", (B, Hq, S), torch.float32, where)
     dev = _check_device({"q": q, "k_rot": k_rot, "v": v, "cs": cs, "o": o, "lse": lse, "dout": dout}, where)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    need = axis_attn_bwd_rope_workspace_bytes(B, Hq, Hkv, S, D, int(deterministic))
+    need = (axis_attn_bwd_det_workspace_bytes if deterministic else axis_attn_bwd_workspace_bytes)(B, Hq, Hkv, S, D)
     with torch.cuda.device(dev):
         ws = torch.empty(need, device=dev, dtype=torch.uint8)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k_rot), torch.empty_like(v)

@@ -35,12 +35,17 @@
 
 namespace axis_attn {
 
-// Compute warps (P^T, dS^T): 8 (two per SM sub-partition, each thread a key
-// row and half the query columns, in 32-column chunks) or 16 (four per
-// sub-partition, a quarter of the columns, in 16-column chunks; more warps to
-// hide the TMEM, MUFU and barrier latencies of each step).
-#ifndef AXIS_ATTN_BWD_CW
-#define AXIS_ATTN_BWD_CW 8
+// Compute warps (P^T, dS^T) at head dim 64 / 128: 16 (four per SM
+// sub-partition, each thread a key row and a quarter of the 128 query
+// columns, in 16-column chunks: more warps hide the TMEM, MUFU and barrier
+// latencies of a step; measured 11% faster than 8 at D = 64) or 8 (two per
+// sub-partition, half of the columns in 32-column chunks: at D = 128 a step
+// has only 64 query columns, and 16 columns a thread measured 5% slower).
+#ifndef AXIS_ATTN_BWD_CW64
+#define AXIS_ATTN_BWD_CW64 16
+#endif
+#ifndef AXIS_ATTN_BWD_CW128
+#define AXIS_ATTN_BWD_CW128 8
 #endif
 // Unroll factor of the per-step loop over a compute thread's TMEM chunks.
 #ifndef AXIS_ATTN_BWD_CC_UNROLL
@@ -70,8 +75,14 @@ struct BwdCfg {
   static constexpr uint32_t QTILE = NSLAB * QSLAB;
   static constexpr uint32_t PS_BYTES = (BM / 64) * 128 * 128;  // dS^T: 128 keys x BM bf16
   static constexpr int ST = 3;                     // Q / dO / LSE / Dr ring depth
-  static constexpr int COLS = BM / (AXIS_ATTN_BWD_CW / 4);  // query columns per compute thread
-  static constexpr int SUBW = AXIS_ATTN_BWD_CW == 16 ? 16 : 32;  // columns per TMEM load
+  // warps: 0 .. CW-1 compute; CW loads; CW+1 score MMAs (and TMEM owner);
+  // CW+2 TMA reduce-adds; CW+3 gradient MMAs; CW+4 .. CW+7 dQ read-out
+  static constexpr int CW = HD == 64 ? AXIS_ATTN_BWD_CW64 : AXIS_ATTN_BWD_CW128;
+  static_assert(CW == 8 || CW == 16, "8 or 16 compute warps");
+  static constexpr int THREADS = (CW + 8) * 32;
+  static constexpr int W_LOAD = CW, W_MMA = CW + 1, W_RED = CW + 2, W_GRAD = CW + 3, W_DQ0 = CW + 4;
+  static constexpr int COLS = BM / (CW / 4);                     // query columns per compute thread
+  static constexpr int SUBW = CW == 16 ? 16 : 32;                // columns per TMEM load
   static constexpr int NSUB = COLS / SUBW;                       // loads per step
   // dQ tile staged for the TMA reduce-add: fp32, four 128B-swizzled boxes of
   // 32 columns x 64 rows (D = 64: rows = queries, columns = features; D = 128:
@@ -107,16 +118,8 @@ struct BwdCfg {
 // score MMAs and owns TMEM; CW+2 issues the TMA reduce-adds of the dQ tiles
 // into the fp32 accumulator; CW+3 issues the gradient MMAs; CW+4 .. CW+7 copy
 // each dQ tile from TMEM into the swizzled staging tile (one TMEM lane quarter
-// each), off the compute warps' critical path.
-constexpr int BWD_CW = AXIS_ATTN_BWD_CW;
+// each), off the compute warps' critical path (BwdCfg).
 constexpr int BWD_CC_UNROLL = AXIS_ATTN_BWD_CC_UNROLL;
-static_assert(BWD_CW == 8 || BWD_CW == 16, "8 or 16 compute warps");
-constexpr int BWD_THREADS = (BWD_CW + 8) * 32;
-constexpr int BWD_WARP_LOAD = BWD_CW;
-constexpr int BWD_WARP_MMA = BWD_CW + 1;
-constexpr int BWD_WARP_RED = BWD_CW + 2;
-constexpr int BWD_WARP_GRAD = BWD_CW + 3;
-constexpr int BWD_WARP_DQ0 = BWD_CW + 4;
 
 enum BwdSite { B_KV = 21, B_QEMPTY, B_QFULL, B_SPFREE, B_PDSFULL, B_DQFREE, B_SPFULL, B_DQFULL, B_FIN, B_PDSFREE,
                B_STGFULL, B_STGFREE };
@@ -158,12 +161,14 @@ __device__ __forceinline__ void bwd_item(int BKV, int nkv, int x, int& j, int& b
 }
 
 template <int HD, bool CAUSAL>
-__global__ void __launch_bounds__(BWD_THREADS, 1)
+__global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
   using C = BwdCfg<HD>;
   constexpr int BM = C::BM, ST = C::ST, COLS = C::COLS, SUBW = C::SUBW, NSUB = C::NSUB;
+  constexpr int BWD_CW = C::CW, BWD_WARP_LOAD = C::W_LOAD, BWD_WARP_MMA = C::W_MMA, BWD_WARP_RED = C::W_RED,
+                BWD_WARP_GRAD = C::W_GRAD, BWD_WARP_DQ0 = C::W_DQ0;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -576,9 +581,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 
 // -Dr = -rowsum(dO * O) (fp32) and -LSE2 = -LSE * log2(e) per (b, h, i); rows
 // S..S_pad-1 of each (b, h) get 0 and -inf (so their P is exactly 0).  Also
-// zeroes the dQ accumulator.  HBM-bound: the rows are visited in memory order
-// ([B, S, Hq] for O and dO), D/8 threads per row with one 16-byte load each of
-// O and dO, and a shuffle reduction inside the row's thread group.
+// zeroes the dQ accumulator.  HBM-bound: D/8 threads per row with one 16-byte
+// load each of O and dO (every row a whole 128- or 256-byte line) and a shuffle
+// reduction inside the row's thread group.  Rows are visited in [B, Hq, S]
+// order, the order of the two fp32 outputs, so that consecutive rows of a warp
+// write consecutive floats (in [B, S, Hq] order each 4-byte result would sit in
+// a 32-byte sector of its own).
 template <int HD>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                             const __nv_bfloat16* __restrict__ dout,
@@ -588,18 +596,21 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
   constexpr int TPR = HD / 8;  // threads per row
   const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t nthreads = (size_t)gridDim.x * blockDim.x;
-  const size_t real_rows = (size_t)rows / S_pad * S;  // B * Hq * S, in [B, S, Hq] order
+  const size_t real_rows = (size_t)rows / S_pad * S;  // B * Hq * S, in [B, Hq, S] order
   const size_t total = real_rows * TPR;
   const size_t warp0 = gtid - (threadIdx.x & 31);  // warp-uniform loop: every lane joins the shuffles
   for (size_t tw = warp0; tw < total; tw += nthreads) {
     const size_t t = tw + (threadIdx.x & 31);
     const bool act = t < total;
-    const size_t r = t / TPR;
+    const size_t r = t / TPR;  // (b * Hq + h) * S + i
     const int part = (int)(t % TPR);
+    const int i = (int)(r % S);
+    const size_t bh = r / S;
+    const size_t src = ((bh / Hq) * S + i) * Hq + bh % Hq;  // row of O, dO in [B, S, Hq]
     float d = 0.f;
     if (act) {
-      const uint4 x = reinterpret_cast<const uint4*>(o + r * HD)[part];
-      const uint4 y = reinterpret_cast<const uint4*>(dout + r * HD)[part];
+      const uint4 x = reinterpret_cast<const uint4*>(o + src * HD)[part];
+      const uint4 y = reinterpret_cast<const uint4*>(dout + src * HD)[part];
       const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -612,10 +623,6 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off, TPR);
     if (act && part == 0) {
-      const int h = (int)(r % Hq);
-      const size_t bi = r / Hq;  // b * S + i
-      const int i = (int)(bi % S);
-      const size_t bh = (bi / S) * Hq + h;
       ndr[bh * S_pad + i] = -d;
       nlse2[bh * S_pad + i] = -lse[bh * S + i] * 1.4426950408889634f;
     }

@@ -40,7 +40,6 @@
 // take turns) P0 [128,192) P1 [192,256) O0 [256,384) O1 [384,512).
 #pragma once
 
-#include "attn_rope.cuh"
 #include "sm100_ptx.cuh"
 
 namespace axis_attn {
@@ -52,7 +51,6 @@ struct FwdArgs {
   float scale_log2;  // scale * log2(e)
   int n_qblocks;     // ceil(S / 256)
   int n_items;       // n_qblocks * B * Hq
-  const double2* rope_cs;  // RoPE kernel only: (cos, sin) table [S][HD/2], fp64
 };
 
 // The it-th item of this CTA: snake order over the grid (even passes left to
@@ -104,7 +102,7 @@ struct FwdCfg {
   static constexpr bool SHARED_S = HD == 128;
   static constexpr uint32_t T_P = SHARED_S ? 128 : 384, T_O = 256;
   static __host__ __device__ constexpr uint32_t t_s(int t) { return SHARED_S ? 0u : 128u * t; }
-  static constexpr int NBAR = 24 + 2 * KST + 2 * VST;
+  static constexpr int NBAR = 23 + 2 * KST + 2 * VST;
   static constexpr uint32_t XCH_OFF = (2 + KST + VST) * TILE;  // row-max / row-sum exchange
   static constexpr uint32_t XCH_BYTES = 2 * 2 * 2 * 128 * 4;   // [parity][tile][half][row] fp32
   static constexpr uint32_t BAR_OFF = XCH_OFF + XCH_BYTES;
@@ -207,18 +205,23 @@ __device__ __forceinline__ void xpose_chunks(uint32_t (&c)[4 * N], int lane) {
 // owner), 18 TMA producer of V, 19 P V issuer.  Five warps per SM
 // sub-partition leave 96 registers a thread: half a row of scores (64) plus
 // its packed probabilities.
-// With RoPE fused (ROPE = true) the whole V-producer warp also rotates each
-// item's Q tiles in shared memory after they land and before the S issuer
-// reads them (a 21st warp would put six warps on one SM sub-partition and
-// cut every thread to 80 registers).
-constexpr int FWD_THREADS = 640;
-constexpr int FWD_SOFTMAX_WARPS = 16;
-constexpr int FWD_WARP_LOAD = 16;
-constexpr int FWD_WARP_MMA = 17;
-constexpr int FWD_WARP_LOADV = 18;
-constexpr int FWD_WARP_PV = 19;
+// Softmax layout: 0 = two warps per 32-row group, each a half row (64
+// columns; partial maxima and sums meet through shared memory), 20 warps,
+// 96 registers; 1 = one thread per whole 128-column row (max and sum stay in
+// the thread), 8 softmax warps + 4 role warps, up to 168 registers.
+#ifndef AXIS_ATTN_FWD_ROWTHREAD
+#define AXIS_ATTN_FWD_ROWTHREAD 0
+#endif
+constexpr bool FWD_ROWTHREAD = AXIS_ATTN_FWD_ROWTHREAD != 0;
+constexpr int FWD_SOFTMAX_WARPS = FWD_ROWTHREAD ? 8 : 16;
+constexpr int FWD_SMW_PER_TILE = FWD_SOFTMAX_WARPS / 2;  // softmax warps of one query tile
+constexpr int FWD_THREADS = (FWD_SOFTMAX_WARPS + 4) * 32;
+constexpr int FWD_WARP_LOAD = FWD_SOFTMAX_WARPS;
+constexpr int FWD_WARP_MMA = FWD_SOFTMAX_WARPS + 1;
+constexpr int FWD_WARP_LOADV = FWD_SOFTMAX_WARPS + 2;
+constexpr int FWD_WARP_PV = FWD_SOFTMAX_WARPS + 3;
 
-template <int HD, bool CAUSAL, bool ROPE>
+template <int HD, bool CAUSAL>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
@@ -251,8 +254,6 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   auto bar_xch = [&](int t, int wq) { return bars + 8u * (B2 + 11 + 4 * t + wq); };
   // O_t has been read out by the epilogue: the next item may overwrite it
   auto bar_ofree = [&](int t) { return bars + 8u * (B2 + 19 + t); };
-  // RoPE kernel: the Q copies land here; the rope warp then completes bar_q
-  const uint32_t bar_qraw = bars + 8u * (B2 + 21);
   float* xch = reinterpret_cast<float*>(gbase + C::XCH_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::BAR_OFF + 8 * C::NBAR);
   volatile WaitCtl* abort = reinterpret_cast<volatile WaitCtl*>(gbase + C::BAR_OFF + 8 * C::NBAR + 4);
@@ -273,15 +274,14 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_sfull(t), 1);
-      mbar_init(bar_pfull(t), 8);
+      mbar_init(bar_pfull(t), FWD_SMW_PER_TILE);
       mbar_init(bar_o(t), 1);
-      mbar_init(bar_sfree(t), 8);
-      mbar_init(bar_tok(t), 8);
-      mbar_init(bar_ofree(t), 8);
+      mbar_init(bar_sfree(t), FWD_SMW_PER_TILE);
+      mbar_init(bar_tok(t), FWD_SMW_PER_TILE);
+      mbar_init(bar_ofree(t), FWD_SMW_PER_TILE);
       for (int wq = 0; wq < 4; ++wq) mbar_init(bar_xch(t, wq), 2);
     }
     mbar_init(bar_fin, 2);  // one commit from each MMA issuer
-    mbar_init(bar_qraw, 1);
     wait_ctl_init(abort);
     fence_barrier_init();
   }
@@ -294,46 +294,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (ROPE && warp == FWD_WARP_LOADV) {
-    // ===================================================== V producer + RoPE of Q
-    // Per item, the whole warp waits for the Q copies, rotates every Q row by
-    // its sequence position in shared memory, makes the generic-proxy writes
-    // visible to the tensor cores and releases Q to the S issuer (bar_q);
-    // then lane 0 streams the item's V tiles as the plain V producer does.
-    if (lane == 0) tma_prefetch_desc(&tm_v);
-    int g = 0;
-    bool ok = true;
-    for (int it = 0; ok; ++it) {
-      const int w = fwd_item(it);
-      if (w >= a.n_items) break;
-      const FwdItem I = fwd_decode(a, w, CAUSAL);
-      if (!(ok = wait_warp<true>(bar_qraw, it & 1, abort, F_Q))) break;
-      rope_tile_smem<HD>(sQ, SLAB, 128, 256 * I.m, a.S, a.rope_cs, lane);
-      if (I.has1) rope_tile_smem<HD>(sQ + TILE, SLAB, 128, 256 * I.m + 128, a.S, a.rope_cs, lane);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar_q);
-        for (int j = 0; j < I.nmax; ++j, ++g) {
-          const int s = g % VST;
-          if (g >= VST && !mbar_wait_bounded<true>(bar_vempty(s), ((g / VST) & 1) ^ 1, abort, F_EMPTY)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar_vfull(s), TILE);
-          for (int sl = 0; sl < C::NSLAB; ++sl)
-            tma_load_4d(sV + s * TILE + sl * SLAB, &tm_v, bar_vfull(s), 64 * sl, I.kvh, 128 * j, I.b);
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    }
-    // Drain (lane 0): every V copy started has landed before the CTA exits.
-    if (lane == 0) {
-      volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
-      for (int x = g - VST > 0 ? g - VST : 0; x < g; ++x)
-        mbar_wait_bounded<true>(bar_vfull(x % VST), (x / VST) & 1, &never, F_VFULL);
-    }
-  } else if (warp == FWD_WARP_LOAD || warp == FWD_WARP_LOADV) {
+  if (warp == FWD_WARP_LOAD || warp == FWD_WARP_LOADV) {
     // ===================================================== TMA producers
     // warp 16: per item Q (once the previous item's S products are done with
     // it), then the K ring (with an L2 prefetch of K and V PF tiles ahead);
@@ -356,13 +317,12 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         const FwdItem I = fwd_decode(a, w, CAUSAL);
         if (is_k) {
           if (it > 0 && !mbar_wait_bounded<true>(bar_qempty, (it - 1) & 1, abort, F_QEMPTY)) break;
-          const uint32_t bq = ROPE ? bar_qraw : bar_q;
-          mbar_arrive_expect_tx(bq, (I.has1 ? 2u : 1u) * TILE);
+          mbar_arrive_expect_tx(bar_q, (I.has1 ? 2u : 1u) * TILE);
           for (int sl = 0; sl < C::NSLAB; ++sl)
-            tma_load_4d(sQ + sl * SLAB, &tm_q, bq, 64 * sl, I.h, 256 * I.m, I.b);
+            tma_load_4d(sQ + sl * SLAB, &tm_q, bar_q, 64 * sl, I.h, 256 * I.m, I.b);
           if (I.has1)
             for (int sl = 0; sl < C::NSLAB; ++sl)
-              tma_load_4d(sQ + TILE + sl * SLAB, &tm_q, bq, 64 * sl, I.h, 256 * I.m + 128, I.b);
+              tma_load_4d(sQ + TILE + sl * SLAB, &tm_q, bar_q, 64 * sl, I.h, 256 * I.m + 128, I.b);
           ++nq;
           constexpr int PF = 4;
           auto prefetch = [&](int j) {
@@ -400,7 +360,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       // (each stage's most recent phase; nothing newer can have started).
       volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
       const int NS = is_k ? KST : VST;
-      if (is_k && nq > 0) mbar_wait_bounded<true>(ROPE ? bar_qraw : bar_q, (nq - 1) & 1, &never, F_Q);
+      if (is_k && nq > 0) mbar_wait_bounded<true>(bar_q, (nq - 1) & 1, &never, F_Q);
       for (int x = g - NS > 0 ? g - NS : 0; x < g; ++x)
         mbar_wait_bounded<true>(is_k ? bar_kfull(x % KST) : bar_vfull(x % VST), (x / NS) & 1, &never,
                           is_k ? F_KFULL : F_VFULL);
@@ -507,7 +467,167 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     mma_commit_w(bar_fin);
     volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
     wait_warp<true>(bar_fin, 0, &never, F_OFIN);
-  } else if (warp < FWD_SOFTMAX_WARPS) {
+  } else if (FWD_ROWTHREAD && warp < FWD_SOFTMAX_WARPS) {
+    // ===================================================== softmax (tile t, thread = whole row)
+    const int t = warp >> 2, wq = warp & 3;
+    const int r = wq * 32 + lane;                   // row in tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::t_s(t);
+    const uint32_t tO = tmem + lane_off + C::T_O + t * HD;
+    const uint32_t tP = tmem + lane_off + C::T_P + t * 64;
+    const float c = a.scale_log2;
+    const uint64_t cc2 = f2_pack(c, c);
+    int J = 0, A_o = 0;  // kv tiles of this tile so far; exponential phases of the other tile in earlier items
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      const int w = fwd_item(it);
+      if (w >= a.n_items) break;
+      const FwdItem I = fwd_decode(a, w, CAUSAL);
+      const int n_t = t == 0 ? I.n0 : I.n1, n_o = t == 0 ? I.n1 : I.n0;
+      const int qt = 2 * I.m + t;
+      const int row_g = qt * 128 + r;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < n_t; ++j, ++J) {
+        if (!wait_warp<true>(bar_sfull(t), J & 1, abort, F_SFULL)) { ok = false; break; }
+        tc_fence_after();
+        const bool masked = CAUSAL ? (j == qt) : (j == nkv - 1 && (a.S & 127) != 0);
+        int limit = 128;
+        if (masked) {
+          limit = a.S - 128 * j;
+          if (CAUSAL && r + 1 < limit) limit = r + 1;
+        }
+        // the 128-column row of S: option 1 keeps it all in registers (one TMEM
+        // pass); option 2 keeps columns 64-127 and reads columns 0-63 twice
+        // (for the row max, then for the exponentials), 64 fewer registers
+        constexpr bool TWO_PASS = AXIS_ATTN_FWD_ROWTHREAD == 2;
+        uint32_t v[4][32];
+        float mx;
+        if (TWO_PASS) {
+          tmem_ld32(tS, v[0]);
+          tmem_ld32(tS + 32, v[1]);
+          tmem_wait_ld();
+          if (masked) {
+            mask_row(v[0], 0, limit);
+            mask_row(v[1], 32, limit);
+          }
+          mx = fmaxf(row_max32(v[0]), row_max32(v[1]));
+          tmem_ld32(tS + 64, v[2]);
+          tmem_ld32(tS + 96, v[3]);
+          tmem_wait_ld();
+          if (masked) {
+            mask_row(v[2], 64, limit);
+            mask_row(v[3], 96, limit);
+          }
+          mx = fmaxf(mx, fmaxf(row_max32(v[2]), row_max32(v[3])));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) tmem_ld32(tS + 32 * k, v[k]);
+          tmem_wait_ld();
+          // S is in registers: its columns may take the next S
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_sfree(C::SHARED_S ? 0 : t));
+          if (masked) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mask_row(v[k], 32 * k, limit);
+          }
+          mx = fmaxf(fmaxf(row_max32(v[0]), row_max32(v[1])), fmaxf(row_max32(v[2]), row_max32(v[3])));
+        }
+        const float m_new = fmaxf(m_used, mx * c);
+        const bool resc = m_new > m_used + 8.0f;
+        float alpha = 1.f;
+        if (resc) {
+          alpha = ex2_approx(m_used - m_new);
+          m_used = m_new;
+        }
+        if (AXIS_ATTN_FWD_TOKEN) {
+          const int need = A_o + (t == 0 ? min(j, n_o) : min(j + 1, n_o));
+          if (need > 0 && !wait_warp<true>(bar_tok(t), (need - 1) & 1, abort, F_TOK)) { ok = false; break; }
+        }
+        // the previous P V must have landed before P_t is overwritten and O_t
+        // rescaled (it was issued a whole kv tile ago): then each 32-column
+        // chunk of P goes to TMEM as soon as it is packed
+        if (J > 0) {
+          if (!wait_warp<true>(bar_o(t), (J - 1) & 1, abort, F_OWAIT)) { ok = false; break; }
+          tc_fence_after();
+        }
+        const uint64_t nm2 = f2_pack(-m_used, -m_used);
+        uint64_t acc = f2_pack(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (TWO_PASS && k < 2) {  // second read of columns 0-63; then S may take the next product
+            tmem_ld32(tS + 32 * k, v[k]);
+            tmem_wait_ld();
+            if (masked) mask_row(v[k], 32 * k, limit);
+            if (k == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar_sfree(C::SHARED_S ? 0 : t));
+            }
+          }
+          uint32_t pk[16];
+          acc = exp_pairs<0, 16>(v[k], cc2, nm2, acc, pk);
+          tmem_st16(tP + 16 * k, pk);
+          if (AXIS_ATTN_FWD_TOKEN && k == 2) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tok(1 - t));
+          }
+        }
+        float rs_lo, rs_hi;
+        f2_unpack(acc, rs_lo, rs_hi);
+        l = l * alpha + (rs_lo + rs_hi);
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+          for (int cc = 0; cc < HD / 32; ++cc) {
+            uint32_t o32[32];
+            tmem_ld32(tO + cc * 32, o32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
+            tmem_st32(tO + cc * 32, o32);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && !(AXIS_ATTN_TEST_DROP_ARRIVE == 1 && J == 0 && t == 0)) mbar_arrive(bar_pfull(t));
+      }
+      A_o += n_o;
+      if (!ok || n_t == 0) continue;
+      // epilogue: O / l -> bf16, LSE = (m + log2 l) ln 2, all in this thread's row
+      if (!wait_warp<true>(bar_o(t), (J - 1) & 1, abort, F_OFIN)) { ok = false; break; }
+      tc_fence_after();
+      const float inv_l = __fdividef(1.f, l);  // l >= 1: the row max contributes 2^(>= 0)
+      constexpr int NCK = HD / 8;  // 16-byte chunks of the row
+      uint32_t pk[4 * NCK];
+#pragma unroll
+      for (int cc = 0; cc < HD / 32; ++cc) {
+        uint32_t o32[32];
+        tmem_ld32(tO + cc * 32, o32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[16 * cc + i] = pack_bf16x2(__uint_as_float(o32[2 * i]) * inv_l, __uint_as_float(o32[2 * i + 1]) * inv_l);
+      }
+      // O_t is out of TMEM: the next item's first P V may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_ofree(t));
+      // coalesced stores: after the chunk transpose, store k of the warp writes
+      // 32 / NCK whole rows (NCK consecutive lanes per row)
+      xpose_chunks<NCK>(pk, lane);
+      const int ck = lane % NCK, rbase = qt * 128 + wq * 32 + (lane / NCK) * NCK;
+#pragma unroll
+      for (int k = 0; k < NCK; ++k) {
+        const int row = rbase + k;
+        if (row < a.S) {
+          uint4* dst = reinterpret_cast<uint4*>(a.o + (((size_t)I.b * a.S + row) * a.Hq + I.h) * HD) + ck;
+          *dst = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+      }
+      if (row_g < a.S) a.lse[(size_t)I.bh * a.S + row_g] = (m_used + __log2f(l)) * 0.69314718055994531f;
+    }
+  } else if (!FWD_ROWTHREAD && warp < FWD_SOFTMAX_WARPS) {
     // ===================================================== softmax (tile t, half hf)
     const int t = warp >> 3, hf = (warp >> 2) & 1, wq = warp & 3;
     const int r = wq * 32 + lane;                   // row in tile == TMEM lane

@@ -1,7 +1,7 @@
 // attn_rope.cuh -- rotary position embedding (RoPE) for the attention inputs:
-// the cos/sin table, the HBM-bound rotation of a [B, S, H, D] tensor, and the
-// in-shared-memory rotation of a TMA-staged 128-row tile that the fused
-// forward applies to Q.
+// the cos/sin table, the HBM-bound rotation of a [B, S, H, D] tensor (forward
+// and transposed), and the transposed rotation of one gradient pair that the
+// backward's epilogues apply to dQ and dK.
 //
 // The axiomlm page (PyPI) lists RoPE among its Key Features and its Quick
 // Start (section 8) calls precompute_rope_frequencies(dim, end) and then
@@ -117,30 +117,6 @@ __global__ void __launch_bounds__(256) rope_apply_back_kernel(const uint4* x, ui
       o[k] = pack_bf16x2(g0, g1);
     }
     y[i] = make_uint4(o[0], o[1], o[2], o[3]);
-  }
-}
-
-// Rotate, in shared memory, the rows of a staged tile: `rows` rows of HD bf16
-// in 64-column slabs of 128-byte rows (128B swizzle, slab stride `slab`), row r
-// at sequence position pos0 + r (rows at or past S are left alone: their data
-// is the TMA's zero fill).  Called by one whole warp; lane l takes the 16-byte
-// words l, l + 32, ... of the tile.  The caller fences (async proxy) and
-// signals afterwards.
-template <int HD>
-__device__ __forceinline__ void rope_tile_smem(uint32_t tile, uint32_t slab, int rows, int pos0, int S,
-                                               const double2* __restrict__ cs, int lane) {
-  constexpr int WPR = HD / 8;  // 16-byte words per row
-  for (int i = lane; i < rows * WPR; i += 32) {
-    const int r = i / WPR, wd = i % WPR;
-    const int pos = pos0 + r;
-    if (pos >= S) continue;
-    const int sl = wd >> 3, c = wd & 7;
-    const uint32_t addr = tile + sl * slab + r * 128 + ((c ^ (r & 7)) << 4);
-    uint4 x;
-    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w) : "r"(addr));
-    const uint4 yv = rope_rotate8_f64(x, cs + (size_t)pos * (HD / 2) + 4 * wd);
-    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(yv.x), "r"(yv.y), "r"(yv.z), "r"(yv.w)
-                 : "memory");
   }
 }
 

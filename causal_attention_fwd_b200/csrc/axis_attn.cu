@@ -94,22 +94,20 @@ bool make_dq_map(CUtensorMap* map, const float* ptr, int BH, int S, int D) {
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct WsLayout {
-  size_t lse2, dr, dqacc, qrot, total;
+  size_t lse2, dr, dqacc, total;
   int S_pad;
 };
 
 // det: no dQ accumulator (the deterministic dQ pass keeps dQ in TMEM), so the
-// workspace is the two row sections only.  rope: plus the rotated Q (bf16
-// [B, S, Hq, D]) that the backward's kernels read in place of Q.
-WsLayout ws_layout(int B, int Hq, int S, int D, bool det = false, bool rope = false) {
+// workspace is the two row sections only.
+WsLayout ws_layout(int B, int Hq, int S, int D, bool det = false) {
   WsLayout w;
   w.S_pad = (S + 127) / 128 * 128;
   const size_t rows = (size_t)B * Hq * w.S_pad;
   w.lse2 = 0;
   w.dr = round256(rows * 4);
   w.dqacc = w.dr + round256(rows * 4);
-  w.qrot = w.dqacc + (det ? 0 : round256((size_t)B * Hq * S * D * 4));
-  w.total = w.qrot + (rope ? round256((size_t)B * S * Hq * D * 2) : 0);
+  w.total = w.dqacc + (det ? 0 : round256((size_t)B * Hq * S * D * 4));
   return w;
 }
 
@@ -137,10 +135,10 @@ int set_smem(K kernel, uint32_t bytes, int dev, bool (&done)[64]) {
   return AXIS_ATTN_OK;
 }
 
-template <int HD, bool CAUSAL, bool ROPE>
+template <int HD, bool CAUSAL>
 int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdArgs& a,
                cudaStream_t st, int dev) {
-  auto kern = attn_fwd_kernel<HD, CAUSAL, ROPE>;
+  auto kern = attn_fwd_kernel<HD, CAUSAL>;
   static bool done[64];
   if (int rc = set_smem(kern, FwdCfg<HD>::SMEM, dev, done)) return rc;
   // persistent: one CTA per SM (the kernel walks its share of the items)
@@ -149,10 +147,9 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
-// The forward kernel over (q, k, v); with a table, Q tiles are rotated in
-// shared memory (k must then hold the rotated keys already).
+// The forward kernel over (q, k, v).
 int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int S, int D,
-            float scale, int causal, const double* rope_cs, cudaStream_t st, int dev) {
+            float scale, int causal, cudaStream_t st, int dev) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, B, S, Hq, D, 128) || !make_map(&mk, k, B, S, Hkv, D, 128) ||
       !make_map(&mv, v, B, S, Hkv, D, 128))
@@ -167,19 +164,9 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
   a.n_qblocks = (S + 255) / 256;
   a.n_items = a.n_qblocks * B * Hq;
-  a.rope_cs = reinterpret_cast<const double2*>(rope_cs);
-  if (rope_cs) {
-    if (D == 64)
-      return causal ? launch_fwd<64, true, true>(mq, mk, mv, a, st, dev)
-                    : launch_fwd<64, false, true>(mq, mk, mv, a, st, dev);
-    return causal ? launch_fwd<128, true, true>(mq, mk, mv, a, st, dev)
-                  : launch_fwd<128, false, true>(mq, mk, mv, a, st, dev);
-  }
   if (D == 64)
-    return causal ? launch_fwd<64, true, false>(mq, mk, mv, a, st, dev)
-                  : launch_fwd<64, false, false>(mq, mk, mv, a, st, dev);
-  return causal ? launch_fwd<128, true, false>(mq, mk, mv, a, st, dev)
-                : launch_fwd<128, false, false>(mq, mk, mv, a, st, dev);
+    return causal ? launch_fwd<64, true>(mq, mk, mv, a, st, dev) : launch_fwd<64, false>(mq, mk, mv, a, st, dev);
+  return causal ? launch_fwd<128, true>(mq, mk, mv, a, st, dev) : launch_fwd<128, false>(mq, mk, mv, a, st, dev);
 }
 
 // y = R x (inverse: R^T x) for x, y [B, S, H, D] bf16 with the table cs [S][D/2].
@@ -213,7 +200,7 @@ int launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
   static bool done[64];
   if (int rc = set_smem(kern, BwdCfg<HD>::SMEM, dev, done)) return rc;
   const unsigned grid = (unsigned)((a.S + 127) / 128) * a.B * a.Hkv;
-  kern<<<grid, BWD_THREADS, BwdCfg<HD>::SMEM, st>>>(mq, mk, mv, mdo, mdq, a);
+  kern<<<grid, BwdCfg<HD>::THREADS, BwdCfg<HD>::SMEM, st>>>(mq, mk, mv, mdo, mdq, a);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
@@ -230,8 +217,7 @@ extern "C" int axis_attn_fwd(const void* q, const void* k, const void* v, void* 
   if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
-  return run_fwd(q, k, v, o, lse, B, Hq, Hkv, S, D, scale, causal, nullptr, static_cast<cudaStream_t>(stream),
-                 dev);
+  return run_fwd(q, k, v, o, lse, B, Hq, Hkv, S, D, scale, causal, static_cast<cudaStream_t>(stream), dev);
 }
 
 extern "C" size_t axis_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
@@ -399,8 +385,8 @@ int run_dq_pass(const void* q, const void* k, const void* v, const void* dO, voi
                 : launch_bwd_dq<128, false>(mq, mk, mv, mdo, a, st, dev);
 }
 
-// The backward; with a RoPE table, k holds the rotated keys, q is rotated into
-// the workspace first, and dQ, dK leave through the transposed rotation.
+// The backward; with a RoPE table, q and k hold the rotated inputs and dQ, dK
+// leave through the transposed rotation.
 int run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
             void* dk, void* dv, int B, int Hq, int Hkv, int S, int D, float scale, int causal, void* workspace,
             size_t workspace_bytes, void* stream, bool det, const double* rope_cs = nullptr) {
@@ -410,22 +396,16 @@ int run_bwd(const void* q, const void* k, const void* v, const void* o, const vo
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (rope_cs && !aligned16(rope_cs)))
     return AXIS_ATTN_ERR_ALIGN;
   if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
-  const WsLayout w = ws_layout(B, Hq, S, D, det, rope_cs != nullptr);
+  const WsLayout w = ws_layout(B, Hq, S, D, det);
   if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
   const WsPtrs p = ws_ptrs(workspace, w);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const void* qk = q;  // the queries the kernels read
-  if (rope_cs) {
-    void* qrot = static_cast<char*>(workspace) + w.qrot;
-    if (int rc = run_rope(q, qrot, rope_cs, B, S, Hq, D, 0, st)) return rc;
-    qk = qrot;
-  }
   if (int rc = run_prepare(o, dO, lse, B, Hq, S, D, w, p, !det, st)) return rc;
-  if (int rc = run_main(qk, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, w, p, det, st, dev, rope_cs))
+  if (int rc = run_main(q, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, w, p, det, st, dev, rope_cs))
     return rc;
-  if (det) return run_dq_pass(qk, k, v, dO, dq, B, Hq, Hkv, S, D, scale, causal, w, p, st, dev, rope_cs);
+  if (det) return run_dq_pass(q, k, v, dO, dq, B, Hq, Hkv, S, D, scale, causal, w, p, st, dev, rope_cs);
   return run_finalize(dq, B, Hq, S, D, p, st, rope_cs);
 }
 
@@ -479,32 +459,28 @@ extern "C" int axis_attn_rope(const void* x, void* y, const double* cs, int B, i
 }
 
 extern "C" int axis_attn_fwd_rope(const void* q, const void* k, const void* v, const double* cs, void* o, float* lse,
-                                  void* k_rot, int B, int Hq, int Hkv, int S, int D, float scale, int causal,
-                                  void* stream) {
-  if (!q || !k || !v || !cs || !o || !lse || !k_rot) return AXIS_ATTN_ERR_NULL;
+                                  void* q_rot, void* k_rot, int B, int Hq, int Hkv, int S, int D, float scale,
+                                  int causal, void* stream) {
+  if (!q || !k || !v || !cs || !o || !lse || !q_rot || !k_rot) return AXIS_ATTN_ERR_NULL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(cs) || !aligned16(o) || !aligned16(lse) ||
-      !aligned16(k_rot))
+      !aligned16(q_rot) || !aligned16(k_rot))
     return AXIS_ATTN_ERR_ALIGN;
   if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (int rc = run_rope(q, q_rot, cs, B, S, Hq, D, 0, st)) return rc;
   if (int rc = run_rope(k, k_rot, cs, B, S, Hkv, D, 0, st)) return rc;
-  return run_fwd(q, k_rot, v, o, lse, B, Hq, Hkv, S, D, scale, causal, cs, st, dev);
+  return run_fwd(q_rot, k_rot, v, o, lse, B, Hq, Hkv, S, D, scale, causal, st, dev);
 }
 
-extern "C" size_t axis_attn_bwd_rope_workspace_bytes(int B, int Hq, int Hkv, int S, int D, int deterministic) {
-  if (check_shape(B, Hq, Hkv, S, D, 1.f) != AXIS_ATTN_OK) return 0;
-  return ws_layout(B, Hq, S, D, deterministic != 0, true).total;
-}
-
-extern "C" int axis_attn_bwd_rope(const void* q, const void* k_rot, const void* v, const double* cs, const void* o,
-                                  const void* dO, const float* lse, void* dq, void* dk, void* dv, int B, int Hq,
-                                  int Hkv, int S, int D, float scale, int causal, int deterministic,
+extern "C" int axis_attn_bwd_rope(const void* q_rot, const void* k_rot, const void* v, const double* cs,
+                                  const void* o, const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                                  int B, int Hq, int Hkv, int S, int D, float scale, int causal, int deterministic,
                                   void* workspace, size_t workspace_bytes, void* stream) {
   if (!cs) return AXIS_ATTN_ERR_NULL;
-  return run_bwd(q, k_rot, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, workspace, workspace_bytes,
-                 stream, deterministic != 0, cs);
+  return run_bwd(q_rot, k_rot, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal, workspace,
+                 workspace_bytes, stream, deterministic != 0, cs);
 }
 
 // ----------------------------------------------------------------------------

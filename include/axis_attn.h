@@ -199,19 +199,19 @@ int axis_attn_bwd_noalloc(const void* q, const void* k, const void* v, const voi
  *   which carries gradients back), x, y [B, S, H, D] bf16 (y may be x), cs
  *   from axis_attn_rope_table for at least S positions.  HBM-bound.
  * axis_attn_fwd_rope: the forward of axis_attn_fwd() on the rotated q and k:
- *   o, lse as for softmax(scale * (R q)(R k)^T) V.  q and k are the caller's
- *   unrotated tensors.  The call rotates K once into k_rot (caller-owned,
- *   [B, S, Hkv, D] bf16; the backward reads it), and the kernel rotates each
- *   Q tile in shared memory right after its TMA load, so the rotated Q never
- *   reaches device memory.  (K tiles are re-read by every query block; turning
- *   them once up front costs less than turning them at every load.)
+ *   o, lse as for softmax(scale * (R q)(R k)^T) V, with q and k the caller's
+ *   unrotated tensors.  It writes the rotated inputs into q_rot [B, S, Hq, D]
+ *   and k_rot [B, S, Hkv, D] (bf16, caller-owned; the backward reads them):
+ *   one HBM-bound pass each, then the forward kernel.  (A rotation of each Q
+ *   tile in shared memory after its TMA load, by one warp per SM, was built
+ *   and measured: at B=4, S=2048, Hq=32, D=64 it made the forward 3.5x
+ *   slower than this pass, because every rotated pair needs a table read.)
  * axis_attn_bwd_rope: the gradients with respect to the UNROTATED q and k (and
- *   v) of that forward: it takes k_rot from the forward, rotates q once into
- *   the workspace, runs the backward of axis_attn_bwd() (deterministic != 0:
- *   that of axis_attn_bwd_det()) and applies the transposed rotation to dQ in
- *   the finalize step and to dK in the main kernel's epilogue.  Workspace:
- *   axis_attn_bwd_rope_workspace_bytes() (the plain backward's plus the
- *   rotated q).
+ *   v) of that forward, from q_rot and k_rot: the backward of axis_attn_bwd()
+ *   (deterministic != 0: of axis_attn_bwd_det()) on the rotated inputs, with
+ *   the transposed rotation applied to dQ in the finalize step (or the
+ *   deterministic dQ pass) and to dK in the main kernel's epilogue.  The
+ *   workspace is that of axis_attn_bwd() (or axis_attn_bwd_det()).
  * Arguments, layouts, requirements and errors otherwise as for axis_attn_fwd()
  * and axis_attn_bwd(); cs must be 16-byte aligned and cover S positions of D.
  */
@@ -219,10 +219,9 @@ int axis_attn_rope_table(double* cs, int S, int D, double base, void* stream);
 int axis_attn_rope(const void* x, void* y, const double* cs, int B, int S, int H, int D, int inverse,
                    void* stream);
 int axis_attn_fwd_rope(const void* q, const void* k, const void* v, const double* cs, void* o,
-                       float* lse, void* k_rot, int B, int Hq, int Hkv, int S, int D, float scale,
-                       int causal, void* stream);
-size_t axis_attn_bwd_rope_workspace_bytes(int B, int Hq, int Hkv, int S, int D, int deterministic);
-int axis_attn_bwd_rope(const void* q, const void* k_rot, const void* v, const double* cs,
+                       float* lse, void* q_rot, void* k_rot, int B, int Hq, int Hkv, int S, int D,
+                       float scale, int causal, void* stream);
+int axis_attn_bwd_rope(const void* q_rot, const void* k_rot, const void* v, const double* cs,
                        const void* o, const void* dO, const float* lse, void* dq, void* dk,
                        void* dv, int B, int Hq, int Hkv, int S, int D, float scale, int causal,
                        int deterministic, void* workspace, size_t workspace_bytes, void* stream);

@@ -194,23 +194,14 @@ def test_decode_workspace_bytes(lib):
     ("axis_attn_rope", (A, A, None, 1, 128, 2, 64, 0, None), 1),
     ("axis_attn_rope", (A, A + 4, A, 1, 128, 2, 64, 0, None), 2),
     ("axis_attn_rope", (A, A, A, 1, 128, 2, 12, 0, None), 3),
-    ("axis_attn_fwd_rope", (A, A, A, None, A, A, A, 1, 2, 1, 128, 64, 0.125, 1, None), 1),
-    ("axis_attn_fwd_rope", (A, A, A, A, A, A, A + 8, 1, 2, 1, 128, 64, 0.125, 1, None), 2),
-    ("axis_attn_fwd_rope", (A, A, A, A, A, A, A, 1, 3, 2, 128, 64, 0.125, 1, None), 3),
-    ("axis_attn_fwd_rope", (A, A, A, A, A, A, A, 1, 2, 1, 128, 96, 0.125, 1, None), 4),
+    ("axis_attn_fwd_rope", (A, A, A, None, A, A, A, A, 1, 2, 1, 128, 64, 0.125, 1, None), 1),
+    ("axis_attn_fwd_rope", (A, A, A, A, A, A, A, None, 1, 2, 1, 128, 64, 0.125, 1, None), 1),
+    ("axis_attn_fwd_rope", (A, A, A, A, A, A, A, A + 8, 1, 2, 1, 128, 64, 0.125, 1, None), 2),
+    ("axis_attn_fwd_rope", (A, A, A, A, A, A, A, A, 1, 3, 2, 128, 64, 0.125, 1, None), 3),
+    ("axis_attn_fwd_rope", (A, A, A, A, A, A, A, A, 1, 2, 1, 128, 96, 0.125, 1, None), 4),
     ("axis_attn_bwd_rope", (A,) * 3 + (None,) + (A,) * 6 + (1, 2, 1, 128, 64, 0.125, 1, 0, A, 1 << 30, None), 1),
     ("axis_attn_bwd_rope", (A,) * 3 + (A + 8,) + (A,) * 6 + (1, 2, 1, 128, 64, 0.125, 1, 0, A, 1 << 30, None), 2),
     ("axis_attn_bwd_rope", (A,) * 10 + (1, 2, 1, 128, 64, 0.125, 1, 0, A, 1000, None), 5),
 ])
 def test_rope_rejects(lib, fn, args, code):
     assert getattr(aa, fn)(*args) == code
-
-
-def test_rope_workspace_adds_the_rotated_q(lib):
-    B, Hq, Hkv, S, D = 2, 12, 4, 1000, 64
-    r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    qrot = r256(B * S * Hq * D * 2)
-    assert aa.axis_attn_bwd_rope_workspace_bytes(B, Hq, Hkv, S, D, 0) == \
-        aa.axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D) + qrot
-    assert aa.axis_attn_bwd_rope_workspace_bytes(B, Hq, Hkv, S, D, 1) == \
-        aa.axis_attn_bwd_det_workspace_bytes(B, Hq, Hkv, S, D) + qrot

@@ -98,13 +98,16 @@ def test_large_workloads_sampled(oracle_mod, name):
     go = np.stack([f64(o[b, i, h]) for b, h, i in qrows])
     gl = np.array([float(lse[b, h, i]) for b, h, i in qrows])
     gdq = np.stack([f64(dq[b, i, h]) for b, h, i in qrows])
-    # key rows in two (b, kv) units; for the longest sequence only among the
-    # last 1024 keys (their dK/dV need the oracle's statistics of fewer query rows)
+    # key rows in two (b, kv) units: the first unit over the whole key range
+    # (key 0 sums over every query row: the longest dK/dV accumulation), the
+    # second, for the longest sequence, among the last 1024 keys (their dK/dV
+    # need the oracle's statistics of fewer query rows)
     g = np.random.default_rng(11)
-    lo = w.S - 1024 if w.S > 8192 else 0
     krows = []
-    for unit in ((0, 0), (w.B - 1, w.Hkv - 1)):
+    for unit, lo in (((0, 0), 0), ((w.B - 1, w.Hkv - 1), w.S - 1024 if w.S > 8192 else 0)):
         js = [int(j) for j in g.integers(lo, w.S, 5)] + [w.S - 1, max(lo, w.S - 129)]
+        if lo == 0:
+            js += [0, 127, 128]
         krows += [(unit[0], unit[1], j) for j in js]
     rdk, rdv = oracle_mod.attn_bwd_dkdv_rows(q, k, v, do, w.scale, w.causal, krows)
     gdk = np.stack([f64(dk[b, j, kv]) for b, kv, j in krows])

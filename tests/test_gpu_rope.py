@@ -5,8 +5,8 @@ rotated q and k are the attention's inputs and are stored in bf16, so the
 test rounds the oracle's fp64 rotation to bf16 once (gpu_util.bf16_rn_from_f64)
 before the oracle's attention, and the gradients with respect to the
 unrotated inputs come back through oracle_rope(inverse=True).  The kernels
-compute the rotation in fp64 and round once as well, so the rotated K they
-write is compared bit for bit; O, LSE and the gradients use the tolerances of
+compute the rotation in fp64 and round once as well, so the rotated Q and K
+they write are compared bit for bit; O, LSE and the gradients use the tolerances of
 the other parity tests.  Shapes: the axiomlm Quick Start's own RoPE example
 (q of shape (2, 1024, 12, 64), k of shape (2, 1024, 4, 64)), a ragged length,
 head dim 128, and the non-causal mask.
@@ -81,14 +81,15 @@ def test_rope_attention_matches_oracle(oracle_mod, B, Hq, Hkv, S, D, causal, det
     dev = torch.device("cuda:0")
     cs = aa.rope_table(S, D, BASE, device=dev)
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
-    o, lse, k_rot = aa.attention_forward_rope(qd, kd, vd, cs, causal=causal, scale=sc)
-    dq, dk, dv = aa.attention_backward_rope(qd, k_rot, vd, cs, o, lse, dod, causal=causal, scale=sc,
+    o, lse, q_rot, k_rot = aa.attention_forward_rope(qd, kd, vd, cs, causal=causal, scale=sc)
+    dq, dk, dv = aa.attention_backward_rope(q_rot, k_rot, vd, cs, o, lse, dod, causal=causal, scale=sc,
                                             deterministic=det)
     aa.check_status()
     # oracle: rotate in fp64, store in bf16, attend, gradients back through R^T
     qr = bf16_rn_from_f64(oracle_mod.rope(q, BASE))
     kr = bf16_rn_from_f64(oracle_mod.rope(k, BASE))
     assert torch.equal(k_rot.cpu().view(torch.int16), kr.view(torch.int16))
+    assert torch.equal(q_rot.cpu().view(torch.int16), qr.view(torch.int16))
     ro, rl = oracle_mod.attn_fwd(qr, kr, v, sc, causal)
     rdq_r, rdk_r, rdv, _ = oracle_mod.attn_bwd(qr, kr, v, do, sc, causal)
     rdq = oracle_mod.rope(rdq_r, BASE, inverse=True)
