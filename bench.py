@@ -494,6 +494,80 @@ def time_decode(aa, name, dev, steps, flush, hbm_gbs):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs}}
 
 
+def time_e2e(aa, w, prob, steps: int, det: bool, world: int, dev) -> dict:
+    """The step end to end through the public torch helpers, from pinned host
+    buffers: every step copies its Q, K, V, dO host->device and its O, LSE,
+    dQ, dK, dV device->host inside the timed region.  Three streams form a
+    pipeline, as a training loop would run it: step i's inputs go up on the
+    copy-in stream while step i-1 computes and step i-2's results come down on
+    the copy-out stream (PCIe is full duplex).  Two device buffer sets
+    alternate; events order each set's reuse.  Time: from an event before the
+    first upload to one after the last download."""
+    import torch
+
+    pin = lambda t: t.pin_memory()  # noqa: E731
+    q_h, k_h, v_h, do_h = prob.host
+    hin = [pin(t) for t in (q_h, k_h, v_h, do_h)]
+    hout = [torch.empty_like(hin[0]).pin_memory(),
+            torch.empty((w.B, w.Hq, w.S), dtype=torch.float32).pin_memory()] + \
+        [torch.empty_like(t).pin_memory() for t in hin[:3]]
+    sets = []
+    for _ in range(2):
+        ins = [torch.empty_like(t) for t in (prob.q, prob.k, prob.v, prob.do)]
+        outs = [torch.empty_like(prob.q), torch.empty_like(prob.lse), torch.empty_like(prob.q),
+                torch.empty_like(prob.k), torch.empty_like(prob.v)]
+        sets.append((ins, outs))
+    s_in, s_out, s_comp = torch.cuda.Stream(dev), torch.cuda.Stream(dev), prob.stream
+    mk = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+    ev_in, ev_done, ev_out = mk(), mk(), mk()
+    used = [False, False]
+
+    def step(i):
+        b = i % 2
+        ins, outs = sets[b]
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(ev_done[b])  # the last compute on this set has read its inputs
+            for dst, src in zip(ins, hin):
+                dst.copy_(src, non_blocking=True)
+            ev_in[b].record(s_in)
+        s_comp.wait_event(ev_in[b])
+        if used[b]:
+            s_comp.wait_event(ev_out[b])  # its previous results are on the host
+        o, lse = aa.attention_forward(ins[0], ins[1], ins[2], causal=w.causal, scale=w.scale, out=outs[0],
+                                      lse=outs[1], stream=s_comp)
+        aa.attention_backward(ins[0], ins[1], ins[2], o, lse, ins[3], causal=w.causal, scale=w.scale,
+                              workspace=prob.ws, grads=tuple(outs[2:]), stream=s_comp, deterministic=det)
+        ev_done[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[b])
+            for dst, src in zip(hout, outs):
+                dst.copy_(src, non_blocking=True)
+            ev_out[b].record(s_out)
+        used[b] = True
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    e0.record(s_in)
+    for i in range(steps):
+        step(i)
+    e1.record(s_out)
+    torch.cuda.synchronize()
+    ems = reduce_max([e0.elapsed_time(e1)], world, dev)
+    aa.check_status(s_comp)
+    h2d = sum(t.numel() * t.element_size() for t in hin)
+    d2h = sum(t.numel() * t.element_size() for t in hout)
+    return {"value": whole_job_tflops(w.fwd_flops + w.bwd_flops, steps, ems[0], world), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "streams": "copy-in / compute / copy-out, two buffer sets"}
+
+
 def summarize(w, total_ms, stage_totals, steps, world, p_meas, det):
     """Per-workload figures: fwd / bwd TFLOP/s and fractions of the peaks."""
     avg = [float(t) / steps for t in stage_totals]
@@ -588,41 +662,7 @@ def main():
     # ---- end to end through the public API, host buffers, copies inside the timed region
     e2e = None
     if args.e2e_steps > 0 and not sharded:
-        pin = lambda t: t.pin_memory()  # noqa: E731
-        q_h, k_h, v_h, do_h = prob.host
-        hq, hk, hv, hdo = pin(q_h), pin(k_h), pin(v_h), pin(do_h)
-        ho, hl = torch.empty_like(hq).pin_memory(), torch.empty((w.B, w.Hq, w.S), dtype=torch.float32).pin_memory()
-        hdq, hdk, hdv = (torch.empty_like(t).pin_memory() for t in (hq, hk, hv))
-        qq, kk, vv, dd = (torch.empty_like(t) for t in (prob.q, prob.k, prob.v, prob.do))
-        stream = prob.stream
-
-        def e2e_step():
-            for dst, src in ((qq, hq), (kk, hk), (vv, hv), (dd, hdo)):
-                dst.copy_(src, non_blocking=True)
-            oo, ll = aa.attention_forward(qq, kk, vv, causal=w.causal, scale=w.scale, out=prob.o, lse=prob.lse)
-            g = aa.attention_backward(qq, kk, vv, oo, ll, dd, causal=w.causal, scale=w.scale, workspace=prob.ws,
-                                      grads=(prob.dq, prob.dk, prob.dv), deterministic=det)
-            for dst, src in ((ho, oo), (hl, ll), (hdq, g[0]), (hdk, g[1]), (hdv, g[2])):
-                dst.copy_(src, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ems = reduce_max([e0.elapsed_time(e1)], world, dev)
-        aa.check_status(stream)
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-        d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
-        e2e = {"value": whole_job_tflops(w.fwd_flops + w.bwd_flops, args.e2e_steps, ems[0], world),
-               "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "steps": args.e2e_steps}
+        e2e = time_e2e(aa, w, prob, args.e2e_steps, det, world, dev)
     clocks = sampler.summary(*win)
     del prob
     torch.cuda.empty_cache()

@@ -149,6 +149,12 @@ __device__ __forceinline__ float row_max32(const uint32_t (&v)[32]) {
 #ifndef AXIS_ATTN_FWD_NOXCH
 #define AXIS_ATTN_FWD_NOXCH 0
 #endif
+// Speculative softmax order (exponentials with the running max before the
+// partial-max exchange completes): bit 0 at head dim 64, bit 1 at head dim
+// 128.
+#ifndef AXIS_ATTN_FWD_PIPE
+#define AXIS_ATTN_FWD_PIPE 0
+#endif
 
 // Scores v[2 I0 .. 2 (I0 + N)) -> probabilities 2^(s*c - m): packed FMA for
 // the argument, MUFU ex2 (or the polynomial, for the pairs the mask selects)
@@ -629,6 +635,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     }
   } else if (!FWD_ROWTHREAD && warp < FWD_SOFTMAX_WARPS) {
     // ===================================================== softmax (tile t, half hf)
+    constexpr bool PIPE = (AXIS_ATTN_FWD_PIPE & (HD == 64 ? 1 : 2)) != 0 && !AXIS_ATTN_FWD_NOXCH &&
+                          !AXIS_ATTN_FWD_TOKEN;
     const int t = warp >> 3, hf = (warp >> 2) & 1, wq = warp & 3;
     const int r = wq * 32 + lane;                   // row in tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
@@ -652,6 +660,108 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       const int qt = 2 * I.m + t;
       const int row_g = qt * 128 + r;
       float m_used = -INFINITY, l = 0.f;
+      if constexpr (PIPE) {
+        // Speculative order: from the second kv tile on, the exponentials
+        // start with the running max before the other half's partial max is
+        // in (the exchange round trip overlaps them).  The running max moves
+        // only when the row max grows by more than 8; when the other half's
+        // max moves it (rare), this half's packed P and partial row sum are
+        // scaled by alpha = 2^(m_old - m_new) in registers, the correction
+        // the online softmax applies to O.
+        for (int j = 0; j < n_t; ++j, ++J, ++X) {
+          if (!wait_warp<true>(bar_sfull(t), J & 1, abort, F_SFULL)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tS, v0);
+          tmem_ld32(tS + 32, v1);
+          tmem_wait_ld();
+          // S is in registers: its columns may take the next S
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_sfree(C::SHARED_S ? 0 : t));
+          const bool masked = CAUSAL ? (j == qt) : (j == nkv - 1 && (a.S & 127) != 0);
+          if (masked) {
+            int limit = a.S - 128 * j;
+            if (CAUSAL && r + 1 < limit) limit = r + 1;
+            limit -= hf * 64;  // in this half's columns
+            mask_row(v0, 0, limit);
+            mask_row(v1, 32, limit);
+          }
+          const float mx = fmaxf(row_max32(v0), row_max32(v1));
+          *xslot(X & 1, hf) = mx;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bx);
+          // speculate with the running max when no lane's own half moves it
+          const bool spec = j > 0 && __all_sync(0xffffffffu, !(fmaxf(m_used, mx * c) > m_used + 8.0f));
+          uint64_t acc = f2_pack(0.f, 0.f);
+          uint32_t pk0[16], pk1[16];
+          float alpha = 1.f;
+          bool resc = false;
+          // the other half's partial max, the row max, and the running max update
+#define AXIS_ATTN_FWD_ROW_MAX()                                                    \
+  if (!wait_warp<true>(bx, X & 1, abort, F_XCH)) {                                 \
+    ok = false;                                                                    \
+    break;                                                                         \
+  }                                                                                \
+  {                                                                                \
+    const float m_new = fmaxf(m_used, fmaxf(mx, *xslot(X & 1, hf ^ 1)) * c);       \
+    resc = m_new > m_used + 8.0f;                                                  \
+    if (resc) {                                                                    \
+      alpha = ex2_approx(m_used - m_new);                                          \
+      m_used = m_new;                                                              \
+    }                                                                              \
+  }
+          if (spec) {
+            {
+              const uint64_t nm2 = f2_pack(-m_used, -m_used);
+              acc = exp_pairs<0, 16>(v0, cc2, nm2, acc, pk0);
+              acc = exp_pairs<0, 16>(v1, cc2, nm2, acc, pk1);
+            }
+            AXIS_ATTN_FWD_ROW_MAX()
+            if (__any_sync(0xffffffffu, resc)) {  // rare: rescale this half's P and row sum
+              const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                pk0[i] = pack_bf16x2(f2_mul(f2_pack(__uint_as_float(pk0[i] << 16), __uint_as_float(pk0[i] & 0xffff0000u)), a2));
+                pk1[i] = pack_bf16x2(f2_mul(f2_pack(__uint_as_float(pk1[i] << 16), __uint_as_float(pk1[i] & 0xffff0000u)), a2));
+              }
+              acc = f2_mul(acc, a2);
+            }
+          } else {
+            AXIS_ATTN_FWD_ROW_MAX()
+            const uint64_t nm2 = f2_pack(-m_used, -m_used);
+            acc = exp_pairs<0, 16>(v0, cc2, nm2, acc, pk0);
+            acc = exp_pairs<0, 16>(v1, cc2, nm2, acc, pk1);
+          }
+#undef AXIS_ATTN_FWD_ROW_MAX
+          const bool any_resc = __any_sync(0xffffffffu, resc);
+          float rs_lo, rs_hi;
+          f2_unpack(acc, rs_lo, rs_hi);
+          l = l * alpha + (rs_lo + rs_hi);
+          // the previous P V must have landed before P_t is overwritten and O_t rescaled
+          if (J > 0) {
+            if (!wait_warp<true>(bar_o(t), (J - 1) & 1, abort, F_OWAIT)) { ok = false; break; }
+            tc_fence_after();
+          }
+          tmem_st16(tP, pk0);
+          tmem_st16(tP + 16, pk1);
+          if (j > 0 && any_resc) {
+#pragma unroll 1
+            for (int cc = 0; cc < HD / 64; ++cc) {
+              uint32_t v[32];
+              tmem_ld32(tO + cc * 32, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+              tmem_st32(tO + cc * 32, v);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0 && !(AXIS_ATTN_TEST_DROP_ARRIVE == 1 && J == 0 && t == 0)) mbar_arrive(bar_pfull(t));
+        }
+      } else
       for (int j = 0; j < n_t; ++j, ++J, X += !AXIS_ATTN_FWD_NOXCH) {
         if (!wait_warp<true>(bar_sfull(t), J & 1, abort, F_SFULL)) { ok = false; break; }
         tc_fence_after();

@@ -154,3 +154,32 @@ def test_short_sequences_over_seeds(oracle_mod, S):
             rdq, rdk, rdv, _ = oracle_mod.attn_bwd(q, k, v, do, sc, causal)
             assert_close(*got, ro, rl, rdq, rdk, rdv, tag=f"S{S} seed{seed} Hq{Hq} Hkv{Hkv} D{D} c{int(causal)}",
                          S=S)
+
+
+@pytest.mark.parametrize("D,causal", [(64, True), (64, False), (128, True)])
+def test_rising_scores_move_the_running_max(oracle_mod, D, causal):
+    """Scores that rise along the keys by about 6 (log2 units) per 64 keys:
+    from the second kv tile on, the running max of a row moves in almost
+    every tile, mostly because of the second half of the tile's columns.
+    That drives the forward's rare paths: the O rescale, and the rescale of
+    P and the partial row sum when the exponentials started with the old
+    max.  Parity with the oracle as everywhere else."""
+    B, Hq, Hkv, S = 1, 4, 2, 1000
+    q, k, v, do = make_inputs(B, Hq, Hkv, S, D, 8100 + D + int(causal))
+    sc = 1.0 / math.sqrt(D)
+    # score_ij ~ scale * A * delta * j = 0.065 j natural-log units, ~12 in
+    # log2 units per 128 keys (the rest of q, k stays random, smaller).  The
+    # ramp's size sits in q (A = 512), not in k: a large k component would
+    # make dQ = scale sum_j dS_ij K_j a cancellation (the dS_ij of a row sum
+    # to zero) that amplifies the bf16 rounding of dS far beyond any bound.
+    A = 512.0
+    delta = 0.065 / (sc * A)
+    q = q.float() * 0.3
+    q[..., 0] = A
+    k = k.float() * 0.3
+    k[..., 0] = delta * torch.arange(S, dtype=torch.float32)[None, :, None]
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    got = run_gpu(q, k, v, do, causal, sc)
+    ro, rl = oracle_mod.attn_fwd(q, k, v, sc, causal)
+    rdq, rdk, rdv, _ = oracle_mod.attn_bwd(q, k, v, do, sc, causal)
+    print(assert_close(*got, ro, rl, rdq, rdk, rdv, tag=f"rising D{D} c{int(causal)}", S=S))
