@@ -39,9 +39,9 @@ METRIC = "attention fwd / bwd TFLOP/s (bf16, causal) and % of B200 tensor peak"
 # helpers, and the host file with its launch configuration).
 KERNEL_SOURCES = {
     "attn_fwd_kernel": ("attn_fwd.cuh", "sm100_ptx.cuh", "axis_attn.cu"),
-    "attn_bwd_kernel": ("attn_bwd.cuh", "sm100_ptx.cuh", "axis_attn.cu"),
+    "attn_bwd_kernel": ("attn_bwd.cuh", "attn_rope.cuh", "sm100_ptx.cuh", "axis_attn.cu"),
     "attn_bwd_prep_kernel": ("attn_bwd.cuh", "axis_attn.cu"),
-    "attn_bwd_dq_convert_kernel": ("attn_bwd.cuh", "axis_attn.cu"),
+    "attn_bwd_dq_convert_kernel": ("attn_bwd.cuh", "attn_rope.cuh", "axis_attn.cu"),
 }
 
 

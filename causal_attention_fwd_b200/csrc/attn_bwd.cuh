@@ -143,8 +143,11 @@ __device__ __forceinline__ void store_row16(uint32_t buf, int kr, int col0, cons
 // key tile.  CTAs resident at the same time then share the Q and dO tiles and
 // the dQ accumulator rows of only about UG units, which stay in L2; UG = 0
 // puts all units in one group (key-tile-major order over the whole grid).
+// Measured: UG = 8 is 1% (llm1b) to 3% (llm8b_gqa) faster than UG = 0, UG = 4
+// 16% slower at llm1b (a group of 4 units at 16 key tiles is less than one
+// wave of CTAs, so the light key tiles of one group wait behind the next).
 #ifndef AXIS_ATTN_BWD_UNIT_GROUP
-#define AXIS_ATTN_BWD_UNIT_GROUP 0
+#define AXIS_ATTN_BWD_UNIT_GROUP 8
 #endif
 __device__ __forceinline__ void bwd_item(int BKV, int nkv, int x, int& j, int& bkv) {
   const int UG = AXIS_ATTN_BWD_UNIT_GROUP > 0 && AXIS_ATTN_BWD_UNIT_GROUP < BKV ? AXIS_ATTN_BWD_UNIT_GROUP : BKV;

@@ -13,10 +13,11 @@
 // about 4 G flops per byte, far below the tensor cores' ridge, so it is
 // HBM-bound: the kernel is built to keep the memory system busy, not the MMA
 // units.
-//   * one CTA per (b, kv head, split of the sequence); a producer thread
-//     streams 32-key pieces of the cache pages through TMA (a 3-D tensor map
-//     over the cache, 128B swizzle) into a ring of shared-memory stages, K and V
-//     of a piece on one mbarrier;
+//   * one CTA per (b, kv head, split of the sequence); a producer warp reads
+//     the block table 32 pieces ahead into shared memory and one of its
+//     threads streams 32-key pieces of the cache pages through TMA (a 3-D
+//     tensor map over the cache, 128B swizzle) into a ring of shared-memory
+//     stages, K and V of a piece on one mbarrier;
 //   * four compute warps take the pieces in turn (piece t -> warp t % 4) and
 //     keep their own running max, sum and O for the G query heads: scores with
 //     lane = key (q broadcast from shared memory, packed fp32 FMA), per-head
@@ -64,7 +65,8 @@ struct DecCfg {
   static constexpr uint32_t OFF_P = OFF_Q + 8 * HD * 4;           // fp32 [DEC_CW][32][8]
   static constexpr uint32_t OFF_C = OFF_P + DEC_CW * 32 * 8 * 4;  // fp32 [DEC_CW][8][HD + 2]
   static constexpr uint32_t OFF_FLAG = OFF_C + DEC_CW * 8 * (HD + 2) * 4;  // int [NST]: piece usable
-  static constexpr uint32_t OFF_BAR = (OFF_FLAG + NST * 4 + 7) & ~7u;
+  static constexpr uint32_t OFF_TBL = OFF_FLAG + NST * 4;                  // int [32][4]: pages of 32 pieces
+  static constexpr uint32_t OFF_BAR = (OFF_TBL + 32 * 4 * 4 + 7) & ~7u;
   static constexpr uint32_t SMEM = OFF_BAR + 8 * 2 * NST + 16 + 1024;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -126,53 +128,77 @@ __global__ void __launch_bounds__(DEC_THREADS)
 
   if (warp == 0) {
     // ============================================================ producer
-    if (lane == 0 && n_pieces > 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
+    // The whole warp reads the block-table entries of 32 pieces at a time
+    // into shared memory (32 independent loads instead of one dependent
+    // global read per page in front of every copy); lane 0 then checks them
+    // and issues the copies.
+    if (n_pieces > 0) {
+      int* tbl = reinterpret_cast<int*>(gbase + C::OFF_TBL);
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+      }
       const int rows = a.page_size < 32 ? a.page_size : 32;  // rows per TMA box
       const int nbox = 32 / rows;                              // boxes per 32-key piece
       int issued = 0;
-      for (int t = 0; t < n_pieces; ++t) {
-        const int s = t % NST;
-        if (t >= NST && !mbar_wait_bounded<true>(bar_empty(s), ((t / NST) & 1) ^ 1, ctl, D_EMPTY)) break;
-        const int kt = k0 + 32 * t;
-        // pages of this piece (at most 4: page_size >= 8), each read once and
-        // checked before any copy
-        int usable = 1, nload = 0, pages[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int key = kt + x * rows;
-          if (x < nbox && key < k1) {
-            pages[x] = a.block_table[(size_t)b * a.max_pages + key / a.page_size];
-            if (pages[x] < 0 || pages[x] >= a.num_pages) usable = 0;
-            ++nload;
-          }
+      bool ok = true;
+      for (int t0 = 0; ok && t0 < n_pieces; t0 += 32) {
+        for (int e = lane; e < 32 * nbox; e += 32) {  // e = (t - t0) * nbox + x
+          const int t = t0 + e / nbox, key = k0 + 32 * t + (e % nbox) * rows;
+          tbl[e] = t < n_pieces && key < k1 ? a.block_table[(size_t)b * a.max_pages + key / a.page_size] : 0;
         }
-        flag[s] = usable;
-        if (!usable) {
-          atomicOr(&g_status, 2u);
-          mbar_arrive(bar_full(s));
-        } else {
-          mbar_arrive_expect_tx(bar_full(s), (uint32_t)(nload * rows * HD * 2 * 2));
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            if (x >= nload) break;
-            const int key = kt + x * rows;
-            const int row = pages[x] * a.page_size + key % a.page_size;
-#pragma unroll
-            for (int sl = 0; sl < C::NSLAB; ++sl) {
-              const uint32_t off = s * C::PIECE + sl * C::SLAB + x * rows * 128;
-              tma_load_3d(sK + off, &tm_k, bar_full(s), 64 * sl, kv, row);
-              tma_load_3d(sV + off, &tm_v, bar_full(s), 64 * sl, kv, row);
+        __syncwarp();
+        if (lane == 0) {
+          const int t1 = min(n_pieces, t0 + 32);
+          for (int t = t0; t < t1; ++t) {
+            const int s = t % NST;
+            if (t >= NST && !mbar_wait_bounded<true>(bar_empty(s), ((t / NST) & 1) ^ 1, ctl, D_EMPTY)) {
+              ok = false;
+              break;
             }
+            const int kt = k0 + 32 * t;
+            // pages of this piece (at most 4: page_size >= 8), checked before any copy
+            int usable = 1, nload = 0, pages[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const int key = kt + x * rows;
+              if (x < nbox && key < k1) {
+                pages[x] = tbl[(t - t0) * nbox + x];
+                if (pages[x] < 0 || pages[x] >= a.num_pages) usable = 0;
+                ++nload;
+              }
+            }
+            flag[s] = usable;
+            if (!usable) {
+              atomicOr(&g_status, 2u);
+              mbar_arrive(bar_full(s));
+            } else {
+              mbar_arrive_expect_tx(bar_full(s), (uint32_t)(nload * rows * HD * 2 * 2));
+#pragma unroll
+              for (int x = 0; x < 4; ++x) {
+                if (x >= nload) break;
+                const int key = kt + x * rows;
+                const int row = pages[x] * a.page_size + key % a.page_size;
+#pragma unroll
+                for (int sl = 0; sl < C::NSLAB; ++sl) {
+                  const uint32_t off = s * C::PIECE + sl * C::SLAB + x * rows * 128;
+                  tma_load_3d(sK + off, &tm_k, bar_full(s), 64 * sl, kv, row);
+                  tma_load_3d(sV + off, &tm_v, bar_full(s), 64 * sl, kv, row);
+                }
+              }
+            }
+            issued = t + 1;
           }
         }
-        issued = t + 1;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        __syncwarp();  // lane 0 is done with this block of table entries
       }
       // drain: every copy started has landed before the CTA exits
-      volatile WaitCtl never = {0, 0, 0};
-      for (int t = issued - NST > 0 ? issued - NST : 0; t < issued; ++t)
-        mbar_wait_bounded<true>(bar_full(t % NST), (t / NST) & 1, &never, D_FULL);
+      if (lane == 0) {
+        volatile WaitCtl never = {0, 0, 0};
+        for (int t = issued - NST > 0 ? issued - NST : 0; t < issued; ++t)
+          mbar_wait_bounded<true>(bar_full(t % NST), (t / NST) & 1, &never, D_FULL);
+      }
     }
   } else {
     // ============================================================ compute warps

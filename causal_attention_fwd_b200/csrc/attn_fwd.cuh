@@ -25,9 +25,12 @@
 //     while it issues the FMA-pipe work).  The running max is only moved when
 //     it grows by more than 8 (a factor 256), so the O rescale in TMEM is rare;
 //     stale-max values stay below 2^8 and are exact to bf16 relative precision;
-//   * the two query tiles take turns on the exponentials (a token passed at
-//     three quarters of each phase), so one tile's exponentials overlap the
-//     other tile's TMEM traffic, row max and MMAs;
+//   * the two query tiles run their softmax phases independently, so one
+//     tile's exponentials overlap the other tile's TMEM traffic, row max and
+//     MMAs (forcing them to alternate with a token barrier, reading the other
+//     half's scores from TMEM instead of exchanging partial maxima, one
+//     thread per whole row, and starting the exponentials before the
+//     exchange completes all measured slower);
 //   * causal: kv tiles after a query tile's diagonal are never loaded or
 //     multiplied; the element mask runs only on the diagonal (and ragged last)
 //     tile;
@@ -102,7 +105,7 @@ struct FwdCfg {
   static constexpr bool SHARED_S = HD == 128;
   static constexpr uint32_t T_P = SHARED_S ? 128 : 384, T_O = 256;
   static __host__ __device__ constexpr uint32_t t_s(int t) { return SHARED_S ? 0u : 128u * t; }
-  static constexpr int NBAR = 23 + 2 * KST + 2 * VST;
+  static constexpr int NBAR = 21 + 2 * KST + 2 * VST;
   static constexpr uint32_t XCH_OFF = (2 + KST + VST) * TILE;  // row-max / row-sum exchange
   static constexpr uint32_t XCH_BYTES = 2 * 2 * 2 * 128 * 4;   // [parity][tile][half][row] fp32
   static constexpr uint32_t BAR_OFF = XCH_OFF + XCH_BYTES;
@@ -111,7 +114,7 @@ struct FwdCfg {
 };
 
 enum FwdSite { F_Q = 1, F_EMPTY, F_KFULL, F_VFULL, F_PFULL, F_OBAR, F_SFULL, F_OWAIT, F_OFIN, F_XCH, F_QEMPTY,
-               F_OFREE, F_TOK };
+               F_OFREE };
 
 // -inf for the columns at or after `limit` (causal diagonal / ragged tail).
 __device__ __forceinline__ void mask_row(uint32_t (&v)[32], int col0, int limit) {
@@ -138,24 +141,6 @@ __device__ __forceinline__ float row_max32(const uint32_t (&v)[32]) {
 #ifndef AXIS_ATTN_FWD_POLY_MASK
 #define AXIS_ATTN_FWD_POLY_MASK 0x0000
 #endif
-// 1: the two query tiles take turns on the exponentials (a token barrier);
-// 0: both run them whenever their scores are ready.
-#ifndef AXIS_ATTN_FWD_TOKEN
-#define AXIS_ATTN_FWD_TOKEN 0
-#endif
-// 1: each half-row thread reads the other half's 64 scores from TMEM for the
-// row max (a second TMEM pass) instead of swapping partial maxima with its
-// partner warp through shared memory (a barrier round trip per kv tile).
-#ifndef AXIS_ATTN_FWD_NOXCH
-#define AXIS_ATTN_FWD_NOXCH 0
-#endif
-// Speculative softmax order (exponentials with the running max before the
-// partial-max exchange completes): bit 0 at head dim 64, bit 1 at head dim
-// 128.
-#ifndef AXIS_ATTN_FWD_PIPE
-#define AXIS_ATTN_FWD_PIPE 0
-#endif
-
 // Scores v[2 I0 .. 2 (I0 + N)) -> probabilities 2^(s*c - m): packed FMA for
 // the argument, MUFU ex2 (or the polynomial, for the pairs the mask selects)
 // for the exponential, packed add into the running row sum, and the bf16
@@ -211,15 +196,7 @@ __device__ __forceinline__ void xpose_chunks(uint32_t (&c)[4 * N], int lane) {
 // owner), 18 TMA producer of V, 19 P V issuer.  Five warps per SM
 // sub-partition leave 96 registers a thread: half a row of scores (64) plus
 // its packed probabilities.
-// Softmax layout: 0 = two warps per 32-row group, each a half row (64
-// columns; partial maxima and sums meet through shared memory), 20 warps,
-// 96 registers; 1 = one thread per whole 128-column row (max and sum stay in
-// the thread), 8 softmax warps + 4 role warps, up to 168 registers.
-#ifndef AXIS_ATTN_FWD_ROWTHREAD
-#define AXIS_ATTN_FWD_ROWTHREAD 0
-#endif
-constexpr bool FWD_ROWTHREAD = AXIS_ATTN_FWD_ROWTHREAD != 0;
-constexpr int FWD_SOFTMAX_WARPS = FWD_ROWTHREAD ? 8 : 16;
+constexpr int FWD_SOFTMAX_WARPS = 16;
 constexpr int FWD_SMW_PER_TILE = FWD_SOFTMAX_WARPS / 2;  // softmax warps of one query tile
 constexpr int FWD_THREADS = (FWD_SOFTMAX_WARPS + 4) * 32;
 constexpr int FWD_WARP_LOAD = FWD_SOFTMAX_WARPS;
@@ -253,13 +230,11 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   auto bar_o = [&](int t) { return bars + 8u * (B2 + 4 + t); };
   const uint32_t bar_fin = bars + 8u * (B2 + 6);
   auto bar_sfree = [&](int t) { return bars + 8u * (B2 + 7 + t); };
-  // exponential-phase token of tile t: arrived by the other tile's warps
-  auto bar_tok = [&](int t) { return bars + 8u * (B2 + 9 + t); };
   // partial-max / row-sum exchange between the two halves of a row block
   // (tile t, lane quarter wq): one phase per kv tile and one per epilogue
-  auto bar_xch = [&](int t, int wq) { return bars + 8u * (B2 + 11 + 4 * t + wq); };
+  auto bar_xch = [&](int t, int wq) { return bars + 8u * (B2 + 9 + 4 * t + wq); };
   // O_t has been read out by the epilogue: the next item may overwrite it
-  auto bar_ofree = [&](int t) { return bars + 8u * (B2 + 19 + t); };
+  auto bar_ofree = [&](int t) { return bars + 8u * (B2 + 17 + t); };
   float* xch = reinterpret_cast<float*>(gbase + C::XCH_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::BAR_OFF + 8 * C::NBAR);
   volatile WaitCtl* abort = reinterpret_cast<volatile WaitCtl*>(gbase + C::BAR_OFF + 8 * C::NBAR + 4);
@@ -283,7 +258,6 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       mbar_init(bar_pfull(t), FWD_SMW_PER_TILE);
       mbar_init(bar_o(t), 1);
       mbar_init(bar_sfree(t), FWD_SMW_PER_TILE);
-      mbar_init(bar_tok(t), FWD_SMW_PER_TILE);
       mbar_init(bar_ofree(t), FWD_SMW_PER_TILE);
       for (int wq = 0; wq < 4; ++wq) mbar_init(bar_xch(t, wq), 2);
     }
@@ -473,170 +447,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     mma_commit_w(bar_fin);
     volatile WaitCtl never = {0, 0, 0};  // drain: bounded by the time limit only
     wait_warp<true>(bar_fin, 0, &never, F_OFIN);
-  } else if (FWD_ROWTHREAD && warp < FWD_SOFTMAX_WARPS) {
-    // ===================================================== softmax (tile t, thread = whole row)
-    const int t = warp >> 2, wq = warp & 3;
-    const int r = wq * 32 + lane;                   // row in tile == TMEM lane
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::t_s(t);
-    const uint32_t tO = tmem + lane_off + C::T_O + t * HD;
-    const uint32_t tP = tmem + lane_off + C::T_P + t * 64;
-    const float c = a.scale_log2;
-    const uint64_t cc2 = f2_pack(c, c);
-    int J = 0, A_o = 0;  // kv tiles of this tile so far; exponential phases of the other tile in earlier items
-    bool ok = true;
-    for (int it = 0; ok; ++it) {
-      const int w = fwd_item(it);
-      if (w >= a.n_items) break;
-      const FwdItem I = fwd_decode(a, w, CAUSAL);
-      const int n_t = t == 0 ? I.n0 : I.n1, n_o = t == 0 ? I.n1 : I.n0;
-      const int qt = 2 * I.m + t;
-      const int row_g = qt * 128 + r;
-      float m_used = -INFINITY, l = 0.f;
-      for (int j = 0; j < n_t; ++j, ++J) {
-        if (!wait_warp<true>(bar_sfull(t), J & 1, abort, F_SFULL)) { ok = false; break; }
-        tc_fence_after();
-        const bool masked = CAUSAL ? (j == qt) : (j == nkv - 1 && (a.S & 127) != 0);
-        int limit = 128;
-        if (masked) {
-          limit = a.S - 128 * j;
-          if (CAUSAL && r + 1 < limit) limit = r + 1;
-        }
-        // the 128-column row of S: option 1 keeps it all in registers (one TMEM
-        // pass); option 2 keeps columns 64-127 and reads columns 0-63 twice
-        // (for the row max, then for the exponentials), 64 fewer registers
-        constexpr bool TWO_PASS = AXIS_ATTN_FWD_ROWTHREAD == 2;
-        uint32_t v[4][32];
-        float mx;
-        if (TWO_PASS) {
-          tmem_ld32(tS, v[0]);
-          tmem_ld32(tS + 32, v[1]);
-          tmem_wait_ld();
-          if (masked) {
-            mask_row(v[0], 0, limit);
-            mask_row(v[1], 32, limit);
-          }
-          mx = fmaxf(row_max32(v[0]), row_max32(v[1]));
-          tmem_ld32(tS + 64, v[2]);
-          tmem_ld32(tS + 96, v[3]);
-          tmem_wait_ld();
-          if (masked) {
-            mask_row(v[2], 64, limit);
-            mask_row(v[3], 96, limit);
-          }
-          mx = fmaxf(mx, fmaxf(row_max32(v[2]), row_max32(v[3])));
-        } else {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) tmem_ld32(tS + 32 * k, v[k]);
-          tmem_wait_ld();
-          // S is in registers: its columns may take the next S
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_sfree(C::SHARED_S ? 0 : t));
-          if (masked) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) mask_row(v[k], 32 * k, limit);
-          }
-          mx = fmaxf(fmaxf(row_max32(v[0]), row_max32(v[1])), fmaxf(row_max32(v[2]), row_max32(v[3])));
-        }
-        const float m_new = fmaxf(m_used, mx * c);
-        const bool resc = m_new > m_used + 8.0f;
-        float alpha = 1.f;
-        if (resc) {
-          alpha = ex2_approx(m_used - m_new);
-          m_used = m_new;
-        }
-        if (AXIS_ATTN_FWD_TOKEN) {
-          const int need = A_o + (t == 0 ? min(j, n_o) : min(j + 1, n_o));
-          if (need > 0 && !wait_warp<true>(bar_tok(t), (need - 1) & 1, abort, F_TOK)) { ok = false; break; }
-        }
-        // the previous P V must have landed before P_t is overwritten and O_t
-        // rescaled (it was issued a whole kv tile ago): then each 32-column
-        // chunk of P goes to TMEM as soon as it is packed
-        if (J > 0) {
-          if (!wait_warp<true>(bar_o(t), (J - 1) & 1, abort, F_OWAIT)) { ok = false; break; }
-          tc_fence_after();
-        }
-        const uint64_t nm2 = f2_pack(-m_used, -m_used);
-        uint64_t acc = f2_pack(0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (TWO_PASS && k < 2) {  // second read of columns 0-63; then S may take the next product
-            tmem_ld32(tS + 32 * k, v[k]);
-            tmem_wait_ld();
-            if (masked) mask_row(v[k], 32 * k, limit);
-            if (k == 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(bar_sfree(C::SHARED_S ? 0 : t));
-            }
-          }
-          uint32_t pk[16];
-          acc = exp_pairs<0, 16>(v[k], cc2, nm2, acc, pk);
-          tmem_st16(tP + 16 * k, pk);
-          if (AXIS_ATTN_FWD_TOKEN && k == 2) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tok(1 - t));
-          }
-        }
-        float rs_lo, rs_hi;
-        f2_unpack(acc, rs_lo, rs_hi);
-        l = l * alpha + (rs_lo + rs_hi);
-        if (j > 0 && __any_sync(0xffffffffu, resc)) {
-#pragma unroll 1
-          for (int cc = 0; cc < HD / 32; ++cc) {
-            uint32_t o32[32];
-            tmem_ld32(tO + cc * 32, o32);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
-            tmem_st32(tO + cc * 32, o32);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0 && !(AXIS_ATTN_TEST_DROP_ARRIVE == 1 && J == 0 && t == 0)) mbar_arrive(bar_pfull(t));
-      }
-      A_o += n_o;
-      if (!ok || n_t == 0) continue;
-      // epilogue: O / l -> bf16, LSE = (m + log2 l) ln 2, all in this thread's row
-      if (!wait_warp<true>(bar_o(t), (J - 1) & 1, abort, F_OFIN)) { ok = false; break; }
-      tc_fence_after();
-      const float inv_l = __fdividef(1.f, l);  // l >= 1: the row max contributes 2^(>= 0)
-      constexpr int NCK = HD / 8;  // 16-byte chunks of the row
-      uint32_t pk[4 * NCK];
-#pragma unroll
-      for (int cc = 0; cc < HD / 32; ++cc) {
-        uint32_t o32[32];
-        tmem_ld32(tO + cc * 32, o32);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[16 * cc + i] = pack_bf16x2(__uint_as_float(o32[2 * i]) * inv_l, __uint_as_float(o32[2 * i + 1]) * inv_l);
-      }
-      // O_t is out of TMEM: the next item's first P V may overwrite it
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_ofree(t));
-      // coalesced stores: after the chunk transpose, store k of the warp writes
-      // 32 / NCK whole rows (NCK consecutive lanes per row)
-      xpose_chunks<NCK>(pk, lane);
-      const int ck = lane % NCK, rbase = qt * 128 + wq * 32 + (lane / NCK) * NCK;
-#pragma unroll
-      for (int k = 0; k < NCK; ++k) {
-        const int row = rbase + k;
-        if (row < a.S) {
-          uint4* dst = reinterpret_cast<uint4*>(a.o + (((size_t)I.b * a.S + row) * a.Hq + I.h) * HD) + ck;
-          *dst = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-        }
-      }
-      if (row_g < a.S) a.lse[(size_t)I.bh * a.S + row_g] = (m_used + __log2f(l)) * 0.69314718055994531f;
-    }
-  } else if (!FWD_ROWTHREAD && warp < FWD_SOFTMAX_WARPS) {
+  } else if (warp < FWD_SOFTMAX_WARPS) {
     // ===================================================== softmax (tile t, half hf)
-    constexpr bool PIPE = (AXIS_ATTN_FWD_PIPE & (HD == 64 ? 1 : 2)) != 0 && !AXIS_ATTN_FWD_NOXCH &&
-                          !AXIS_ATTN_FWD_TOKEN;
     const int t = warp >> 3, hf = (warp >> 2) & 1, wq = warp & 3;
     const int r = wq * 32 + lane;                   // row in tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
@@ -648,121 +460,18 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     auto xslot = [&](int par, int half) { return xch + ((par * 2 + t) * 2 + half) * 128 + r; };
     const float c = a.scale_log2;
     const uint64_t cc2 = f2_pack(c, c);
-    // phases over all items: J kv tiles of this tile, X exchanges, A_o
-    // exponential phases of the other tile in earlier items
-    int J = 0, X = 0, A_o = 0;
+    // phases over all items: J kv tiles of this tile, X exchanges
+    int J = 0, X = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
       const int w = fwd_item(it);
       if (w >= a.n_items) break;
       const FwdItem I = fwd_decode(a, w, CAUSAL);
-      const int n_t = t == 0 ? I.n0 : I.n1, n_o = t == 0 ? I.n1 : I.n0;
+      const int n_t = t == 0 ? I.n0 : I.n1;
       const int qt = 2 * I.m + t;
       const int row_g = qt * 128 + r;
       float m_used = -INFINITY, l = 0.f;
-      if constexpr (PIPE) {
-        // Speculative order: from the second kv tile on, the exponentials
-        // start with the running max before the other half's partial max is
-        // in (the exchange round trip overlaps them).  The running max moves
-        // only when the row max grows by more than 8; when the other half's
-        // max moves it (rare), this half's packed P and partial row sum are
-        // scaled by alpha = 2^(m_old - m_new) in registers, the correction
-        // the online softmax applies to O.
-        for (int j = 0; j < n_t; ++j, ++J, ++X) {
-          if (!wait_warp<true>(bar_sfull(t), J & 1, abort, F_SFULL)) { ok = false; break; }
-          tc_fence_after();
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tS, v0);
-          tmem_ld32(tS + 32, v1);
-          tmem_wait_ld();
-          // S is in registers: its columns may take the next S
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_sfree(C::SHARED_S ? 0 : t));
-          const bool masked = CAUSAL ? (j == qt) : (j == nkv - 1 && (a.S & 127) != 0);
-          if (masked) {
-            int limit = a.S - 128 * j;
-            if (CAUSAL && r + 1 < limit) limit = r + 1;
-            limit -= hf * 64;  // in this half's columns
-            mask_row(v0, 0, limit);
-            mask_row(v1, 32, limit);
-          }
-          const float mx = fmaxf(row_max32(v0), row_max32(v1));
-          *xslot(X & 1, hf) = mx;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bx);
-          // speculate with the running max when no lane's own half moves it
-          const bool spec = j > 0 && __all_sync(0xffffffffu, !(fmaxf(m_used, mx * c) > m_used + 8.0f));
-          uint64_t acc = f2_pack(0.f, 0.f);
-          uint32_t pk0[16], pk1[16];
-          float alpha = 1.f;
-          bool resc = false;
-          // the other half's partial max, the row max, and the running max update
-#define AXIS_ATTN_FWD_ROW_MAX()                                                    \
-  if (!wait_warp<true>(bx, X & 1, abort, F_XCH)) {                                 \
-    ok = false;                                                                    \
-    break;                                                                         \
-  }                                                                                \
-  {                                                                                \
-    const float m_new = fmaxf(m_used, fmaxf(mx, *xslot(X & 1, hf ^ 1)) * c);       \
-    resc = m_new > m_used + 8.0f;                                                  \
-    if (resc) {                                                                    \
-      alpha = ex2_approx(m_used - m_new);                                          \
-      m_used = m_new;                                                              \
-    }                                                                              \
-  }
-          if (spec) {
-            {
-              const uint64_t nm2 = f2_pack(-m_used, -m_used);
-              acc = exp_pairs<0, 16>(v0, cc2, nm2, acc, pk0);
-              acc = exp_pairs<0, 16>(v1, cc2, nm2, acc, pk1);
-            }
-            AXIS_ATTN_FWD_ROW_MAX()
-            if (__any_sync(0xffffffffu, resc)) {  // rare: rescale this half's P and row sum
-              const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                pk0[i] = pack_bf16x2(f2_mul(f2_pack(__uint_as_float(pk0[i] << 16), __uint_as_float(pk0[i] & 0xffff0000u)), a2));
-                pk1[i] = pack_bf16x2(f2_mul(f2_pack(__uint_as_float(pk1[i] << 16), __uint_as_float(pk1[i] & 0xffff0000u)), a2));
-              }
-              acc = f2_mul(acc, a2);
-            }
-          } else {
-            AXIS_ATTN_FWD_ROW_MAX()
-            const uint64_t nm2 = f2_pack(-m_used, -m_used);
-            acc = exp_pairs<0, 16>(v0, cc2, nm2, acc, pk0);
-            acc = exp_pairs<0, 16>(v1, cc2, nm2, acc, pk1);
-          }
-#undef AXIS_ATTN_FWD_ROW_MAX
-          const bool any_resc = __any_sync(0xffffffffu, resc);
-          float rs_lo, rs_hi;
-          f2_unpack(acc, rs_lo, rs_hi);
-          l = l * alpha + (rs_lo + rs_hi);
-          // the previous P V must have landed before P_t is overwritten and O_t rescaled
-          if (J > 0) {
-            if (!wait_warp<true>(bar_o(t), (J - 1) & 1, abort, F_OWAIT)) { ok = false; break; }
-            tc_fence_after();
-          }
-          tmem_st16(tP, pk0);
-          tmem_st16(tP + 16, pk1);
-          if (j > 0 && any_resc) {
-#pragma unroll 1
-            for (int cc = 0; cc < HD / 64; ++cc) {
-              uint32_t v[32];
-              tmem_ld32(tO + cc * 32, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-              tmem_st32(tO + cc * 32, v);
-            }
-          }
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0 && !(AXIS_ATTN_TEST_DROP_ARRIVE == 1 && J == 0 && t == 0)) mbar_arrive(bar_pfull(t));
-        }
-      } else
-      for (int j = 0; j < n_t; ++j, ++J, X += !AXIS_ATTN_FWD_NOXCH) {
+      for (int j = 0; j < n_t; ++j, ++J, ++X) {
         if (!wait_warp<true>(bar_sfull(t), J & 1, abort, F_SFULL)) { ok = false; break; }
         tc_fence_after();
         const bool masked = CAUSAL ? (j == qt) : (j == nkv - 1 && (a.S & 127) != 0);
@@ -771,22 +480,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           limit = a.S - 128 * j;
           if (CAUSAL && r + 1 < limit) limit = r + 1;
         }
-        float mo = -INFINITY;  // the other half's partial max (second TMEM pass)
-        uint32_t v0[32], v1[32];
-        if (AXIS_ATTN_FWD_NOXCH) {
-          const uint32_t tSo = tS + (hf ? -64 : 64);
-          tmem_ld32(tSo, v0);
-          tmem_ld32(tSo + 32, v1);
-          tmem_wait_ld();
-          if (masked) {
-            const int lo = limit - (hf ^ 1) * 64;
-            mask_row(v0, 0, lo);
-            mask_row(v1, 32, lo);
-          }
-          mo = fmaxf(row_max32(v0), row_max32(v1));
-        }
         limit -= hf * 64;  // in this half's columns
         // this half of the 128-column row of S in registers (one TMEM pass)
+        uint32_t v0[32], v1[32];
         tmem_ld32(tS, v0);
         tmem_ld32(tS + 32, v1);
         tmem_wait_ld();
@@ -798,17 +494,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           mask_row(v0, 0, limit);
           mask_row(v1, 32, limit);
         }
-        // row max: this half's, then the other half's (from TMEM, or through shared memory)
+        // row max: this half's, then the other half's (through shared memory)
         float mx = fmaxf(row_max32(v0), row_max32(v1));
-        if (AXIS_ATTN_FWD_NOXCH) {
-          mx = fmaxf(mx, mo);
-        } else {
-          *xslot(X & 1, hf) = mx;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bx);
-          if (!wait_warp<true>(bx, X & 1, abort, F_XCH)) { ok = false; break; }
-          mx = fmaxf(mx, *xslot(X & 1, hf ^ 1));
-        }
+        *xslot(X & 1, hf) = mx;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bx);
+        if (!wait_warp<true>(bx, X & 1, abort, F_XCH)) { ok = false; break; }
+        mx = fmaxf(mx, *xslot(X & 1, hf ^ 1));
         const float m_new = fmaxf(m_used, mx * c);
         const bool resc = m_new > m_used + 8.0f;
         float alpha = 1.f;
@@ -816,27 +508,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           alpha = ex2_approx(m_used - m_new);
           m_used = m_new;
         }
-        // Take turns with the other tile on the exponentials.  The phases of
-        // both tiles form one sequence over all items, t0(0) t1(0) t0(1)
-        // t1(1) ... (the longer tile's extra phases last); wait until the
-        // other tile has finished every phase before this one in it.
-        if (AXIS_ATTN_FWD_TOKEN) {
-          const int need = A_o + (t == 0 ? min(j, n_o) : min(j + 1, n_o));
-          if (need > 0 && !wait_warp<true>(bar_tok(t), (need - 1) & 1, abort, F_TOK)) { ok = false; break; }
-        }
         // p = 2^(s*c - m) (masked entries are -inf and give 0), row sum, bf16
-        // P pairs in registers; the token goes to the other tile three
-        // quarters of the way through, to hide its wake-up
+        // P pairs in registers
         const uint64_t nm2 = f2_pack(-m_used, -m_used);
         uint64_t acc = f2_pack(0.f, 0.f);
         uint32_t pk0[16], pk1[16];
         acc = exp_pairs<0, 16>(v0, cc2, nm2, acc, pk0);
-        acc = exp_pairs<0, 8>(v1, cc2, nm2, acc, pk1);
-        if (AXIS_ATTN_FWD_TOKEN) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_tok(1 - t));
-        }
-        acc = exp_pairs<8, 8>(v1, cc2, nm2, acc, pk1);
+        acc = exp_pairs<0, 16>(v1, cc2, nm2, acc, pk1);
         float rs_lo, rs_hi;
         f2_unpack(acc, rs_lo, rs_hi);
         l = l * alpha + (rs_lo + rs_hi);
@@ -864,7 +542,6 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         __syncwarp();
         if (lane == 0 && !(AXIS_ATTN_TEST_DROP_ARRIVE == 1 && J == 0 && t == 0)) mbar_arrive(bar_pfull(t));
       }
-      A_o += n_o;
       if (!ok || n_t == 0) continue;
       // epilogue: the halves' row sums are added, O / l -> bf16 (each half
       // its HD/2 columns), LSE = (m + log2 l) ln 2

@@ -278,7 +278,7 @@ int axis_attn_get_status(void* stream);
  * Diagnostics: the raw device status word that the last axis_attn_get_status()
  * call read before clearing it (0 if none was set).  Bit 0: a wait timed out;
  * bit 1: a decode index was out of range; bits 8..15: the wait site that first
- * timed out (1..13: forward kernel, 21..32: backward main kernel, 41..42:
+ * timed out (1..12: forward kernel, 21..32: backward main kernel, 41..42:
  * decode kernel).
  */
 unsigned int axis_attn_last_status_word(void);

@@ -83,6 +83,10 @@ CASES = [
     (1, 32, 8, 128, 8192, 64, [8192]),               # one long sequence: split-K
     (2, 24, 8, 64, 5000, 8, [4999, 3]),               # G = 3, small pages, split-K
     (64, 32, 8, 128, 600, 16, list(range(9, 9 + 64 * 9, 9))),  # many sequences: no split
+    # more than 32 pieces of 32 keys per CTA: the producer reads the block
+    # table in several blocks of 32 pieces (3 at 2100 keys, 2 at 1500)
+    (40, 8, 8, 64, 2100, 8, [2100, 1, 1024, 1025, 2047, 2048, 2049, 33] * 5),
+    (40, 16, 8, 128, 1500, 16, [1500, 1023, 1056, 17, 1499] * 8),
 ]
 
 
