@@ -494,6 +494,13 @@ def time_decode(aa, name, dev, steps, flush, hbm_gbs):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs}}
 
 
+def launches_per_step(aa, w) -> int:
+    """Kernels of ours one step launches: the forward, the backward's
+    preprocess, main kernel and dQ stage (finalize, or the deterministic dQ
+    pass), and the partial dK/dV sum when the backward splits the heads."""
+    return 4 + (aa.axis_attn_bwd_head_split(w.B, w.Hq, w.Hkv, w.S, w.D) > 1)
+
+
 def time_e2e(aa, w, prob, steps: int, det: bool, world: int, dev) -> dict:
     """The step end to end through the public torch helpers, from pinned host
     buffers: every step copies its Q, K, V, dO host->device and its O, LSE,
@@ -574,7 +581,7 @@ def summarize(w, total_ms, stage_totals, steps, world, p_meas, det):
     fwd_tf = w.fwd_flops / (avg[0] * 1e-3) / 1e12
     bwd_ms = sum(avg[1:])
     bwd_tf = w.bwd_flops / (bwd_ms * 1e-3) / 1e12
-    names = STAGES if not det else ["attn_fwd_kernel", "-", "-", "axis_attn_bwd_det (prep + main + dq_sum)"]
+    names = STAGES if not det else ["attn_fwd_kernel", "-", "-", "axis_attn_bwd_det (prep + main + dQ pass)"]
     return {
         "value": whole_job_tflops(w.fwd_flops + w.bwd_flops, steps, total_ms, world),
         "ms_per_step": total_ms / steps, "steps": steps,
@@ -678,7 +685,10 @@ def main():
         summ["config"] = wo.describe()
         summ["clocks"] = sampler.summary(*wwin)
         others[name] = summ
-        summ["gpu_launches"] = 4 * ko
+        summ["gpu_launches"] = launches_per_step(aa, wo) * ko
+        hs = aa.axis_attn_bwd_head_split(wo.B, wo.Hq, wo.Hkv, wo.S, wo.D)
+        if hs > 1:  # the main-kernel stage then also holds the partial dK/dV sum
+            summ["bwd_head_split"] = hs
         del po
         torch.cuda.empty_cache()
     # ---- the headline workload with RoPE fused, and the decode step
@@ -716,7 +726,7 @@ def main():
                                     "kernel_ms")},
             "bwd_mode": "deterministic (axis_attn_bwd_det)" if det else "ordinary (axis_attn_bwd stages)",
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": 4 * K, "clocks": clocks,
+            "gpu_launches": launches_per_step(aa, w) * K, "clocks": clocks,
             "workloads": others, "rope": rope, "decode": decode,
         }
         print(json.dumps(line))

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(PKG, "libaxis_attn.so")
 EXPORTS = (
     "axis_attn_fwd",
     "axis_attn_bwd_workspace_bytes",
+    "axis_attn_bwd_head_split",
     "axis_attn_bwd",
     "axis_attn_bwd_prepare",
     "axis_attn_bwd_main",
@@ -80,6 +81,8 @@ def load():
             lib.axis_attn_fwd.restype = i
             lib.axis_attn_bwd_workspace_bytes.argtypes = [i] * 5
             lib.axis_attn_bwd_workspace_bytes.restype = sz
+            lib.axis_attn_bwd_head_split.argtypes = [i] * 5
+            lib.axis_attn_bwd_head_split.restype = i
             lib.axis_attn_bwd.argtypes = [vp] * 9 + [i] * 5 + [f, i, vp, sz, vp]
             lib.axis_attn_bwd.restype = i
             lib.axis_attn_bwd_prepare.argtypes = [vp] * 3 + [i] * 5 + [vp, sz, vp]
@@ -123,6 +126,10 @@ def axis_attn_fwd(q, k, v, o, lse, B, Hq, Hkv, S, D, scale, causal, stream) -> i
 
 def axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D) -> int:
     return int(load().axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D))
+
+
+def axis_attn_bwd_head_split(B, Hq, Hkv, S, D) -> int:
+    return int(load().axis_attn_bwd_head_split(B, Hq, Hkv, S, D))
 
 
 def axis_attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, causal,

@@ -62,6 +62,13 @@ struct BwdArgs {
   float scale, scale_log2;
   int no_dq;           // 1: dK, dV only (deterministic mode: attn_bwd_dq_kernel computes dQ)
   const double2* rope_cs;  // RoPE: (cos, sin) table [S][HD/2], fp64; dK leaves through the transposed rotation
+  // Head split (small grids): hsplit CTAs share a (b, kv head, key tile), each
+  // taking G / hsplit of the group's query heads, and write fp32 partial dK
+  // (x scale), dV to dk_part, dv_part [hsplit][B][S][Hkv][HD] for
+  // attn_bwd_dkv_sum_kernel to add up; hsplit = 1: dK, dV straight to dk, dv.
+  int hsplit;
+  float* dk_part;
+  float* dv_part;
 };
 
 template <int HD>
@@ -203,12 +210,16 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work item
+  // ---- work item: key tile j of unit (b, kv head); with a head split, the
+  // hsplit CTAs of a unit and key tile are adjacent in the launch order (they
+  // share K_j, V_j in L2) and take consecutive blocks of the group's heads
   const int BKV = a.B * a.Hkv;
+  const int hs = (int)blockIdx.x % a.hsplit;
   int j, bkv;
-  bwd_item(BKV, (a.S + 127) / 128, (int)blockIdx.x, j, bkv);
+  bwd_item(BKV, (a.S + 127) / 128, (int)blockIdx.x / a.hsplit, j, bkv);
   const int b = bkv / a.Hkv, kvh = bkv % a.Hkv;
-  const int G = a.Hq / a.Hkv;
+  const int G = a.Hq / a.Hkv / a.hsplit;  // query heads of this CTA
+  const int h0 = kvh * (G * a.hsplit) + hs * G;
   const int nqt = (a.S + BM - 1) / BM;
   const int i0 = CAUSAL ? (128 * j) / BM : 0;
   const int per_head = nqt - i0;
@@ -257,7 +268,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
       // L2 prefetch of the Q / dO tiles PF steps ahead of the loads
       constexpr int PF = 4;
       auto prefetch = [&](int it) {
-        const int h = kvh * G + it / per_head;
+        const int h = h0 + it / per_head;
         const int q0 = (i0 + it % per_head) * BM;
         for (int sl = 0; sl < C::NSLAB; ++sl) {
           tma_prefetch_4d(&tm_q, 64 * sl, h, q0, b);
@@ -270,7 +281,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
         const int s = it % ST;
         if (it + PF < n_it) prefetch(it + PF);
         if (!mbar_wait_bounded(bar_qempty(s), ((it / ST) & 1) ^ 1, abort, B_QEMPTY)) break;
-        const int h = kvh * G + it / per_head;
+        const int h = h0 + it / per_head;
         const int q0 = (i0 + it % per_head) * BM;
         const size_t row = ((size_t)b * a.Hq + h) * a.S_pad + q0;
         mbar_arrive_expect_tx(bar_qfull(s), 2 * C::QTILE + 2 * BM * 4);
@@ -373,7 +384,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
       tma_prefetch_desc(&tm_dq);
       for (int t = 0; t < n_it; ++t) {
         if (!mbar_wait_bounded(bar_stgfull, t & 1, abort, B_STGFULL)) break;
-        const int h = kvh * G + t / per_head;
+        const int h = h0 + t / per_head;
         const int q0 = (i0 + t % per_head) * BM;
         const int bh = b * a.Hq + h;
         for (int bx = 0; bx < 4; ++bx) {
@@ -544,12 +555,25 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
       const int f0 = (ch % GPT) * (HD / GPT);  // first feature of this group
       const uint32_t tcol = (is_dv ? C::T_DV : C::T_DK) + f0;
       const float mul = is_dv ? 1.f : a.scale;
-      __nv_bfloat16* dst_row = (is_dv ? a.dv : a.dk) + (((size_t)b * a.S + key) * a.Hkv + kvh) * HD + f0;
+      const size_t row_off = (((size_t)b * a.S + key) * a.Hkv + kvh) * HD + f0;
+      __nv_bfloat16* dst_row = (is_dv ? a.dv : a.dk) + row_off;
+      float* part_row = a.hsplit > 1 ? (is_dv ? a.dv_part : a.dk_part) + (size_t)hs * a.B * a.S * a.Hkv * HD + row_off
+                                     : nullptr;
 #pragma unroll 1
       for (int cc = 0; cc < HD / GPT / 32; ++cc) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_off + tcol + cc * 32, v);
         tmem_wait_ld();
+        if (part_row != nullptr) {  // head split: this CTA's fp32 share, summed (and rotated) later
+          if (key < a.S) {
+            float4* dst = reinterpret_cast<float4*>(part_row + cc * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]) * mul, __uint_as_float(v[4 * i + 1]) * mul,
+                                   __uint_as_float(v[4 * i + 2]) * mul, __uint_as_float(v[4 * i + 3]) * mul);
+          }
+          continue;
+        }
         uint32_t pk2[16];
         if (a.rope_cs != nullptr && !is_dv && key < a.S) {
           // dK = R(key)^T dK': pairs of features f0 + 32 cc + 2 i
@@ -672,6 +696,48 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
     out.z = pack_bf16x2(y.x, y.y);
     out.w = pack_bf16x2(y.z, y.w);
     reinterpret_cast<uint4*>(dq + row * HD)[c8] = out;
+  }
+}
+
+// Head split: dk[b,j,kv,:] = bf16(sum over the hsplit partial rows), likewise
+// dv; the partials are added in a fixed order (bitwise reproducible).  With a
+// RoPE table dK leaves through the transposed rotation of position j.  8
+// features per thread.
+template <int HD>
+__global__ void __launch_bounds__(256) attn_bwd_dkv_sum_kernel(const float* __restrict__ dk_part,
+                                                               const float* __restrict__ dv_part,
+                                                               __nv_bfloat16* __restrict__ dk,
+                                                               __nv_bfloat16* __restrict__ dv, int hsplit,
+                                                               int S, int Hkv, size_t n8,
+                                                               const double2* __restrict__ rope_cs) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  const size_t part = n8 * 8;  // floats of one partial tensor
+  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < 2 * n8; k += stride) {
+    const bool is_k = k < n8;
+    const size_t e = is_k ? k : k - n8;  // 8-feature chunk in [B, S, Hkv, HD / 8]
+    const float* src = (is_k ? dk_part : dv_part) + 8 * e;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+    for (int g = 0; g < hsplit; ++g) {
+      const float4 a0 = reinterpret_cast<const float4*>(src + g * part)[0];
+      const float4 a1 = reinterpret_cast<const float4*>(src + g * part)[1];
+      x.x += a0.x; x.y += a0.y; x.z += a0.z; x.w += a0.w;
+      y.x += a1.x; y.y += a1.y; y.z += a1.z; y.w += a1.w;
+    }
+    const int c8 = (int)(e % (HD / 8));
+    if (is_k && rope_cs != nullptr) {
+      const int pos = (int)((e / (HD / 8) / Hkv) % S);
+      const double2* t = rope_cs + (size_t)pos * (HD / 2) + 4 * c8;
+      rope_back(x.x, x.y, t[0]);
+      rope_back(x.z, x.w, t[1]);
+      rope_back(y.x, y.y, t[2]);
+      rope_back(y.z, y.w, t[3]);
+    }
+    uint4 out;
+    out.x = pack_bf16x2(x.x, x.y);
+    out.y = pack_bf16x2(x.z, x.w);
+    out.z = pack_bf16x2(y.x, y.y);
+    out.w = pack_bf16x2(y.z, y.w);
+    reinterpret_cast<uint4*>(is_k ? dk : dv)[e] = out;
   }
 }
 

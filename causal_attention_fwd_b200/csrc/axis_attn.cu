@@ -93,21 +93,42 @@ bool make_dq_map(CUtensorMap* map, const float* ptr, int BH, int S, int D) {
 
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Head split of the backward main kernel: with fewer than BWD_SPLIT_CTAS
+// (b, kv head, key tile) CTAs and more than one query head per kv head, the
+// group's heads are dealt over hsplit CTAs (the smallest divisor of G that
+// reaches that many CTAs, else G), which write fp32 partial dK, dV.
+#ifndef AXIS_ATTN_BWD_SPLIT_CTAS
+#define AXIS_ATTN_BWD_SPLIT_CTAS 148
+#endif
+constexpr long long BWD_SPLIT_CTAS = AXIS_ATTN_BWD_SPLIT_CTAS;
+int bwd_hsplit(int B, int Hq, int Hkv, int S) {
+  const int G = Hq / Hkv;
+  const long long ctas = (long long)((S + 127) / 128) * B * Hkv;
+  if (G <= 1 || ctas >= BWD_SPLIT_CTAS) return 1;
+  for (int d = 2; d < G; ++d)
+    if (G % d == 0 && ctas * d >= BWD_SPLIT_CTAS) return d;
+  return G;
+}
+
 struct WsLayout {
-  size_t lse2, dr, dqacc, total;
-  int S_pad;
+  size_t lse2, dr, dqacc, dkpart, dvpart, total;
+  int S_pad, hsplit;
 };
 
-// det: no dQ accumulator (the deterministic dQ pass keeps dQ in TMEM), so the
-// workspace is the two row sections only.
-WsLayout ws_layout(int B, int Hq, int S, int D, bool det = false) {
+// det: no dQ accumulator (the deterministic dQ pass keeps dQ in TMEM).  With a
+// head split, two fp32 partial sections [hsplit][B][S][Hkv][D] follow.
+WsLayout ws_layout(int B, int Hq, int Hkv, int S, int D, bool det = false) {
   WsLayout w;
   w.S_pad = (S + 127) / 128 * 128;
+  w.hsplit = bwd_hsplit(B, Hq, Hkv, S);
   const size_t rows = (size_t)B * Hq * w.S_pad;
   w.lse2 = 0;
   w.dr = round256(rows * 4);
   w.dqacc = w.dr + round256(rows * 4);
-  w.total = w.dqacc + (det ? 0 : round256((size_t)B * Hq * S * D * 4));
+  w.dkpart = w.dqacc + (det ? 0 : round256((size_t)B * Hq * S * D * 4));
+  const size_t part = w.hsplit > 1 ? round256((size_t)w.hsplit * B * S * Hkv * D * 4) : 0;
+  w.dvpart = w.dkpart + part;
+  w.total = w.dvpart + part;
   return w;
 }
 
@@ -199,7 +220,7 @@ int launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensor
   auto kern = attn_bwd_kernel<HD, CAUSAL>;
   static bool done[64];
   if (int rc = set_smem(kern, BwdCfg<HD>::SMEM, dev, done)) return rc;
-  const unsigned grid = (unsigned)((a.S + 127) / 128) * a.B * a.Hkv;
+  const unsigned grid = (unsigned)((a.S + 127) / 128) * a.B * a.Hkv * a.hsplit;
   kern<<<grid, BwdCfg<HD>::THREADS, BwdCfg<HD>::SMEM, st>>>(mq, mk, mv, mdo, mdq, a);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
@@ -222,7 +243,12 @@ extern "C" int axis_attn_fwd(const void* q, const void* k, const void* v, void* 
 
 extern "C" size_t axis_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
   if (check_shape(B, Hq, Hkv, S, D, 1.f) != AXIS_ATTN_OK) return 0;
-  return ws_layout(B, Hq, S, D).total;
+  return ws_layout(B, Hq, Hkv, S, D).total;
+}
+
+extern "C" int axis_attn_bwd_head_split(int B, int Hq, int Hkv, int S, int D) {
+  if (check_shape(B, Hq, Hkv, S, D, 1.f) != AXIS_ATTN_OK) return 0;
+  return bwd_hsplit(B, Hq, Hkv, S);
 }
 
 namespace {
@@ -234,13 +260,14 @@ int check_ws(void* workspace, size_t workspace_bytes, const WsLayout& w) {
 }
 
 struct WsPtrs {
-  float *lse2, *dr, *dqacc;
+  float *lse2, *dr, *dqacc, *dkpart, *dvpart;
 };
 
 WsPtrs ws_ptrs(void* workspace, const WsLayout& w) {
   char* ws = static_cast<char*>(workspace);
   return {reinterpret_cast<float*>(ws + w.lse2), reinterpret_cast<float*>(ws + w.dr),
-          reinterpret_cast<float*>(ws + w.dqacc)};
+          reinterpret_cast<float*>(ws + w.dqacc), reinterpret_cast<float*>(ws + w.dkpart),
+          reinterpret_cast<float*>(ws + w.dvpart)};
 }
 
 }  // namespace
@@ -293,11 +320,28 @@ int run_main(const void* q, const void* k, const void* v, const void* dO, void* 
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
   a.no_dq = det ? 1 : 0;
   a.rope_cs = reinterpret_cast<const double2*>(rope_cs);
+  a.hsplit = w.hsplit;
+  a.dk_part = p.dkpart;
+  a.dv_part = p.dvpart;
+  int rc;
   if (D == 64)
-    return causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, mdq, a, st, dev)
-                  : launch_bwd_main<64, false>(mq, mk, mv, mdo, mdq, a, st, dev);
-  return causal ? launch_bwd_main<128, true>(mq, mk, mv, mdo, mdq, a, st, dev)
+    rc = causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, mdq, a, st, dev)
+                : launch_bwd_main<64, false>(mq, mk, mv, mdo, mdq, a, st, dev);
+  else
+    rc = causal ? launch_bwd_main<128, true>(mq, mk, mv, mdo, mdq, a, st, dev)
                 : launch_bwd_main<128, false>(mq, mk, mv, mdo, mdq, a, st, dev);
+  if (rc || w.hsplit == 1) return rc;
+  // head split: add up the partial dK, dV (fixed order) into bf16 dk, dv
+  const size_t n8 = (size_t)B * S * Hkv * D / 8;
+  const unsigned grid = (unsigned)((2 * n8 + 255) / 256 < 148 * 8 ? (2 * n8 + 255) / 256 : 148 * 8);
+  auto* dkb = static_cast<__nv_bfloat16*>(dk);
+  auto* dvb = static_cast<__nv_bfloat16*>(dv);
+  const double2* cs = reinterpret_cast<const double2*>(rope_cs);
+  if (D == 64)
+    attn_bwd_dkv_sum_kernel<64><<<grid, 256, 0, st>>>(p.dkpart, p.dvpart, dkb, dvb, w.hsplit, S, Hkv, n8, cs);
+  else
+    attn_bwd_dkv_sum_kernel<128><<<grid, 256, 0, st>>>(p.dkpart, p.dvpart, dkb, dvb, w.hsplit, S, Hkv, n8, cs);
+  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
 // Stage 3: dQ to bf16 [B,S,Hq,D].
@@ -322,7 +366,7 @@ extern "C" int axis_attn_bwd_prepare(const void* o, const void* dO, const float*
   if (!o || !dO || !lse) return AXIS_ATTN_ERR_NULL;
   if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return AXIS_ATTN_ERR_ALIGN;
   if (int rc = check_shape(B, Hq, Hkv, S, D, 1.f)) return rc;
-  const WsLayout w = ws_layout(B, Hq, S, D);
+  const WsLayout w = ws_layout(B, Hq, Hkv, S, D);
   if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
@@ -336,7 +380,7 @@ extern "C" int axis_attn_bwd_main(const void* q, const void* k, const void* v, c
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv))
     return AXIS_ATTN_ERR_ALIGN;
   if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
-  const WsLayout w = ws_layout(B, Hq, S, D);
+  const WsLayout w = ws_layout(B, Hq, Hkv, S, D);
   if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
@@ -349,7 +393,7 @@ extern "C" int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, i
   if (!dq) return AXIS_ATTN_ERR_NULL;
   if (!aligned16(dq)) return AXIS_ATTN_ERR_ALIGN;
   if (int rc = check_shape(B, Hq, Hkv, S, D, 1.f)) return rc;
-  const WsLayout w = ws_layout(B, Hq, S, D);
+  const WsLayout w = ws_layout(B, Hq, Hkv, S, D);
   if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
@@ -396,7 +440,7 @@ int run_bwd(const void* q, const void* k, const void* v, const void* o, const vo
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (rope_cs && !aligned16(rope_cs)))
     return AXIS_ATTN_ERR_ALIGN;
   if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
-  const WsLayout w = ws_layout(B, Hq, S, D, det);
+  const WsLayout w = ws_layout(B, Hq, Hkv, S, D, det);
   if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
@@ -420,7 +464,7 @@ extern "C" int axis_attn_bwd(const void* q, const void* k, const void* v, const 
 
 extern "C" size_t axis_attn_bwd_det_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
   if (check_shape(B, Hq, Hkv, S, D, 1.f) != AXIS_ATTN_OK) return 0;
-  return ws_layout(B, Hq, S, D, true).total;
+  return ws_layout(B, Hq, Hkv, S, D, true).total;
 }
 
 extern "C" int axis_attn_bwd_det(const void* q, const void* k, const void* v, const void* o, const void* dO,
@@ -521,7 +565,7 @@ extern "C" int axis_attn_bwd_noalloc(const void* q, const void* k, const void* v
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return AXIS_ATTN_ERR_ALIGN;
   if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
-  if (ws_layout(B, Hq, S, D).total > (size_t)AXIS_ATTN_NOALLOC_SCRATCH_BYTES) return AXIS_ATTN_ERR_WORKSPACE;
+  if (ws_layout(B, Hq, Hkv, S, D).total > (size_t)AXIS_ATTN_NOALLOC_SCRATCH_BYTES) return AXIS_ATTN_ERR_WORKSPACE;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
   void* scratch = nullptr;

@@ -75,9 +75,23 @@ int axis_attn_fwd(const void* q, const void* k, const void* v, void* o, float* l
  * Bytes of device workspace axis_attn_bwd() needs for these sizes (0 if the
  * sizes are invalid).  It holds, per (b, query head), fp32 rows of
  * log2-scaled LSE and of Dr = rowsum(dO * O), padded to a multiple of 128,
- * and an fp32 dQ accumulator [B, Hq, S, D].
+ * and an fp32 dQ accumulator [B, Hq, S, D]; each section starts on a 256-byte
+ * boundary.  Small problems add two fp32 sections [hsplit, B, S, Hkv, D] of
+ * partial dK, dV (see axis_attn_bwd_head_split()).
  */
 size_t axis_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int S, int D);
+
+/*
+ * How many CTAs share each (b, kv head, 128-key tile) of the backward main
+ * kernel: 1, or for small problems -- fewer than 148 such tiles and more
+ * than one query head per kv head -- the smallest divisor of G = Hq / Hkv
+ * that gives at least 148 CTAs (else G).  The G query heads of a kv head are
+ * then dealt over that many CTAs, each writes its fp32 share of dK and dV to
+ * the workspace, and one more kernel adds the shares up in a fixed order
+ * into dk and dv (so the result stays bitwise reproducible).  0 for invalid
+ * sizes.  Informational: the other calls apply it themselves.
+ */
+int axis_attn_bwd_head_split(int B, int Hq, int Hkv, int S, int D);
 
 /*
  * Backward.  Given the forward's inputs q, k, v, its outputs o and lse, and the
@@ -105,7 +119,8 @@ int axis_attn_bwd(const void* q, const void* k, const void* v, const void* o,
  *   prepare:  Dr = rowsum(dO * O) and LSE * log2(e) into the workspace; zeroes
  *             the fp32 dQ accumulator.  Reads o, dO, lse.
  *   main:     dk, dv (written) and the dQ accumulator (added into).  Reads q, k,
- *             v, dO and the workspace.
+ *             v, dO and the workspace.  (With a head split, a second kernel
+ *             adds up the partial dK, dV.)
  *   finalize: dq = bf16(dQ accumulator).
  */
 int axis_attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, int Hkv,
@@ -139,7 +154,9 @@ int axis_attn_bwd_finalize(void* dq, int B, int Hq, int Hkv, int S, int D, void*
  * smaller workspace
  *   axis_attn_bwd_det_workspace_bytes() = 2 * round256(4 * B * Hq * S_pad),
  *   S_pad = ceil(S / 128) * 128
- * (about 2.1 MB for B=4, Hq=32, S=2048).  A workspace shorter than that
+ * (about 2.1 MB for B=4, Hq=32, S=2048), plus, with a head split
+ * (axis_attn_bwd_head_split() = n > 1), 2 * round256(4 * n * B * S * Hkv * D)
+ * for the partial dK, dV.  A workspace shorter than that
  * returns AXIS_ATTN_ERR_WORKSPACE and launches nothing.  Returns 0 from the
  * size function for invalid sizes.
  */

@@ -46,12 +46,38 @@ def test_strerror_covers_every_status(lib):
     assert aa.axis_attn_strerror(99) == "unknown status"
 
 
+def head_split(B, Hq, Hkv, S):
+    """The header's rule: with fewer than 148 (b, kv head, 128-key tile) CTAs
+    and G = Hq / Hkv > 1, the smallest divisor of G reaching 148 CTAs, else G."""
+    G, ctas = Hq // Hkv, -(-S // 128) * B * Hkv
+    if G == 1 or ctas >= 148:
+        return 1
+    return next((d for d in range(2, G) if G % d == 0 and ctas * d >= 148), G)
+
+
+def test_head_split_rule(lib):
+    for B, Hq, Hkv, S, want in ((4, 32, 8, 2048, 1),      # llm1b: 512 CTAs
+                                (2, 12, 4, 1024, 3),      # gpt2s_gqa: 64 CTAs, G = 3
+                                (1, 1, 1, 128, 1),        # G = 1: nothing to split
+                                (1, 8, 1, 1000, 8),       # 8 CTAs: every head its own CTA
+                                (2, 16, 2, 2048, 4),      # 64 CTAs x 2 = 128 < 148: the next divisor
+                                (3, 16, 2, 2048, 2)):     # 96 x 2 = 192 >= 148
+        got = aa.axis_attn_bwd_head_split(B, Hq, Hkv, S, 64)
+        assert got == head_split(B, Hq, Hkv, S) == want, (B, Hq, Hkv, S)
+    assert aa.axis_attn_bwd_head_split(1, 3, 2, 128, 64) == 0  # invalid sizes
+
+
 def test_workspace_bytes(lib):
     # lse2 + dr rows padded to 128, each section rounded to 256 bytes, + fp32 dQ accumulator
-    B, Hq, Hkv, S, D = 2, 12, 4, 1000, 64
-    rows = B * Hq * 1024
+    # (+ two fp32 partial dK, dV sections when the backward splits the heads)
     r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    B, Hq, Hkv, S, D = 4, 32, 8, 1000, 64  # 256 CTAs: no head split
+    rows = B * Hq * 1024
     assert aa.axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D) == 2 * r256(rows * 4) + r256(B * Hq * S * D * 4)
+    B, Hq, Hkv, S, D = 2, 12, 4, 1000, 64  # 64 CTAs, G = 3: split in 3
+    rows = B * Hq * 1024
+    assert aa.axis_attn_bwd_workspace_bytes(B, Hq, Hkv, S, D) == (
+        2 * r256(rows * 4) + r256(B * Hq * S * D * 4) + 2 * r256(3 * B * S * Hkv * D * 4))
     assert aa.axis_attn_bwd_workspace_bytes(1, 3, 2, 128, 64) == 0      # Hq % Hkv != 0
     assert aa.axis_attn_bwd_workspace_bytes(1, 1, 1, 128, 96) == 0      # unsupported D
     assert aa.axis_attn_bwd_workspace_bytes(1, 1, 1, 0, 64) == 0        # empty sequence
@@ -59,10 +85,14 @@ def test_workspace_bytes(lib):
 
 def test_det_workspace_bytes(lib):
     # only the two row sections: dQ stays on chip in the deterministic pass
-    B, Hq, Hkv, S, D = 2, 12, 4, 1000, 64
-    rows = B * Hq * 1024
+    B, Hq, Hkv, S, D = 4, 12, 4, 5000, 64  # 320 CTAs: no head split
+    rows = B * Hq * 5120
     r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
     assert aa.axis_attn_bwd_det_workspace_bytes(B, Hq, Hkv, S, D) == 2 * r256(rows * 4)
+    # a head split adds the partial dK, dV sections (2 x 12 x 1000: 64 CTAs, split in 3)
+    B, Hq, Hkv, S, D = 2, 12, 4, 1000, 64
+    assert aa.axis_attn_bwd_det_workspace_bytes(B, Hq, Hkv, S, D) == (
+        2 * r256(B * Hq * 1024 * 4) + 2 * r256(3 * B * S * Hkv * D * 4))
     # the header's example: B=4, Hq=32, S=2048 needs about 2.1 MB, flat in D
     assert aa.axis_attn_bwd_det_workspace_bytes(4, 32, 8, 2048, 64) == 2 * r256(4 * 32 * 2048 * 4)
     assert aa.axis_attn_bwd_det_workspace_bytes(4, 32, 8, 2048, 128) == 2 * r256(4 * 32 * 2048 * 4)
@@ -115,8 +145,8 @@ def test_bwd_rejects(lib, over, code):
 @pytest.mark.parametrize("over,code", [
     (dict(dO=None), 1), (dict(dq=None), 1), (dict(dk=A + 8), 2), (dict(S=0), 3), (dict(D=80), 4),
     (dict(workspace=None), 5), (dict(workspace=A + 16), 5),
-    # one byte short of the two row sections
-    (dict(S=1000, workspace_bytes=2 * 1024 * 2 * 4 - 1), 5),
+    # one byte short of the two row sections and the two partial sections (split in 2)
+    (dict(S=1000, workspace_bytes=2 * 1024 * 2 * 4 + 2 * 2 * 1000 * 64 * 4 - 1), 5),
 ])
 def test_bwd_det_rejects(lib, over, code):
     args = dict(q=A, k=A, v=A, o=A, dO=A, lse=A, dq=A, dk=A, dv=A, B=1, Hq=2, Hkv=1, S=128, D=64,
