@@ -1,6 +1,7 @@
 // attn_fwd.cuh -- forward kernel: O = softmax(scale * Q K^T, causal mask) V and
 // the per-row log-sum-exp.  Persistent: one CTA per SM walks a list of work
-// items, each 256 query rows of one (batch, query head).
+// items, each 256 query rows of one (batch, query head) (128 rows when items
+// of 256 would leave SMs idle).
 //
 // What it computes is the fused attention forward of the Axis page
 // (zyoralabs.com/axis, feature list: fused flash attention; bf16 storage, fp32
@@ -9,7 +10,9 @@
 //
 //   * a work item is two 128-row query tiles (Q0, Q1) of one (b, h); they
 //     share a ring of K tiles and a ring of V tiles (128 keys each) that two
-//     TMA threads stream in.  Items are dealt heaviest first (causal) in a
+//     TMA threads stream in.  When two-tile items would be fewer than the
+//     SMs, an item is one tile (Q1 absent, as for a ragged last block): twice
+//     the items and half the longest chain of kv tiles.  Items are dealt heaviest first (causal) in a
 //     snake order over the CTAs, which balances the causal triangle;
 //   * two threads issue the tcgen05.mma work, one S_t = Q_t K_j^T (both
 //     operands K-major in shared memory) into TMEM, the other O_t += P_t V_j
@@ -52,7 +55,8 @@ struct FwdArgs {
   float* lse;
   int B, Hq, Hkv, S;
   float scale_log2;  // scale * log2(e)
-  int n_qblocks;     // ceil(S / 256)
+  int tpi;           // 128-row query tiles per item: 2, or 1 when two-tile items cannot fill the SMs
+  int n_qblocks;     // ceil(S / (128 * tpi))
   int n_items;       // n_qblocks * B * Hq
 };
 
@@ -66,22 +70,23 @@ __device__ __forceinline__ int fwd_item(int it) {
 }
 
 struct FwdItem {
-  int b, h, bh, kvh, m;  // batch, head, b * Hq + h, kv head, query block (256 rows)
-  int n0, n1, nmax;      // kv tiles of query tile 0 / 1 (0: no tile 1), max
+  int b, h, bh, kvh, qt0;  // batch, head, b * Hq + h, kv head, first 128-row query tile
+  int n0, n1, nmax;        // kv tiles of query tile 0 / 1 (0: no tile 1), max
   bool has1;
 };
 
 __device__ __forceinline__ FwdItem fwd_decode(const FwdArgs& a, int w, bool causal) {
   FwdItem it;
   const int BH = a.B * a.Hq;
-  it.m = a.n_qblocks - 1 - w / BH;  // heaviest (last) query blocks first
+  const int m = a.n_qblocks - 1 - w / BH;  // heaviest (last) query blocks first
   it.bh = w % BH;
   it.b = it.bh / a.Hq;
   it.h = it.bh % a.Hq;
   it.kvh = it.h / (a.Hq / a.Hkv);
   const int nkv = (a.S + 127) / 128;
-  const int qt0 = 2 * it.m, qt1 = 2 * it.m + 1;
-  it.has1 = qt1 * 128 < a.S;
+  const int qt0 = a.tpi * m, qt1 = qt0 + 1;
+  it.qt0 = qt0;
+  it.has1 = a.tpi == 2 && qt1 * 128 < a.S;
   it.n0 = causal ? qt0 + 1 : nkv;
   it.n1 = it.has1 ? (causal ? qt1 + 1 : nkv) : 0;
   it.nmax = it.n1 > it.n0 ? it.n1 : it.n0;
@@ -299,10 +304,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           if (it > 0 && !mbar_wait_bounded<true>(bar_qempty, (it - 1) & 1, abort, F_QEMPTY)) break;
           mbar_arrive_expect_tx(bar_q, (I.has1 ? 2u : 1u) * TILE);
           for (int sl = 0; sl < C::NSLAB; ++sl)
-            tma_load_4d(sQ + sl * SLAB, &tm_q, bar_q, 64 * sl, I.h, 256 * I.m, I.b);
+            tma_load_4d(sQ + sl * SLAB, &tm_q, bar_q, 64 * sl, I.h, 128 * I.qt0, I.b);
           if (I.has1)
             for (int sl = 0; sl < C::NSLAB; ++sl)
-              tma_load_4d(sQ + TILE + sl * SLAB, &tm_q, bar_q, 64 * sl, I.h, 256 * I.m + 128, I.b);
+              tma_load_4d(sQ + TILE + sl * SLAB, &tm_q, bar_q, 64 * sl, I.h, 128 * I.qt0 + 128, I.b);
           ++nq;
           constexpr int PF = 4;
           auto prefetch = [&](int j) {
@@ -468,7 +473,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       if (w >= a.n_items) break;
       const FwdItem I = fwd_decode(a, w, CAUSAL);
       const int n_t = t == 0 ? I.n0 : I.n1;
-      const int qt = 2 * I.m + t;
+      const int qt = I.qt0 + t;
       const int row_g = qt * 128 + r;
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n_t; ++j, ++J, ++X) {

@@ -168,6 +168,11 @@ int launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& 
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
+// 0: always two query tiles per forward item.
+#ifndef AXIS_ATTN_FWD_SINGLE_TILE_ITEMS
+#define AXIS_ATTN_FWD_SINGLE_TILE_ITEMS 1
+#endif
+
 // The forward kernel over (q, k, v).
 int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int S, int D,
             float scale, int causal, cudaStream_t st, int dev) {
@@ -183,7 +188,10 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
   a.Hkv = Hkv;
   a.S = S;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
-  a.n_qblocks = (S + 255) / 256;
+  // two query tiles per item, unless that leaves SMs without an item: then
+  // one (twice the items, half the longest chain of kv tiles)
+  a.tpi = AXIS_ATTN_FWD_SINGLE_TILE_ITEMS && (long long)((S + 255) / 256) * B * Hq < sm_count(dev) ? 1 : 2;
+  a.n_qblocks = (S + 128 * a.tpi - 1) / (128 * a.tpi);
   a.n_items = a.n_qblocks * B * Hq;
   if (D == 64)
     return causal ? launch_fwd<64, true>(mq, mk, mv, a, st, dev) : launch_fwd<64, false>(mq, mk, mv, a, st, dev);
