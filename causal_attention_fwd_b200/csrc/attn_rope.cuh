@@ -37,29 +37,10 @@ __global__ void __launch_bounds__(256) rope_table_kernel(double2* __restrict__ c
   }
 }
 
-// fp64 -> bf16 bits, round to nearest even from the fp64 value itself (one
-// rounding: 45 mantissa bits dropped).  Values below the smallest normal bf16
-// flush to signed zero; the attention inputs never come near either end of
-// the range.
-__device__ __forceinline__ uint32_t f64_to_bf16_rn(double x) {
-  const unsigned long long u = (unsigned long long)__double_as_longlong(x);
-  const uint32_t sign = (uint32_t)(u >> 63) << 15;
-  int e = (int)((u >> 52) & 0x7ff) - 1023 + 127;
-  if (e <= 0) return sign;
-  unsigned long long keep = (u >> 45) & 0x7f;
-  const unsigned long long rest = u & ((1ull << 45) - 1), half = 1ull << 44;
-  if (rest > half || (rest == half && (keep & 1))) {
-    if (++keep == 0x80) {
-      keep = 0;
-      ++e;
-    }
-  }
-  if (e >= 255) return sign | 0x7f80u;
-  return sign | ((uint32_t)e << 7) | (uint32_t)keep;
-}
-
 // Rotate the 4 pairs of one 16-byte word (8 bf16) by table entries t[0..3]
-// (fp64), result correctly rounded to bf16.
+// (fp64), each result rounded once from fp64 to bf16 (round to nearest even:
+// CUDA's __double2bfloat16), so the stored value is the correctly rounded
+// rotation.
 __device__ __forceinline__ uint4 rope_rotate8_f64(uint4 x, const double2* __restrict__ t) {
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
   uint32_t o[4];
@@ -67,8 +48,8 @@ __device__ __forceinline__ uint4 rope_rotate8_f64(uint4 x, const double2* __rest
   for (int i = 0; i < 4; ++i) {
     const double2 cs = t[i];
     const double x0 = (double)__uint_as_float(w[i] << 16), x1 = (double)__uint_as_float(w[i] & 0xffff0000u);
-    const uint32_t y0 = f64_to_bf16_rn(fma(x0, cs.x, -x1 * cs.y));
-    const uint32_t y1 = f64_to_bf16_rn(fma(x0, cs.y, x1 * cs.x));
+    const uint32_t y0 = __bfloat16_as_ushort(__double2bfloat16(fma(x0, cs.x, -x1 * cs.y)));
+    const uint32_t y1 = __bfloat16_as_ushort(__double2bfloat16(fma(x0, cs.y, x1 * cs.x)));
     o[i] = y0 | (y1 << 16);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
@@ -82,41 +63,56 @@ __device__ __forceinline__ void rope_back(float& g0, float& g1, double2 cs) {
   g1 = b;
 }
 
-// y = R x for x, y [B, S, H, D] bf16 (in place allowed), one thread per
-// 16-byte word (4 pairs), grid-stride; HBM-bound (the table stays in L2).
+// The 16-byte words of [B, S, H, D] bf16 are walked position by position
+// (b, s): a position's H * D / 8 words are contiguous and share one row of the
+// table, so the position index costs one modulo per position, not three
+// 64-bit divisions per word.  A block takes ppb positions at a time (several
+// when a position has fewer words than the block has threads).
+struct RopeWalk {
+  int wpp, ppb;  // words per position, positions per block step
+  __device__ RopeWalk(int H, int D) : wpp(H * D / 8), ppb(wpp < (int)blockDim.x ? (int)blockDim.x / wpp : 1) {}
+};
+
+// y = R x for x, y [B, S, H, D] bf16 (in place allowed); HBM-bound (the table
+// stays in L2 / L1).
 __global__ void __launch_bounds__(256) rope_apply_kernel(const uint4* x, uint4* y, const double2* __restrict__ cs,
-                                                         long long n16, int S, int H, int D) {
-  const int w_per_row = D / 8;
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += stride) {
-    const long long row = i / w_per_row;  // (b * S + s) * H + h
-    const int wd = (int)(i % w_per_row);
-    const int s = (int)((row / H) % S);
-    y[i] = rope_rotate8_f64(x[i], cs + (size_t)s * (D / 2) + 4 * wd);
+                                                         long long npos, int S, int H, int D) {
+  const RopeWalk rw(H, D);
+  const int wpr = D / 8;  // words per head row (8 or 16)
+  const int sub = (int)threadIdx.x / rw.wpp, w0 = (int)threadIdx.x % rw.wpp;
+  if (sub >= rw.ppb) return;
+  for (long long p = (long long)blockIdx.x * rw.ppb + sub; p < npos; p += (long long)gridDim.x * rw.ppb) {
+    const double2* t = cs + (size_t)(p % S) * (D / 2);
+    const size_t base = (size_t)p * rw.wpp;
+    for (int w = w0; w < rw.wpp; w += rw.ppb == 1 ? (int)blockDim.x : rw.wpp)
+      y[base + w] = rope_rotate8_f64(x[base + w], t + 4 * (w & (wpr - 1)));
   }
 }
 
 // y = R^T x (the gradient direction), fp32 math, for the standalone call.
 __global__ void __launch_bounds__(256) rope_apply_back_kernel(const uint4* x, uint4* y,
-                                                              const double2* __restrict__ cs, long long n16, int S,
+                                                              const double2* __restrict__ cs, long long npos, int S,
                                                               int H, int D) {
-  const int w_per_row = D / 8;
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += stride) {
-    const long long row = i / w_per_row;
-    const int wd = (int)(i % w_per_row);
-    const int s = (int)((row / H) % S);
-    const double2* t = cs + (size_t)s * (D / 2) + 4 * wd;
-    const uint4 xv = x[i];
-    const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
-    uint32_t o[4];
+  const RopeWalk rw(H, D);
+  const int wpr = D / 8;
+  const int sub = (int)threadIdx.x / rw.wpp, w0 = (int)threadIdx.x % rw.wpp;
+  if (sub >= rw.ppb) return;
+  for (long long p = (long long)blockIdx.x * rw.ppb + sub; p < npos; p += (long long)gridDim.x * rw.ppb) {
+    const double2* tp = cs + (size_t)(p % S) * (D / 2);
+    const size_t base = (size_t)p * rw.wpp;
+    for (int w = w0; w < rw.wpp; w += rw.ppb == 1 ? (int)blockDim.x : rw.wpp) {
+      const double2* t = tp + 4 * (w & (wpr - 1));
+      const uint4 xv = x[base + w];
+      const uint32_t v[4] = {xv.x, xv.y, xv.z, xv.w};
+      uint32_t o[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float g0 = __uint_as_float(w[k] << 16), g1 = __uint_as_float(w[k] & 0xffff0000u);
-      rope_back(g0, g1, t[k]);
-      o[k] = pack_bf16x2(g0, g1);
+      for (int k = 0; k < 4; ++k) {
+        float g0 = __uint_as_float(v[k] << 16), g1 = __uint_as_float(v[k] & 0xffff0000u);
+        rope_back(g0, g1, t[k]);
+        o[k] = pack_bf16x2(g0, g1);
+      }
+      y[base + w] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    y[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 

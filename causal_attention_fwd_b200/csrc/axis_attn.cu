@@ -200,14 +200,17 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
 
 // y = R x (inverse: R^T x) for x, y [B, S, H, D] bf16 with the table cs [S][D/2].
 int run_rope(const void* x, void* y, const double* cs, int B, int S, int H, int D, int inverse, cudaStream_t st) {
-  const long long n16 = (long long)B * S * H * D / 8;
-  const unsigned grid = (unsigned)((n16 + 255) / 256 < 148 * 16 ? (n16 + 255) / 256 : 148 * 16);
+  const long long npos = (long long)B * S;
+  const int wpp = H * D / 8;
+  const long long ppb = wpp < 256 ? 256 / wpp : 1;  // positions per block step (RopeWalk)
+  const long long blocks = (npos + ppb - 1) / ppb;
+  const unsigned grid = (unsigned)(blocks < 148 * 8 ? blocks : 148 * 8);
   const auto* t = reinterpret_cast<const double2*>(cs);
   if (inverse)
-    rope_apply_back_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y), t, n16, S,
+    rope_apply_back_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y), t, npos, S,
                                                  H, D);
   else
-    rope_apply_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y), t, n16, S, H, D);
+    rope_apply_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y), t, npos, S, H, D);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
