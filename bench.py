@@ -568,11 +568,18 @@ def time_e2e(aa, w, prob, steps: int, det: bool, world: int, dev) -> dict:
     torch.cuda.synchronize()
     ems = reduce_max([e0.elapsed_time(e1)], world, dev)
     aa.check_status(s_comp)
+    # the results that came back to the host are the device step's own: O, LSE, dK, dV bit for bit
+    # (the same inputs, deterministic kernels), dQ to rounding (its fp32 additions arrive in any order)
+    dev_out = [prob.o, prob.lse, prob.dq, prob.dk, prob.dv]
+    same = all(torch.equal(h, d.cpu()) for i, (h, d) in enumerate(zip(hout, dev_out)) if i != 2)
+    dq_h, dq_d = hout[2].double(), dev_out[2].cpu().double()
+    dq_rel = float((dq_h - dq_d).norm() / dq_d.norm().clamp_min(1e-30))
     h2d = sum(t.numel() * t.element_size() for t in hin)
     d2h = sum(t.numel() * t.element_size() for t in hout)
     return {"value": whole_job_tflops(w.fwd_flops + w.bwd_flops, steps, ems[0], world), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "streams": "copy-in / compute / copy-out, two buffer sets"}
+            "streams": "copy-in / compute / copy-out, two buffer sets",
+            "verified": bool(same and dq_rel <= 1e-3), "dq_rel_to_device_step": dq_rel}
 
 
 def summarize(w, total_ms, stage_totals, steps, world, p_meas, det):
