@@ -85,7 +85,9 @@ __device__ __forceinline__ int dec_len(const DecArgs& a, int b) {
   return len;
 }
 
-// GM: the head group rounded up (2, 4 or 8); the kernel handles the first G.
+// GM: the head group (1, 2, 3 or 4 exactly; 5..8 rounded up to 8, the kernel
+// then handling the first G): every head costs the same score and P V work,
+// so a padded head is pure overhead.
 template <int HD, int GM>
 __global__ void __launch_bounds__(DEC_THREADS)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -211,13 +213,14 @@ __global__ void __launch_bounds__(DEC_THREADS)
     asm volatile("bar.sync 1, 128;" ::: "memory");
 
     constexpr int FPL = HD / 32;  // features per lane in O += p V
-    float m[GM], lsum[GM], acc_o[GM][FPL];
+    float m[GM], lsum[GM];
+    uint64_t acc_o[GM][FPL / 2];  // O of each head, packed feature pairs (fp32 x2)
 #pragma unroll
     for (int g = 0; g < GM; ++g) {
       m[g] = -INFINITY;
       lsum[g] = 0.f;
 #pragma unroll
-      for (int f = 0; f < FPL; ++f) acc_o[g][f] = 0.f;
+      for (int f = 0; f < FPL / 2; ++f) acc_o[g][f] = f2_pack(0.f, 0.f);
     }
     float* pw = p_s + cw * 32 * 8;
     bool ok = true;
@@ -265,11 +268,15 @@ __global__ void __launch_bounds__(DEC_THREADS)
           m[g] = m_new;
           lsum[g] = lsum[g] * alpha + p;
 #pragma unroll
-          for (int f = 0; f < FPL; ++f) acc_o[g][f] *= alpha;
+          for (int f = 0; f < FPL / 2; ++f) acc_o[g][f] = f2_mul(acc_o[g][f], f2_pack(alpha, alpha));
           pw[r * 8 + g] = p;
         }
         __syncwarp();
-        // ---- O += p V: lane = FPL consecutive features of every key row
+        // ---- O += p V: lane = FPL consecutive features of every key row (unrolled
+        // so that several rows' shared-memory loads are in flight at once; rows
+        // past the sequence's end are never read: they hold whatever the page
+        // pool holds there)
+#pragma unroll 4
         for (int rr = 0; rr < n_valid; ++rr) {
           const uint32_t byte = lane * FPL * 2;  // this lane's bytes in the row
           const uint32_t vaddr = sV + s * C::PIECE + (byte >> 7) * C::SLAB + rr * 128 +
@@ -288,11 +295,15 @@ __global__ void __launch_bounds__(DEC_THREADS)
             vf[0] = __uint_as_float(vx << 16);
             vf[1] = __uint_as_float(vx & 0xffff0000u);
           }
+          // the row's p of every head in one or two 16-byte loads
+          float pr[8];
+          *reinterpret_cast<float4*>(pr) = *reinterpret_cast<const float4*>(pw + rr * 8);
+          if constexpr (GM > 4) *reinterpret_cast<float4*>(pr + 4) = *reinterpret_cast<const float4*>(pw + rr * 8 + 4);
 #pragma unroll
           for (int g = 0; g < GM; ++g) {
-            const float p = pw[rr * 8 + g];
+            const uint64_t p2 = f2_pack(pr[g], pr[g]);
 #pragma unroll
-            for (int f = 0; f < FPL; ++f) acc_o[g][f] = fmaf(p, vf[f], acc_o[g][f]);
+            for (int f = 0; f < FPL / 2; ++f) acc_o[g][f] = f2_fma(p2, f2_pack(vf[2 * f], vf[2 * f + 1]), acc_o[g][f]);
           }
         }
       }
@@ -307,7 +318,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
       for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
       float* cs = c_s + (cw * 8 + g) * (HD + 2);
 #pragma unroll
-      for (int f = 0; f < FPL; ++f) cs[2 + lane * FPL + f] = acc_o[g][f];
+      for (int f = 0; f < FPL / 2; ++f) f2_unpack(acc_o[g][f], cs[2 + lane * FPL + 2 * f], cs[3 + lane * FPL + 2 * f]);
       if (lane == 0) {
         cs[0] = m[g];
         cs[1] = l;

@@ -651,8 +651,10 @@ int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a
 
 template <int HD>
 int launch_decode_g(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev) {
-  if (a.G <= 2) return launch_decode<HD, 2>(mk, mv, a, st, dev);
-  if (a.G <= 4) return launch_decode<HD, 4>(mk, mv, a, st, dev);
+  if (a.G == 1) return launch_decode<HD, 1>(mk, mv, a, st, dev);
+  if (a.G == 2) return launch_decode<HD, 2>(mk, mv, a, st, dev);
+  if (a.G == 3) return launch_decode<HD, 3>(mk, mv, a, st, dev);
+  if (a.G == 4) return launch_decode<HD, 4>(mk, mv, a, st, dev);
   return launch_decode<HD, 8>(mk, mv, a, st, dev);
 }
 
