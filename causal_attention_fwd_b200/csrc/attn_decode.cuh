@@ -11,22 +11,26 @@
 //
 // Design on sm_100a.  The step reads every cached key and value once and does
 // about 4 G flops per byte, far below the tensor cores' ridge, so it is
-// HBM-bound: the kernel is built to keep the memory system busy, not the MMA
-// units.
-//   * one CTA per (b, kv head, split of the sequence); a producer warp reads
-//     the block table 32 pieces ahead into shared memory and one of its
-//     threads streams 32-key pieces of the cache pages through TMA (a 3-D
-//     tensor map over the cache, 128B swizzle) into a ring of shared-memory
-//     stages, K and V of a piece on one mbarrier;
-//   * four compute warps take the pieces in turn (piece t -> warp t % 4) and
-//     keep their own running max, sum and O for the G query heads: scores with
-//     lane = key (q broadcast from shared memory, packed fp32 FMA), per-head
-//     max by warp shuffles, p = 2^(s - m) on the MUFU, then O += p V with
-//     lane = feature slice;
-//   * at the end the four warps' states are merged in shared memory; a split
-//     writes its unnormalised (m, l, O) to the workspace, which a second kernel
-//     merges (split-K over long sequences keeps every SM busy at small batch);
-//     with one split the CTA writes O and LSE itself.
+// HBM-bound: the kernel is built to keep the memory system busy.
+//   * persistent: as many CTAs as fit on the SMs walk the work items (b, kv
+//     head, split of the sequence); a producer warp reads the block table 32
+//     pieces ahead into shared memory and one of its threads streams 32-key
+//     pieces of the cache pages through TMA (a 3-D tensor map over the cache,
+//     128B swizzle) into a ring of shared-memory stages, K and V of a piece on
+//     one mbarrier, running ahead across item boundaries;
+//   * four compute warps take the pieces in turn and keep their own running
+//     max, sum and O for the G <= 8 query heads of the item.  The products
+//     run on the warp-level tensor-core MMA (m16n8k16, bf16 in, fp32 out),
+//     the heads as rows of a 16-row tile: S = Q K^T with K's fragments
+//     loaded straight from the swizzled rows (ldmatrix), the online softmax in
+//     the accumulator layout (a row's 32 keys in the 4 lanes of a quad), P
+//     kept in registers as the A operand of O += P V, V through the
+//     transposing load.  Per 8 KB piece that is about a tenth of the
+//     instructions of the same arithmetic on the CUDA cores;
+//   * at the end of an item the four warps' states are merged in shared
+//     memory; a split writes its unnormalised (m, l, O) to the workspace,
+//     which a second kernel merges (split-K over long sequences keeps every
+//     SM busy at small batch); with one split the CTA writes O and LSE itself.
 // Page indices and sequence lengths are device data: a page index outside
 // [0, num_pages) or a length outside [1, max_pages * page_size] is never used
 // for an access; it sets bit 1 of the device status word (reported by
@@ -61,9 +65,7 @@ struct DecCfg {
   static constexpr int NST = HD == 64 ? 8 : 4;          // ring stages (2 or 1 per compute warp)
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = NST * PIECE;
-  static constexpr uint32_t OFF_Q = 2 * NST * PIECE;              // fp32 [8][HD], pre-scaled
-  static constexpr uint32_t OFF_P = OFF_Q + 8 * HD * 4;           // fp32 [DEC_CW][32][8]
-  static constexpr uint32_t OFF_C = OFF_P + DEC_CW * 32 * 8 * 4;  // fp32 [DEC_CW][8][HD + 2]
+  static constexpr uint32_t OFF_C = 2 * NST * PIECE;              // fp32 [DEC_CW][8][HD + 2]
   static constexpr uint32_t OFF_FLAG = OFF_C + DEC_CW * 8 * (HD + 2) * 4;  // int [NST]: piece usable
   static constexpr uint32_t OFF_TBL = OFF_FLAG + NST * 4;                  // int [32][4]: pages of 32 pieces
   static constexpr uint32_t OFF_BAR = (OFF_TBL + 32 * 4 * 4 + 7) & ~7u;
@@ -73,22 +75,33 @@ struct DecCfg {
 
 enum DecSite { D_EMPTY = 41, D_FULL };
 
-// Sequence length of b, clamped to the valid range (an out-of-range value is
-// reported through the status word).
-__device__ __forceinline__ int dec_len(const DecArgs& a, int b) {
-  int len = a.seq_lens[b];
+// One work item: (b, kv head, split of the sequence), its key range and pieces.
+struct DecItem {
+  int b, kv, split, k0, k1, n_pieces;
+};
+__device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report) {
+  DecItem it;
+  it.split = w % a.n_splits;
+  const int bkv = w / a.n_splits;
+  it.b = bkv / a.Hkv;
+  it.kv = bkv % a.Hkv;
+  int len = a.seq_lens[it.b];
   const int cap = a.max_pages * a.page_size;
-  if (len < 1 || len > cap) {
-    atomicOr(&g_status, 2u);
+  if (len < 1 || len > cap) {  // clamped; reported once (by the producer)
+    if (report) atomicOr(&g_status, 2u);
     len = len < 1 ? 1 : cap;
   }
-  return len;
+  it.k0 = it.split * a.keys_per_split;
+  it.k1 = min(len, it.k0 + a.keys_per_split);
+  it.n_pieces = it.k1 > it.k0 ? (it.k1 - it.k0 + 31) / 32 : 0;
+  return it;
 }
 
-// GM: the head group (1, 2, 3 or 4 exactly; 5..8 rounded up to 8, the kernel
-// then handling the first G): every head costs the same score and P V work,
-// so a padded head is pure overhead.
-template <int HD, int GM>
+// Persistent: each CTA walks the items w = blockIdx.x, blockIdx.x + gridDim.x,
+// ...; the ring positions count pieces over all of its items, so the producer
+// streams the next item's pieces while the compute warps finish this one.
+// Compute warp (g mod 4) takes the CTA's g-th piece.
+template <int HD>
 __global__ void __launch_bounds__(DEC_THREADS)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const DecArgs a) {
@@ -99,8 +112,6 @@ __global__ void __launch_bounds__(DEC_THREADS)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
-  float* q_s = reinterpret_cast<float*>(gbase + C::OFF_Q);
-  float* p_s = reinterpret_cast<float*>(gbase + C::OFF_P);
   float* c_s = reinterpret_cast<float*>(gbase + C::OFF_C);
   volatile int* flag = reinterpret_cast<volatile int*>(gbase + C::OFF_FLAG);
   const uint32_t bars = base + C::OFF_BAR;
@@ -109,14 +120,8 @@ __global__ void __launch_bounds__(DEC_THREADS)
   volatile WaitCtl* ctl = reinterpret_cast<volatile WaitCtl*>(gbase + C::OFF_BAR + 16 * NST + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = (int)(blockIdx.x % a.n_splits);
-  const int bkv = (int)(blockIdx.x / a.n_splits);
-  const int b = bkv / a.Hkv, kv = bkv % a.Hkv;
+  const int n_items = a.B * a.Hkv * a.n_splits;
   const int G = a.G;
-  const int len = dec_len(a, b);
-  const int k0 = split * a.keys_per_split;
-  const int k1 = min(len, k0 + a.keys_per_split);
-  const int n_pieces = k1 > k0 ? (k1 - k0 + 31) / 32 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -134,37 +139,38 @@ __global__ void __launch_bounds__(DEC_THREADS)
     // into shared memory (32 independent loads instead of one dependent
     // global read per page in front of every copy); lane 0 then checks them
     // and issues the copies.
-    if (n_pieces > 0) {
-      int* tbl = reinterpret_cast<int*>(gbase + C::OFF_TBL);
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-      }
-      const int rows = a.page_size < 32 ? a.page_size : 32;  // rows per TMA box
-      const int nbox = 32 / rows;                              // boxes per 32-key piece
-      int issued = 0;
-      bool ok = true;
-      for (int t0 = 0; ok && t0 < n_pieces; t0 += 32) {
+    int* tbl = reinterpret_cast<int*>(gbase + C::OFF_TBL);
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
+    const int rows = a.page_size < 32 ? a.page_size : 32;  // rows per TMA box
+    const int nbox = 32 / rows;                              // boxes per 32-key piece
+    int g = 0;  // pieces issued (over all items)
+    bool ok = true;
+    for (int w = (int)blockIdx.x; ok && w < n_items; w += (int)gridDim.x) {
+      const DecItem I = dec_item(a, w, lane == 0);
+      for (int t0 = 0; ok && t0 < I.n_pieces; t0 += 32) {
         for (int e = lane; e < 32 * nbox; e += 32) {  // e = (t - t0) * nbox + x
-          const int t = t0 + e / nbox, key = k0 + 32 * t + (e % nbox) * rows;
-          tbl[e] = t < n_pieces && key < k1 ? a.block_table[(size_t)b * a.max_pages + key / a.page_size] : 0;
+          const int t = t0 + e / nbox, key = I.k0 + 32 * t + (e % nbox) * rows;
+          tbl[e] = t < I.n_pieces && key < I.k1 ? a.block_table[(size_t)I.b * a.max_pages + key / a.page_size] : 0;
         }
         __syncwarp();
         if (lane == 0) {
-          const int t1 = min(n_pieces, t0 + 32);
-          for (int t = t0; t < t1; ++t) {
-            const int s = t % NST;
-            if (t >= NST && !mbar_wait_bounded<true>(bar_empty(s), ((t / NST) & 1) ^ 1, ctl, D_EMPTY)) {
+          const int t1 = min(I.n_pieces, t0 + 32);
+          for (int t = t0; t < t1; ++t, ++g) {
+            const int s = g % NST;
+            if (g >= NST && !mbar_wait_bounded<true>(bar_empty(s), ((g / NST) & 1) ^ 1, ctl, D_EMPTY)) {
               ok = false;
               break;
             }
-            const int kt = k0 + 32 * t;
+            const int kt = I.k0 + 32 * t;
             // pages of this piece (at most 4: page_size >= 8), checked before any copy
             int usable = 1, nload = 0, pages[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
               const int key = kt + x * rows;
-              if (x < nbox && key < k1) {
+              if (x < nbox && key < I.k1) {
                 pages[x] = tbl[(t - t0) * nbox + x];
                 if (pages[x] < 0 || pages[x] >= a.num_pages) usable = 0;
                 ++nload;
@@ -184,177 +190,191 @@ __global__ void __launch_bounds__(DEC_THREADS)
 #pragma unroll
                 for (int sl = 0; sl < C::NSLAB; ++sl) {
                   const uint32_t off = s * C::PIECE + sl * C::SLAB + x * rows * 128;
-                  tma_load_3d(sK + off, &tm_k, bar_full(s), 64 * sl, kv, row);
-                  tma_load_3d(sV + off, &tm_v, bar_full(s), 64 * sl, kv, row);
+                  tma_load_3d(sK + off, &tm_k, bar_full(s), 64 * sl, I.kv, row);
+                  tma_load_3d(sV + off, &tm_v, bar_full(s), 64 * sl, I.kv, row);
                 }
               }
             }
-            issued = t + 1;
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
+        g = __shfl_sync(0xffffffffu, g, 0);
         __syncwarp();  // lane 0 is done with this block of table entries
       }
-      // drain: every copy started has landed before the CTA exits
-      if (lane == 0) {
-        volatile WaitCtl never = {0, 0, 0};
-        for (int t = issued - NST > 0 ? issued - NST : 0; t < issued; ++t)
-          mbar_wait_bounded<true>(bar_full(t % NST), (t / NST) & 1, &never, D_FULL);
-      }
+    }
+    // drain: every copy started has landed before the CTA exits
+    if (lane == 0) {
+      volatile WaitCtl never = {0, 0, 0};
+      for (int x = g - NST > 0 ? g - NST : 0; x < g; ++x)
+        mbar_wait_bounded<true>(bar_full(x % NST), (x / NST) & 1, &never, D_FULL);
     }
   } else {
     // ============================================================ compute warps
+    // Per 32-key piece: S (16 x 32) = Q K^T and O (16 x D) += P V on the
+    // warp-level MMA, the G <= 8 query heads as rows 0..G-1 of a 16-row tile
+    // (rows G..15 zero).  Lane l holds, in the accumulator layout, row
+    // g0 = l / 4 and the columns 2 (l % 4) + {0, 1} of every 8-column tile.
     const int cw = warp - 1;
-    // q of the group's G heads -> shared memory, fp32, pre-scaled to log2 units
-    for (int x = threadIdx.x - 32; x < GM * HD; x += DEC_CW * 32) {
-      const int g = x / HD;
-      q_s[x] = g < G ? __bfloat162float(a.q[((size_t)b * a.Hq + kv * G + g) * HD + x % HD]) * a.scale_log2 : 0.f;
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-
-    constexpr int FPL = HD / 32;  // features per lane in O += p V
-    float m[GM], lsum[GM];
-    uint64_t acc_o[GM][FPL / 2];  // O of each head, packed feature pairs (fp32 x2)
-#pragma unroll
-    for (int g = 0; g < GM; ++g) {
-      m[g] = -INFINITY;
-      lsum[g] = 0.f;
-#pragma unroll
-      for (int f = 0; f < FPL / 2; ++f) acc_o[g][f] = f2_pack(0.f, 0.f);
-    }
-    float* pw = p_s + cw * 32 * 8;
+    const float c = a.scale_log2;
+    constexpr int KS = HD / 16;  // k-steps of the score product (features)
+    constexpr int ND = HD / 8;   // 8-feature column tiles of O
+    constexpr int FPL = HD / 32;  // features per lane in the merge
+    const int g0 = lane >> 2, q2 = 2 * (lane & 3);
+    int gbase_item = 0;  // pieces of this CTA's earlier items
     bool ok = true;
-    for (int t = cw; ok && t < n_pieces; t += DEC_CW) {
-      const int s = t % NST;
-      if (!wait_warp<true>(bar_full(s), (t / NST) & 1, ctl, D_FULL)) { ok = false; break; }
-      const int n_valid = min(32, k1 - (k0 + 32 * t));
-      if (flag[s]) {
-        // ---- scores: lane = key row of the piece
-        const int r = lane;
-        uint64_t sc2[GM];
+    // Every compute warp walks every item, also after a wait has given up
+    // (its later waits then return at once: the CTA's abort flag is set), so
+    // that all four reach each of the named barriers below.
+    for (int w = (int)blockIdx.x; w < n_items; w += (int)gridDim.x) {
+      const DecItem I = dec_item(a, w, false);
+      // Q as A fragments: (row g0, columns 16 ks + q2 + {0,1}) and (+8); the
+      // fragments of rows 8..15 are zero
+      uint32_t qa[KS][2];
 #pragma unroll
-        for (int g = 0; g < GM; ++g) sc2[g] = f2_pack(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < HD / 8; ++c) {
-          const uint32_t addr = sK + s * C::PIECE + (c >> 3) * C::SLAB + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-          uint32_t kx, ky, kz, kw;
-          asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(kx), "=r"(ky), "=r"(kz), "=r"(kw) : "r"(addr));
-          const uint64_t k01 = f2_pack(__uint_as_float(kx << 16), __uint_as_float(kx & 0xffff0000u));
-          const uint64_t k23 = f2_pack(__uint_as_float(ky << 16), __uint_as_float(ky & 0xffff0000u));
-          const uint64_t k45 = f2_pack(__uint_as_float(kz << 16), __uint_as_float(kz & 0xffff0000u));
-          const uint64_t k67 = f2_pack(__uint_as_float(kw << 16), __uint_as_float(kw & 0xffff0000u));
-#pragma unroll
-          for (int g = 0; g < GM; ++g) {
-            const float4 qa = *reinterpret_cast<const float4*>(q_s + g * HD + 8 * c);
-            const float4 qb = *reinterpret_cast<const float4*>(q_s + g * HD + 8 * c + 4);
-            sc2[g] = f2_fma(f2_pack(qa.x, qa.y), k01, sc2[g]);
-            sc2[g] = f2_fma(f2_pack(qa.z, qa.w), k23, sc2[g]);
-            sc2[g] = f2_fma(f2_pack(qb.x, qb.y), k45, sc2[g]);
-            sc2[g] = f2_fma(f2_pack(qb.z, qb.w), k67, sc2[g]);
-          }
+      for (int ks = 0; ks < KS; ++ks) {
+        qa[ks][0] = qa[ks][1] = 0u;
+        if (g0 < G) {
+          const __nv_bfloat16* qrow = a.q + ((size_t)I.b * a.Hq + I.kv * G + g0) * HD + 16 * ks + q2;
+          qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow);
+          qa[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 8);
         }
-        // ---- online softmax per head (log2 domain)
+      }
+      float o_acc[ND][4];
 #pragma unroll
-        for (int g = 0; g < GM; ++g) {
-          float lo, hi;
-          f2_unpack(sc2[g], lo, hi);
-          const float sv = r < n_valid ? lo + hi : -INFINITY;
-          float mx = sv;
+      for (int nd = 0; nd < ND; ++nd) o_acc[nd][0] = o_acc[nd][1] = o_acc[nd][2] = o_acc[nd][3] = 0.f;
+      float m_run = -INFINITY, l_part = 0.f;  // row g0: running max (log2 units), this lane's share of the sum
+      // this warp's pieces of the item: the CTA's piece gbase_item + t goes to warp (gbase_item + t) % 4
+      for (int t = (cw - gbase_item % DEC_CW + DEC_CW) % DEC_CW; ok && t < I.n_pieces; t += DEC_CW) {
+        const int gp = gbase_item + t;
+        const int s = gp % NST;
+        if (!wait_warp<true>(bar_full(s), (gp / NST) & 1, ctl, D_FULL)) { ok = false; break; }
+        const int n_valid = min(32, I.k1 - (I.k0 + 32 * t));
+        if (flag[s]) {
+          const uint32_t kb = sK + s * C::PIECE, vb = sV + s * C::PIECE;
+          // rows past the sequence's end hold whatever the page pool holds there:
+          // zero their V (a 0 weight times a NaN would still be NaN in the MMA)
+          if (n_valid < 32) {
+            for (int x = lane; x < (32 - n_valid) * (HD / 8); x += 32) {
+              const int key = n_valid + x / (HD / 8), ch = x % (HD / 8);
+              const uint32_t addr = vb + (ch >> 3) * C::SLAB + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(addr), "r"(0u) : "memory");
+            }
+            __syncwarp();
+          }
+          // ---- S = Q K^T: 4 tiles of 8 keys; B fragments straight from the swizzled K rows
+          float sc[4][4];
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-          const float m_new = fmaxf(m[g], mx);
-          const float alpha = ex2_approx(m[g] - m_new);  // 0 on the first piece (m = -inf)
-          const float p = ex2_approx(sv - m_new);        // masked keys: 0
-          m[g] = m_new;
-          lsum[g] = lsum[g] * alpha + p;
+          for (int nt = 0; nt < 4; ++nt) {
+            sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
-          for (int f = 0; f < FPL / 2; ++f) acc_o[g][f] = f2_mul(acc_o[g][f], f2_pack(alpha, alpha));
-          pw[r * 8 + g] = p;
+            for (int k2 = 0; k2 < KS / 2; ++k2) {
+              // matrix lane / 8: features 32 k2 + 8 (lane / 8) .. + 7 of key 8 nt + lane % 8
+              const int key = 8 * nt + (lane & 7), f0 = 32 * k2 + 8 * (lane >> 3);
+              uint32_t bk[4];
+              ldsm_x4(kb + (f0 >> 6) * C::SLAB + key * 128 + ((((f0 & 63) >> 3) ^ (key & 7)) << 4), bk);
+              mma_16816(sc[nt], qa[2 * k2][0], 0u, qa[2 * k2][1], 0u, bk[0], bk[1]);
+              mma_16816(sc[nt], qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u, bk[2], bk[3]);
+            }
+          }
+          // ---- online softmax of row g0 (the 4 lanes of a quad hold its 32 keys)
+          float mx = -INFINITY;
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              if (8 * nt + q2 + e >= n_valid) sc[nt][e] = -INFINITY;
+              mx = fmaxf(mx, sc[nt][e]);
+            }
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          const float m_new = fmaxf(m_run, mx * c);
+          if (m_new > m_run + 8.0f) {  // the running max moves only by more than 8 (a factor 256)
+            const float alpha = ex2_approx(m_run - m_new);  // 0 on the first piece
+            m_run = m_new;
+            l_part *= alpha;
+#pragma unroll
+            for (int nd = 0; nd < ND; ++nd) {
+              o_acc[nd][0] *= alpha;
+              o_acc[nd][1] *= alpha;
+            }
+          }
+          // p = 2^(s c - m); bf16 P as the A fragments of P V: k-step k2 takes the
+          // key tiles 2 k2 (columns 0..7) and 2 k2 + 1 (columns 8..15)
+          uint32_t pa[4];
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+            const float p0 = ex2_approx(fmaf(sc[nt][0], c, -m_run));
+            const float p1 = ex2_approx(fmaf(sc[nt][1], c, -m_run));
+            l_part += p0 + p1;
+            pa[nt] = pack_bf16x2(p0, p1);
+          }
+          // ---- O += P V: B fragments of V (rows = keys) through the transposing load
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2)
+#pragma unroll
+            for (int n2 = 0; n2 < ND / 2; ++n2) {
+              // matrix lane / 8: keys 16 k2 + 8 ((lane / 8) & 1) .., features 16 n2 + 8 (lane / 16)
+              const int key = 16 * k2 + 8 * ((lane >> 3) & 1) + (lane & 7), f0 = 16 * n2 + 8 * (lane >> 4);
+              uint32_t bv[4];
+              ldsm_x4_t(vb + (f0 >> 6) * C::SLAB + key * 128 + ((((f0 & 63) >> 3) ^ (key & 7)) << 4), bv);
+              mma_16816(o_acc[2 * n2], pa[2 * k2], 0u, pa[2 * k2 + 1], 0u, bv[0], bv[1]);
+              mma_16816(o_acc[2 * n2 + 1], pa[2 * k2], 0u, pa[2 * k2 + 1], 0u, bv[2], bv[3]);
+            }
         }
         __syncwarp();
-        // ---- O += p V: lane = FPL consecutive features of every key row (unrolled
-        // so that several rows' shared-memory loads are in flight at once; rows
-        // past the sequence's end are never read: they hold whatever the page
-        // pool holds there)
-#pragma unroll 4
-        for (int rr = 0; rr < n_valid; ++rr) {
-          const uint32_t byte = lane * FPL * 2;  // this lane's bytes in the row
-          const uint32_t vaddr = sV + s * C::PIECE + (byte >> 7) * C::SLAB + rr * 128 +
-                                 ((((byte & 127) >> 4) ^ (rr & 7)) << 4) + (byte & 15);
-          float vf[FPL];
-          if constexpr (FPL == 4) {
-            uint32_t vx, vy;
-            asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(vx), "=r"(vy) : "r"(vaddr));
-            vf[0] = __uint_as_float(vx << 16);
-            vf[1] = __uint_as_float(vx & 0xffff0000u);
-            vf[2] = __uint_as_float(vy << 16);
-            vf[3] = __uint_as_float(vy & 0xffff0000u);
-          } else {
-            uint32_t vx;
-            asm volatile("ld.shared.b32 %0, [%1];" : "=r"(vx) : "r"(vaddr));
-            vf[0] = __uint_as_float(vx << 16);
-            vf[1] = __uint_as_float(vx & 0xffff0000u);
-          }
-          // the row's p of every head in one or two 16-byte loads
-          float pr[8];
-          *reinterpret_cast<float4*>(pr) = *reinterpret_cast<const float4*>(pw + rr * 8);
-          if constexpr (GM > 4) *reinterpret_cast<float4*>(pr + 4) = *reinterpret_cast<const float4*>(pw + rr * 8 + 4);
+        if (lane == 0) mbar_arrive(bar_empty(s));
+      }
+      gbase_item += I.n_pieces;
+      // ---- this warp's (m, l, O) of each head, then the merge of the four warps
+      float l = l_part;
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      if (g0 < G) {
+        float* cs = c_s + (cw * 8 + g0) * (HD + 2);
 #pragma unroll
-          for (int g = 0; g < GM; ++g) {
-            const uint64_t p2 = f2_pack(pr[g], pr[g]);
+        for (int nd = 0; nd < ND; ++nd) {
+          cs[2 + 8 * nd + q2] = o_acc[nd][0];
+          cs[3 + 8 * nd + q2] = o_acc[nd][1];
+        }
+        if ((lane & 3) == 0) {
+          cs[0] = m_run;
+          cs[1] = l;
+        }
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int g = cw; g < G; g += DEC_CW) {
+        float mm = -INFINITY;
 #pragma unroll
-            for (int f = 0; f < FPL / 2; ++f) acc_o[g][f] = f2_fma(p2, f2_pack(vf[2 * f], vf[2 * f + 1]), acc_o[g][f]);
+        for (int x = 0; x < DEC_CW; ++x) mm = fmaxf(mm, c_s[(x * 8 + g) * (HD + 2)]);
+        float lt = 0.f, ov[FPL];
+#pragma unroll
+        for (int f = 0; f < FPL; ++f) ov[f] = 0.f;
+#pragma unroll
+        for (int x = 0; x < DEC_CW; ++x) {
+          const float* cs = c_s + (x * 8 + g) * (HD + 2);
+          const float e = cs[1] > 0.f ? ex2_approx(cs[0] - mm) : 0.f;  // warps without keys weigh 0
+          lt += cs[1] * e;
+#pragma unroll
+          for (int f = 0; f < FPL; ++f) ov[f] += cs[2 + lane * FPL + f] * e;
+        }
+        const int bh = I.b * a.Hq + I.kv * G + g;
+        if (a.n_splits == 1) {
+          const float inv = lt > 0.f ? 1.f / lt : 0.f;
+#pragma unroll
+          for (int f = 0; f < FPL; ++f) a.o[(size_t)bh * HD + lane * FPL + f] = __float2bfloat16_rn(ov[f] * inv);
+          if (lane == 0) a.lse[bh] = (mm + __log2f(lt)) * 0.69314718055994531f;
+        } else {
+          float* dst = a.part + ((size_t)bh * a.n_splits + I.split) * (HD + 2);
+#pragma unroll
+          for (int f = 0; f < FPL; ++f) dst[2 + lane * FPL + f] = ov[f];
+          if (lane == 0) {
+            dst[0] = mm;
+            dst[1] = lt;
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_empty(s));
-    }
-    // ---- merge the four warps' states, then write the split's result
-#pragma unroll
-    for (int g = 0; g < GM; ++g) {
-      float l = lsum[g];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-      float* cs = c_s + (cw * 8 + g) * (HD + 2);
-#pragma unroll
-      for (int f = 0; f < FPL / 2; ++f) f2_unpack(acc_o[g][f], cs[2 + lane * FPL + 2 * f], cs[3 + lane * FPL + 2 * f]);
-      if (lane == 0) {
-        cs[0] = m[g];
-        cs[1] = l;
-      }
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    for (int g = cw; g < G; g += DEC_CW) {
-      float mm = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < DEC_CW; ++w) mm = fmaxf(mm, c_s[(w * 8 + g) * (HD + 2)]);
-      float l = 0.f, ov[FPL];
-#pragma unroll
-      for (int f = 0; f < FPL; ++f) ov[f] = 0.f;
-#pragma unroll
-      for (int w = 0; w < DEC_CW; ++w) {
-        const float* cs = c_s + (w * 8 + g) * (HD + 2);
-        const float e = cs[1] > 0.f ? ex2_approx(cs[0] - mm) : 0.f;  // warps without keys weigh 0
-        l += cs[1] * e;
-#pragma unroll
-        for (int f = 0; f < FPL; ++f) ov[f] += cs[2 + lane * FPL + f] * e;
-      }
-      const int bh = b * a.Hq + kv * G + g;
-      if (a.n_splits == 1) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-        for (int f = 0; f < FPL; ++f) a.o[(size_t)bh * HD + lane * FPL + f] = __float2bfloat16_rn(ov[f] * inv);
-        if (lane == 0) a.lse[bh] = (mm + __log2f(l)) * 0.69314718055994531f;
-      } else {
-        float* dst = a.part + ((size_t)bh * a.n_splits + split) * (HD + 2);
-#pragma unroll
-        for (int f = 0; f < FPL; ++f) dst[2 + lane * FPL + f] = ov[f];
-        if (lane == 0) {
-          dst[0] = mm;
-          dst[1] = l;
-        }
-      }
+      // the merge has read every warp's share before the next item's are written
+      asm volatile("bar.sync 1, 128;" ::: "memory");
     }
   }
 }

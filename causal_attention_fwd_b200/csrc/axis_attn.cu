@@ -639,23 +639,24 @@ bool make_cache_map(CUtensorMap* map, const void* ptr, int rows, int Hkv, int D,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int HD, int GM>
+// Persistent decode: as many CTAs as fit on the SMs at once (or one per item).
+template <int HD>
 int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev) {
-  auto kern = attn_decode_kernel<HD, GM>;
+  auto kern = attn_decode_kernel<HD>;
   static bool done[64];
+  static int per_sm[64];
   if (int rc = set_smem(kern, DecCfg<HD>::SMEM, dev, done)) return rc;
-  const unsigned grid = (unsigned)(a.B * a.Hkv * a.n_splits);
+  if (per_sm[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, DEC_THREADS, DecCfg<HD>::SMEM) != cudaSuccess || n < 1)
+      n = 1;
+    per_sm[dev] = n;
+  }
+  const long long items = (long long)a.B * a.Hkv * a.n_splits;
+  const long long cap = (long long)per_sm[dev] * sm_count(dev);
+  const unsigned grid = (unsigned)(items < cap ? items : cap);
   kern<<<grid, DEC_THREADS, DecCfg<HD>::SMEM, st>>>(mk, mv, a);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
-}
-
-template <int HD>
-int launch_decode_g(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev) {
-  if (a.G == 1) return launch_decode<HD, 1>(mk, mv, a, st, dev);
-  if (a.G == 2) return launch_decode<HD, 2>(mk, mv, a, st, dev);
-  if (a.G == 3) return launch_decode<HD, 3>(mk, mv, a, st, dev);
-  if (a.G == 4) return launch_decode<HD, 4>(mk, mv, a, st, dev);
-  return launch_decode<HD, 8>(mk, mv, a, st, dev);
 }
 
 }  // namespace
@@ -704,7 +705,7 @@ extern "C" int axis_attn_decode(const void* q, const void* k_cache, const void* 
   a.n_splits = sp.n_splits;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int rc = D == 64 ? launch_decode_g<64>(mk, mv, a, st, dev) : launch_decode_g<128>(mk, mv, a, st, dev);
+  int rc = D == 64 ? launch_decode<64>(mk, mv, a, st, dev) : launch_decode<128>(mk, mv, a, st, dev);
   if (rc || sp.n_splits == 1) return rc;
   const int rows = B * Hq;
   const unsigned grid = (unsigned)((rows + 7) / 8 < 4096 ? (rows + 7) / 8 : 4096);
