@@ -11,11 +11,16 @@ Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
 The headline workload (default llm1b, B=4 S=2048 Hq=32 Hkv=8 D=64) gives the
 line's value, roofline, e2e and cpu_baseline; the other four workloads are
 timed after it the same way (fewer steps) and reported under "workloads", each
-with its own clocks and oracle baseline.  Under torchrun (N > 1) every rank
-runs its own batch of each workload (weak scaling; no collective on the data
-path).  Timing: CUDA events around each step on the launching stream, L2
-flushed (256 MiB write) before every step, outside the events; the reported
-time is the max over ranks.  Rank 0 prints one JSON line.
+with its own clocks and oracle baseline; "rope" times the headline step with
+the rotary embedding fused, "decode" two decode steps against a paged KV cache
+(HBM roofline).  "e2e" is the same step from pinned host memory through the
+public torch helpers, uploads and downloads inside the timed region, pipelined
+over three streams, its results checked against the device step's.  Under
+torchrun (N > 1) every rank runs its own batch of each workload (weak scaling;
+no collective on the data path), or with --shard one problem's (b, kv) units.
+Timing: CUDA events around each step on the launching stream, L2 flushed (256
+MiB write) before every step, outside the events; the reported time is the max
+over ranks.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
