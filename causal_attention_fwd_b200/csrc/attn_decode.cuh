@@ -54,19 +54,31 @@ struct DecArgs {
   float scale_log2;        // scale * log2(e)
 };
 
-constexpr int DEC_THREADS = 160;  // warp 0: producer; warps 1-4: compute
-constexpr int DEC_CW = 4;         // compute warps
+// Compute warps per CTA at head dim 64 / 128 (warp 0 is the producer).
+#ifndef AXIS_ATTN_DEC_CW64
+#define AXIS_ATTN_DEC_CW64 4
+#endif
+#ifndef AXIS_ATTN_DEC_NST64
+#define AXIS_ATTN_DEC_NST64 8
+#endif
 
 template <int HD>
 struct DecCfg {
   static constexpr int NSLAB = HD / 64;
   static constexpr uint32_t SLAB = 32 * 128;            // 32 rows x 128 bytes
   static constexpr uint32_t PIECE = NSLAB * SLAB;       // 32 keys x HD bf16
-  static constexpr int NST = HD == 64 ? 8 : 4;          // ring stages (2 or 1 per compute warp)
+  static constexpr int CW = HD == 64 ? AXIS_ATTN_DEC_CW64 : 4;  // compute warps
+  static constexpr int THREADS = 32 * (1 + CW);
+  static constexpr int NST = HD == 64 ? AXIS_ATTN_DEC_NST64 : 4;  // ring stages
+  // A compute warp waits on the phase of a stage only after the stage's
+  // previous phase has completed (a parity wait cannot tell phase k from
+  // phase k - 2): the previous piece in a stage must be the same warp's,
+  // which holds when the ring depth is a multiple of the warp count.
+  static_assert(NST % CW == 0, "ring depth must be a multiple of the compute warps");
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = NST * PIECE;
-  static constexpr uint32_t OFF_C = 2 * NST * PIECE;              // fp32 [DEC_CW][8][HD + 2]
-  static constexpr uint32_t OFF_FLAG = OFF_C + DEC_CW * 8 * (HD + 2) * 4;  // int [NST]: piece usable
+  static constexpr uint32_t OFF_C = 2 * NST * PIECE;              // fp32 [CW][8][HD + 2]
+  static constexpr uint32_t OFF_FLAG = OFF_C + CW * 8 * (HD + 2) * 4;  // int [NST]: piece usable
   static constexpr uint32_t OFF_TBL = OFF_FLAG + NST * 4;                  // int [32][4]: pages of 32 pieces
   static constexpr uint32_t OFF_BAR = (OFF_TBL + 32 * 4 * 4 + 7) & ~7u;
   static constexpr uint32_t SMEM = OFF_BAR + 8 * 2 * NST + 16 + 1024;
@@ -102,11 +114,11 @@ __device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report
 // streams the next item's pieces while the compute warps finish this one.
 // Compute warp (g mod 4) takes the CTA's g-th piece.
 template <int HD>
-__global__ void __launch_bounds__(DEC_THREADS)
+__global__ void __launch_bounds__(DecCfg<HD>::THREADS)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const DecArgs a) {
   using C = DecCfg<HD>;
-  constexpr int NST = C::NST;
+  constexpr int NST = C::NST, CW = C::CW;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -244,7 +256,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
       for (int nd = 0; nd < ND; ++nd) o_acc[nd][0] = o_acc[nd][1] = o_acc[nd][2] = o_acc[nd][3] = 0.f;
       float m_run = -INFINITY, l_part = 0.f;  // row g0: running max (log2 units), this lane's share of the sum
       // this warp's pieces of the item: the CTA's piece gbase_item + t goes to warp (gbase_item + t) % 4
-      for (int t = (cw - gbase_item % DEC_CW + DEC_CW) % DEC_CW; ok && t < I.n_pieces; t += DEC_CW) {
+      for (int t = (cw - gbase_item % CW + CW) % CW; ok && t < I.n_pieces; t += CW) {
         const int gp = gbase_item + t;
         const int s = gp % NST;
         if (!wait_warp<true>(bar_full(s), (gp / NST) & 1, ctl, D_FULL)) { ok = false; break; }
@@ -341,16 +353,16 @@ __global__ void __launch_bounds__(DEC_THREADS)
           cs[1] = l;
         }
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      for (int g = cw; g < G; g += DEC_CW) {
+      named_bar_sync(1, 32 * CW);
+      for (int g = cw; g < G; g += CW) {
         float mm = -INFINITY;
 #pragma unroll
-        for (int x = 0; x < DEC_CW; ++x) mm = fmaxf(mm, c_s[(x * 8 + g) * (HD + 2)]);
+        for (int x = 0; x < CW; ++x) mm = fmaxf(mm, c_s[(x * 8 + g) * (HD + 2)]);
         float lt = 0.f, ov[FPL];
 #pragma unroll
         for (int f = 0; f < FPL; ++f) ov[f] = 0.f;
 #pragma unroll
-        for (int x = 0; x < DEC_CW; ++x) {
+        for (int x = 0; x < CW; ++x) {
           const float* cs = c_s + (x * 8 + g) * (HD + 2);
           const float e = cs[1] > 0.f ? ex2_approx(cs[0] - mm) : 0.f;  // warps without keys weigh 0
           lt += cs[1] * e;
@@ -374,7 +386,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
         }
       }
       // the merge has read every warp's share before the next item's are written
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      named_bar_sync(1, 32 * CW);
     }
   }
 }

@@ -648,14 +648,14 @@ int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a
   if (int rc = set_smem(kern, DecCfg<HD>::SMEM, dev, done)) return rc;
   if (per_sm[dev] == 0) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, DEC_THREADS, DecCfg<HD>::SMEM) != cudaSuccess || n < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, DecCfg<HD>::THREADS, DecCfg<HD>::SMEM) != cudaSuccess || n < 1)
       n = 1;
     per_sm[dev] = n;
   }
   const long long items = (long long)a.B * a.Hkv * a.n_splits;
   const long long cap = (long long)per_sm[dev] * sm_count(dev);
   const unsigned grid = (unsigned)(items < cap ? items : cap);
-  kern<<<grid, DEC_THREADS, DecCfg<HD>::SMEM, st>>>(mk, mv, a);
+  kern<<<grid, DecCfg<HD>::THREADS, DecCfg<HD>::SMEM, st>>>(mk, mv, a);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 

@@ -392,6 +392,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
 }
 
 // ------------------------------------------------------------- arithmetic
+// Named barrier `id` over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Warp-level MMA (m16n8k16, bf16 in, fp32 accumulate) and its 8x8 matrix
 // loads from shared memory: for the small decode products, where G <= 8 query
 // rows would fill a tcgen05 tile to a few percent.
