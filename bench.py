@@ -480,13 +480,23 @@ def time_decode(aa, name, dev, steps, flush, hbm_gbs):
     need = aa.axis_attn_decode_workspace_bytes(B, Hq, Hkv, D, page, max_pages)
     ws = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
     st = torch.cuda.current_stream(dev)
+    import ctypes
+
+    sp = ctypes.c_void_p(st.cuda_stream)
+    # the C ABI straight (as the main step does): the torch helper's checks would run on the host
+    # between the events while the GPU waits, and count as device time
+    args = (q.data_ptr(), kc.data_ptr(), vc.data_ptr(), table.data_ptr(), lens.data_ptr(), o.data_ptr(),
+            lse.data_ptr(), B, Hq, Hkv, D, page, max_pages, num_pages, 1.0 / math.sqrt(D), ws.data_ptr(),
+            ws.numel(), sp)
     ev = []
     for n in range(3 + steps):
         flush.fill_(n & 0xFF)
         e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         e[0].record(st)
-        aa.attention_decode(q, kc, vc, table, lens, out=o, lse=lse, workspace=ws)
+        rc = aa.axis_attn_decode(*args)
         e[1].record(st)
+        if rc:
+            raise aa.AxisAttnError(rc, "axis_attn_decode")
         if n >= 3:
             ev.append(e)
     torch.cuda.synchronize()
