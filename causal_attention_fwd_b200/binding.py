@@ -35,6 +35,7 @@ EXPORTS = (
     "axis_attn_bwd_rope",
     "axis_attn_decode_workspace_bytes",
     "axis_attn_decode",
+    "axis_attn_decode_hnd",
     "axis_attn_get_status",
     "axis_attn_last_status_word",
     "axis_attn_strerror",
@@ -109,6 +110,8 @@ def load():
             lib.axis_attn_decode_workspace_bytes.restype = sz
             lib.axis_attn_decode.argtypes = [vp] * 7 + [i] * 7 + [f, vp, sz, vp]
             lib.axis_attn_decode.restype = i
+            lib.axis_attn_decode_hnd.argtypes = [vp] * 7 + [i] * 7 + [f, vp, sz, vp]
+            lib.axis_attn_decode_hnd.restype = i
             lib.axis_attn_get_status.argtypes = [vp]
             lib.axis_attn_get_status.restype = i
             lib.axis_attn_last_status_word.argtypes = []
@@ -199,6 +202,13 @@ def axis_attn_decode(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, 
     """Decode step against a paged KV cache (see include/axis_attn.h)."""
     return load().axis_attn_decode(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
                                    max_pages, num_pages, scale, workspace, workspace_bytes, stream)
+
+
+def axis_attn_decode_hnd(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size, max_pages,
+                         num_pages, scale, workspace, workspace_bytes, stream) -> int:
+    """Decode step against a head-major paged KV cache (see include/axis_attn.h)."""
+    return load().axis_attn_decode_hnd(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
+                                       max_pages, num_pages, scale, workspace, workspace_bytes, stream)
 
 
 def axis_attn_get_status(stream) -> int:
@@ -414,21 +424,30 @@ def attention_backward_rope(q_rot, k_rot, v, cs, o, lse, dout, causal: bool = Tr
 
 
 def attention_decode(q, k_cache, v_cache, block_table, seq_lens, scale: float | None = None, out=None,
-                     lse=None, workspace=None, stream=None):
+                     lse=None, workspace=None, stream=None, layout: str = "NHD"):
     """Decode step: q [B, Hq, D] bf16, k_cache / v_cache [num_pages, page_size,
-    Hkv, D] bf16, block_table [B, max_pages] int32, seq_lens [B] int32, all on
-    one CUDA device.  Returns (o [B, Hq, D] bf16, lse [B, Hq] fp32)."""
+    Hkv, D] bf16 (layout "NHD") or [num_pages, Hkv, page_size, D] (layout
+    "HND"), block_table [B, max_pages] int32, seq_lens [B] int32, all on one
+    CUDA device.  Returns (o [B, Hq, D] bf16, lse [B, Hq] fp32)."""
     import torch
 
     where = "attention_decode"
+    _require(layout in ("NHD", "HND"), ERR_SHAPE, where, "layout must be 'NHD' or 'HND'")
+    hnd = layout == "HND"
+    dims = "[num_pages, Hkv, page_size, D]" if hnd else "[num_pages, page_size, Hkv, D]"
     _require(isinstance(q, torch.Tensor) and q.dim() == 3, ERR_SHAPE, where, "q must be a 3-D tensor [B, Hq, D]")
     _require(isinstance(k_cache, torch.Tensor) and k_cache.dim() == 4, ERR_SHAPE, where,
-             "k_cache must be a 4-D tensor [num_pages, page_size, Hkv, D]")
+             f"k_cache must be a 4-D tensor {dims}")
     B, Hq, D = q.shape
-    num_pages, page_size, Hkv, _ = k_cache.shape
+    if hnd:
+        num_pages, Hkv, page_size, _ = k_cache.shape
+        cache_shape = (num_pages, Hkv, page_size, D)
+    else:
+        num_pages, page_size, Hkv, _ = k_cache.shape
+        cache_shape = (num_pages, page_size, Hkv, D)
     _check_tensor(q, "q", (B, Hq, D), torch.bfloat16, where)
-    _check_tensor(k_cache, "k_cache", (num_pages, page_size, Hkv, D), torch.bfloat16, where)
-    _check_tensor(v_cache, "v_cache", (num_pages, page_size, Hkv, D), torch.bfloat16, where)
+    _check_tensor(k_cache, "k_cache", cache_shape, torch.bfloat16, where)
+    _check_tensor(v_cache, "v_cache", cache_shape, torch.bfloat16, where)
     _require(isinstance(block_table, torch.Tensor) and block_table.dim() == 2, ERR_SHAPE, where,
              "block_table must be a 2-D tensor [B, max_pages]")
     max_pages = block_table.shape[1]
@@ -451,11 +470,12 @@ def attention_decode(q, k_cache, v_cache, block_table, seq_lens, scale: float | 
             workspace = torch.empty(need, device=dev, dtype=torch.uint8)
         wp = workspace.data_ptr() if workspace is not None else None
         wb = workspace.numel() * workspace.element_size() if workspace is not None else 0
-        rc = axis_attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
-                              seq_lens.data_ptr(), o.data_ptr(), l.data_ptr(), B, Hq, Hkv, D, page_size, max_pages,
-                              num_pages, scale, wp, wb, _stream(stream, dev))
+        call = axis_attn_decode_hnd if hnd else axis_attn_decode
+        rc = call(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
+                  o.data_ptr(), l.data_ptr(), B, Hq, Hkv, D, page_size, max_pages, num_pages, scale, wp, wb,
+                  _stream(stream, dev))
     if rc:
-        raise AxisAttnError(rc, "axis_attn_decode")
+        raise AxisAttnError(rc, call.__name__)
     return o, l
 
 

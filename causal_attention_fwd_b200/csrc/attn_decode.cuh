@@ -13,13 +13,15 @@
 // about 4 G flops per byte, far below the tensor cores' ridge, so it is
 // HBM-bound: the kernel is built to keep the memory system busy.
 //   * persistent: as many CTAs as fit on the SMs walk the work items (b, kv
-//     head, split of the sequence); a producer warp reads the block table 32
-//     pieces ahead into shared memory and one of its threads streams 32-key
-//     pieces of the cache pages through TMA (a 3-D tensor map over the cache,
-//     128B swizzle) into a ring of shared-memory stages, K and V of a piece on
-//     one mbarrier, running ahead across item boundaries;
-//   * four compute warps take the pieces in turn and keep their own running
-//     max, sum and O for the G <= 8 query heads of the item.  The products
+//     head, split of the sequence); a producer warp prepares 32 pieces at a
+//     time (one lane per piece reads its block-table entries and forms its
+//     copies' coordinates) and streams 32-key pieces of the cache pages
+//     through TMA (a 3-D tensor map over the cache, 128B swizzle) into a ring
+//     of shared-memory stages, K and V of a piece on one mbarrier, running
+//     ahead across item boundaries;
+//   * the compute warps (4 at D = 64, 1 at D = 128) take the pieces in turn
+//     and keep their own running max, sum and O for the G <= 8 query heads
+//     of the item.  The products
 //     run on the warp-level tensor-core MMA (m16n8k16, bf16 in, fp32 out),
 //     the heads as rows of a 16-row tile: S = Q K^T with K's fragments
 //     loaded straight from the swizzled rows (ldmatrix), the online softmax in
@@ -27,7 +29,7 @@
 //     kept in registers as the A operand of O += P V, V through the
 //     transposing load.  Per 8 KB piece that is about a tenth of the
 //     instructions of the same arithmetic on the CUDA cores;
-//   * at the end of an item the four warps' states are merged in shared
+//   * at the end of an item the warps' states are merged in shared
 //     memory; a split writes its unnormalised (m, l, O) to the workspace,
 //     which a second kernel merges (split-K over long sequences keeps every
 //     SM busy at small batch); with one split the CTA writes O and LSE itself.
@@ -49,17 +51,30 @@ struct DecArgs {
   float* lse;              // [B, Hq]
   float* part;             // [B * Hq][n_splits][D + 2]: m, l, O (n_splits > 1)
   int B, Hq, Hkv, G, page_size, max_pages, num_pages;
+  int hnd;                 // cache layout: 0 [pages, page_size, Hkv, D]; 1 [pages, Hkv, page_size, D]
   int keys_per_split;      // a multiple of 32
   int n_splits;
   float scale_log2;        // scale * log2(e)
 };
 
-// Compute warps per CTA at head dim 64 / 128 (warp 0 is the producer).
+// Compute warps per CTA and ring stages at head dim 64 / 128 (warp 0 is the
+// producer).  Small CTAs, many per SM: each CTA's producer and compute warps
+// form one dependent chain per piece, so the SM's throughput grows with the
+// number of chains.  Measured at page size 16 to 64 (HBM fraction): D = 64,
+// 4 warps x 4 stages (5 CTAs / SM) 0.79-0.91 against 0.70-0.72 with 8 stages
+// (3 CTAs / SM); D = 128, 1 warp x 2 stages (6 CTAs / SM) 0.94-0.98 against
+// 0.90-0.96 with 4 x 4 (2 CTAs / SM).
 #ifndef AXIS_ATTN_DEC_CW64
 #define AXIS_ATTN_DEC_CW64 4
 #endif
 #ifndef AXIS_ATTN_DEC_NST64
-#define AXIS_ATTN_DEC_NST64 8
+#define AXIS_ATTN_DEC_NST64 4
+#endif
+#ifndef AXIS_ATTN_DEC_CW128
+#define AXIS_ATTN_DEC_CW128 1
+#endif
+#ifndef AXIS_ATTN_DEC_NST128
+#define AXIS_ATTN_DEC_NST128 2
 #endif
 
 template <int HD>
@@ -67,9 +82,9 @@ struct DecCfg {
   static constexpr int NSLAB = HD / 64;
   static constexpr uint32_t SLAB = 32 * 128;            // 32 rows x 128 bytes
   static constexpr uint32_t PIECE = NSLAB * SLAB;       // 32 keys x HD bf16
-  static constexpr int CW = HD == 64 ? AXIS_ATTN_DEC_CW64 : 4;  // compute warps
+  static constexpr int CW = HD == 64 ? AXIS_ATTN_DEC_CW64 : AXIS_ATTN_DEC_CW128;  // compute warps
   static constexpr int THREADS = 32 * (1 + CW);
-  static constexpr int NST = HD == 64 ? AXIS_ATTN_DEC_NST64 : 4;  // ring stages
+  static constexpr int NST = HD == 64 ? AXIS_ATTN_DEC_NST64 : AXIS_ATTN_DEC_NST128;  // ring stages
   // A compute warp waits on the phase of a stage only after the stage's
   // previous phase has completed (a parity wait cannot tell phase k from
   // phase k - 2): the previous piece in a stage must be the same warp's,
@@ -112,7 +127,7 @@ __device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report
 // Persistent: each CTA walks the items w = blockIdx.x, blockIdx.x + gridDim.x,
 // ...; the ring positions count pieces over all of its items, so the producer
 // streams the next item's pieces while the compute warps finish this one.
-// Compute warp (g mod 4) takes the CTA's g-th piece.
+// Compute warp (g mod CW) takes the CTA's g-th piece.
 template <int HD>
 __global__ void __launch_bounds__(DecCfg<HD>::THREADS)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -147,71 +162,72 @@ __global__ void __launch_bounds__(DecCfg<HD>::THREADS)
 
   if (warp == 0) {
     // ============================================================ producer
-    // The whole warp reads the block-table entries of 32 pieces at a time
-    // into shared memory (32 independent loads instead of one dependent
-    // global read per page in front of every copy); lane 0 then checks them
-    // and issues the copies.
-    int* tbl = reinterpret_cast<int*>(gbase + C::OFF_TBL);
+    // Per block of 32 pieces, lane j prepares piece j at once with the other
+    // lanes: it reads the block-table entries of its piece's pages (32
+    // independent loads instead of one dependent global read in front of
+    // every copy), checks them and forms its boxes' coordinates.  The lanes
+    // then take their turns at the ring: lane j waits for its stage, sets its
+    // flag and issues its copies.  The single issuing thread's work per piece
+    // is thereby the wait and the copies alone (a thread doing all of it
+    // issued one 8 KB piece per ~0.5 us: below HBM speed with 3 CTAs per SM).
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
     }
     const int rows = a.page_size < 32 ? a.page_size : 32;  // rows per TMA box
     const int nbox = 32 / rows;                              // boxes per 32-key piece
-    int g = 0;  // pieces issued (over all items)
+    const int ps_shift = 31 - __clz(a.page_size);            // page_size is a power of two
+    const int ps_mask = a.page_size - 1;
+    int g = 0;  // pieces issued (over all items); the same in every lane
     bool ok = true;
     for (int w = (int)blockIdx.x; ok && w < n_items; w += (int)gridDim.x) {
       const DecItem I = dec_item(a, w, lane == 0);
+      const int* row_tbl = a.block_table + (size_t)I.b * a.max_pages;
       for (int t0 = 0; ok && t0 < I.n_pieces; t0 += 32) {
-        for (int e = lane; e < 32 * nbox; e += 32) {  // e = (t - t0) * nbox + x
-          const int t = t0 + e / nbox, key = I.k0 + 32 * t + (e % nbox) * rows;
-          tbl[e] = t < I.n_pieces && key < I.k1 ? a.block_table[(size_t)I.b * a.max_pages + key / a.page_size] : 0;
+        const int kt = I.k0 + 32 * (t0 + lane);  // this lane's piece
+        // boxes x < nload of this lane's piece: cache coordinates (c1[x], c2[x]) of box row 0
+        int c1[4], c2[4], nload = 0, usable = 1;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int key = kt + x * rows;
+          c1[x] = c2[x] = 0;
+          if (t0 + lane < I.n_pieces && x < nbox && key < I.k1) {
+            const int page = row_tbl[key >> ps_shift];
+            if (page < 0 || page >= a.num_pages) usable = 0;
+            c1[x] = a.hnd ? (key & ps_mask) : I.kv;
+            c2[x] = a.hnd ? page * a.Hkv + I.kv : page * a.page_size + (key & ps_mask);
+            ++nload;
+          }
         }
-        __syncwarp();
-        if (lane == 0) {
-          const int t1 = min(I.n_pieces, t0 + 32);
-          for (int t = t0; t < t1; ++t, ++g) {
+        const int n = min(32, I.n_pieces - t0);
+        for (int j = 0; j < n; ++j, ++g) {
+          if (lane == j) {
             const int s = g % NST;
             if (g >= NST && !mbar_wait_bounded<true>(bar_empty(s), ((g / NST) & 1) ^ 1, ctl, D_EMPTY)) {
               ok = false;
-              break;
-            }
-            const int kt = I.k0 + 32 * t;
-            // pages of this piece (at most 4: page_size >= 8), checked before any copy
-            int usable = 1, nload = 0, pages[4] = {0, 0, 0, 0};
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              const int key = kt + x * rows;
-              if (x < nbox && key < I.k1) {
-                pages[x] = tbl[(t - t0) * nbox + x];
-                if (pages[x] < 0 || pages[x] >= a.num_pages) usable = 0;
-                ++nload;
-              }
-            }
-            flag[s] = usable;
-            if (!usable) {
-              atomicOr(&g_status, 2u);
-              mbar_arrive(bar_full(s));
             } else {
-              mbar_arrive_expect_tx(bar_full(s), (uint32_t)(nload * rows * HD * 2 * 2));
+              flag[s] = usable;
+              if (!usable) {
+                atomicOr(&g_status, 2u);
+                mbar_arrive(bar_full(s));
+              } else {
+                mbar_arrive_expect_tx(bar_full(s), (uint32_t)(nload * rows * HD * 2 * 2));
 #pragma unroll
-              for (int x = 0; x < 4; ++x) {
-                if (x >= nload) break;
-                const int key = kt + x * rows;
-                const int row = pages[x] * a.page_size + key % a.page_size;
+                for (int x = 0; x < 4; ++x) {
+                  if (x >= nload) break;
 #pragma unroll
-                for (int sl = 0; sl < C::NSLAB; ++sl) {
-                  const uint32_t off = s * C::PIECE + sl * C::SLAB + x * rows * 128;
-                  tma_load_3d(sK + off, &tm_k, bar_full(s), 64 * sl, I.kv, row);
-                  tma_load_3d(sV + off, &tm_v, bar_full(s), 64 * sl, I.kv, row);
+                  for (int sl = 0; sl < C::NSLAB; ++sl) {
+                    const uint32_t off = s * C::PIECE + sl * C::SLAB + x * rows * 128;
+                    tma_load_3d(sK + off, &tm_k, bar_full(s), 64 * sl, c1[x], c2[x]);
+                    tma_load_3d(sV + off, &tm_v, bar_full(s), 64 * sl, c1[x], c2[x]);
+                  }
                 }
               }
             }
           }
+          ok = __shfl_sync(0xffffffffu, ok, j);
+          if (!ok) break;
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        g = __shfl_sync(0xffffffffu, g, 0);
-        __syncwarp();  // lane 0 is done with this block of table entries
       }
     }
     // drain: every copy started has landed before the CTA exits
@@ -236,7 +252,7 @@ __global__ void __launch_bounds__(DecCfg<HD>::THREADS)
     bool ok = true;
     // Every compute warp walks every item, also after a wait has given up
     // (its later waits then return at once: the CTA's abort flag is set), so
-    // that all four reach each of the named barriers below.
+    // that all of them reach each of the named barriers below.
     for (int w = (int)blockIdx.x; w < n_items; w += (int)gridDim.x) {
       const DecItem I = dec_item(a, w, false);
       // Q as A fragments: (row g0, columns 16 ks + q2 + {0,1}) and (+8); the
@@ -255,7 +271,7 @@ __global__ void __launch_bounds__(DecCfg<HD>::THREADS)
 #pragma unroll
       for (int nd = 0; nd < ND; ++nd) o_acc[nd][0] = o_acc[nd][1] = o_acc[nd][2] = o_acc[nd][3] = 0.f;
       float m_run = -INFINITY, l_part = 0.f;  // row g0: running max (log2 units), this lane's share of the sum
-      // this warp's pieces of the item: the CTA's piece gbase_item + t goes to warp (gbase_item + t) % 4
+      // this warp's pieces of the item: the CTA's piece gbase_item + t goes to warp (gbase_item + t) % CW
       for (int t = (cw - gbase_item % CW + CW) % CW; ok && t < I.n_pieces; t += CW) {
         const int gp = gbase_item + t;
         const int s = gp % NST;
@@ -337,7 +353,7 @@ __global__ void __launch_bounds__(DecCfg<HD>::THREADS)
         if (lane == 0) mbar_arrive(bar_empty(s));
       }
       gbase_item += I.n_pieces;
-      // ---- this warp's (m, l, O) of each head, then the merge of the four warps
+      // ---- this warp's (m, l, O) of each head, then the merge of the CW warps
       float l = l_part;
       l += __shfl_xor_sync(0xffffffffu, l, 1);
       l += __shfl_xor_sync(0xffffffffu, l, 2);

@@ -609,10 +609,13 @@ int check_decode_shape(int B, int Hq, int Hkv, int D, int page_size, int max_pag
 struct DecSplit {
   int n_splits, keys_per_split;
 };
+#ifndef AXIS_ATTN_DEC_SPLIT_ITEMS
+#define AXIS_ATTN_DEC_SPLIT_ITEMS 296
+#endif
 DecSplit decode_split(int B, int Hkv, int page_size, int max_pages) {
   const long long keys = (long long)max_pages * page_size;
   const long long units = (long long)B * Hkv;
-  long long n = (296 + units - 1) / units;
+  long long n = (AXIS_ATTN_DEC_SPLIT_ITEMS + units - 1) / units;
   const long long n_max = (keys + 255) / 256;
   if (n > n_max) n = n_max;
   if (n < 1) n = 1;
@@ -633,6 +636,22 @@ bool make_cache_map(CUtensorMap* map, const void* ptr, int rows, int Hkv, int D,
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)rows};
   const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
   const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The same pool in the head-major layout [num_pages, Hkv, page_size, D]: a
+// 3-D map (D, page_size, num_pages * Hkv), box (64, box_rows, 1); a box lands
+// in shared memory exactly as the other layout's does (box_rows rows of 128 B).
+bool make_cache_map_hnd(CUtensorMap* map, const void* ptr, int num_pages, int page_size, int Hkv, int D,
+                        int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)page_size, (cuuint64_t)num_pages * Hkv};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)page_size * D * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -667,10 +686,11 @@ extern "C" size_t axis_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D
   return decode_ws_bytes(B, Hq, D, decode_split(B, Hkv, page_size, max_pages));
 }
 
-extern "C" int axis_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
-                                const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
-                                int page_size, int max_pages, int num_pages, float scale, void* workspace,
-                                size_t workspace_bytes, void* stream) {
+namespace axis_attn {
+namespace {
+int run_decode(const void* q, const void* k_cache, const void* v_cache, const int* block_table, const int* seq_lens,
+               void* o, float* lse, int B, int Hq, int Hkv, int D, int page_size, int max_pages, int num_pages,
+               float scale, void* workspace, size_t workspace_bytes, void* stream, bool hnd) {
   if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !o || !lse) return AXIS_ATTN_ERR_NULL;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse) ||
       (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
@@ -684,9 +704,12 @@ extern "C" int axis_attn_decode(const void* q, const void* k_cache, const void* 
   if (int rc = check_device(&dev)) return rc;
   CUtensorMap mk, mv;
   const int box_rows = page_size < 32 ? page_size : 32;
-  if (!make_cache_map(&mk, k_cache, num_pages * page_size, Hkv, D, box_rows) ||
-      !make_cache_map(&mv, v_cache, num_pages * page_size, Hkv, D, box_rows))
-    return AXIS_ATTN_ERR_CUDA;
+  const bool maps_ok =
+      hnd ? make_cache_map_hnd(&mk, k_cache, num_pages, page_size, Hkv, D, box_rows) &&
+                make_cache_map_hnd(&mv, v_cache, num_pages, page_size, Hkv, D, box_rows)
+          : make_cache_map(&mk, k_cache, num_pages * page_size, Hkv, D, box_rows) &&
+                make_cache_map(&mv, v_cache, num_pages * page_size, Hkv, D, box_rows);
+  if (!maps_ok) return AXIS_ATTN_ERR_CUDA;
   DecArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.block_table = block_table;
@@ -701,6 +724,7 @@ extern "C" int axis_attn_decode(const void* q, const void* k_cache, const void* 
   a.page_size = page_size;
   a.max_pages = max_pages;
   a.num_pages = num_pages;
+  a.hnd = hnd ? 1 : 0;
   a.keys_per_split = sp.keys_per_split;
   a.n_splits = sp.n_splits;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
@@ -714,6 +738,24 @@ extern "C" int axis_attn_decode(const void* q, const void* k_cache, const void* 
   else
     attn_decode_combine_kernel<128><<<grid, 256, 0, st>>>(a.part, a.o, lse, rows, sp.n_splits);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+}  // namespace
+}  // namespace axis_attn
+
+extern "C" int axis_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                                const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
+                                int page_size, int max_pages, int num_pages, float scale, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  return axis_attn::run_decode(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
+                               max_pages, num_pages, scale, workspace, workspace_bytes, stream, false);
+}
+
+extern "C" int axis_attn_decode_hnd(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                                    const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
+                                    int page_size, int max_pages, int num_pages, float scale, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return axis_attn::run_decode(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
+                               max_pages, num_pages, scale, workspace, workspace_bytes, stream, true);
 }
 
 static unsigned int g_last_status_word;

@@ -280,6 +280,20 @@ int axis_attn_decode(const void* q, const void* k_cache, const void* v_cache, co
                      size_t workspace_bytes, void* stream);
 
 /*
+ * The same decode step on a head-major pool: k_cache, v_cache are
+ * [num_pages, Hkv, page_size, D] bf16, so one kv head's rows of a page are
+ * contiguous (page_size * D * 2 bytes) instead of D * 2-byte pieces at a
+ * stride of Hkv * D * 2 bytes.  Position j of sequence b is row j % page_size
+ * of head kv in page block_table[b * max_pages + j / page_size].  Every other
+ * argument, the workspace (axis_attn_decode_workspace_bytes), the results, the
+ * requirements and the error behaviour are those of axis_attn_decode.
+ */
+int axis_attn_decode_hnd(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                         const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int D,
+                         int page_size, int max_pages, int num_pages, float scale, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then returns AXIS_ATTN_ERR_TIMEOUT if any kernel of
  * this library on the current device has reported a timed-out device wait since
  * the last call, else AXIS_ATTN_ERR_INDEX if a decode step met an out-of-range

@@ -186,12 +186,12 @@ def test_valid_args_without_gpu_report_cuda_error(lib):
     assert _fwd() in (4, 6)
 
 
-def _dec(**over):
+def _dec(fn="axis_attn_decode", **over):
     args = dict(q=A, k_cache=A, v_cache=A, block_table=A, seq_lens=A, o=A, lse=A, B=1, Hq=32, Hkv=8, D=128,
                 page_size=64, max_pages=128, num_pages=128, scale=0.088, workspace=A, workspace_bytes=1 << 30,
                 stream=None)
     args.update(over)
-    return aa.axis_attn_decode(*args.values())
+    return getattr(aa, fn)(*args.values())
 
 
 @pytest.mark.parametrize("over,code", [
@@ -203,8 +203,9 @@ def _dec(**over):
     (dict(page_size=512), 4),
     (dict(workspace=None), 5), (dict(workspace=A + 16), 5), (dict(workspace_bytes=100), 5),
 ])
-def test_decode_rejects(lib, over, code):
-    assert _dec(**over) == code
+@pytest.mark.parametrize("fn", ["axis_attn_decode", "axis_attn_decode_hnd"])
+def test_decode_rejects(lib, fn, over, code):
+    assert _dec(fn, **over) == code
 
 
 def test_decode_workspace_bytes(lib):

@@ -89,3 +89,25 @@ def test_mixed_devices_are_rejected_before_any_call():
     q, k, v = qkv()
     e = fwd_error(q, k, torch.empty((B, S, Hkv, D), dtype=torch.bfloat16, device="meta"))
     assert e.code == 4  # the first tensor is not on CUDA
+
+
+def dec_error(layout="NHD", **over):
+    a = dict(q=bf(2, 8, D), k_cache=bf(5, 16, 4, D), v_cache=bf(5, 16, 4, D),
+             block_table=torch.zeros(2, 3, dtype=torch.int32), seq_lens=torch.ones(2, dtype=torch.int32))
+    a.update(over)
+    with pytest.raises(aa.AxisAttnError) as e:
+        aa.attention_decode(a["q"], a["k_cache"], a["v_cache"], a["block_table"], a["seq_lens"], layout=layout)
+    return e.value
+
+
+def test_decode_layouts_read_the_cache_shape_their_own_way():
+    # [num_pages, page_size, Hkv, D] and [num_pages, Hkv, page_size, D] of the same pool
+    e = dec_error("NHD")
+    assert e.code == 4 and "CUDA device" in str(e)
+    e = dec_error("HND", k_cache=bf(5, 4, 16, D), v_cache=bf(5, 4, 16, D))
+    assert e.code == 4 and "CUDA device" in str(e)
+    # v_cache in the other layout than k_cache
+    e = dec_error("HND", k_cache=bf(5, 4, 16, D))
+    assert "v_cache" in str(e)
+    e = dec_error("BHSD")
+    assert "layout" in str(e)

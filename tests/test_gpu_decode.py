@@ -8,6 +8,9 @@ abs <= 1e-4).  Cases cover both head dims, GQA groups 1..8 (including 3),
 page sizes 8..256, ragged lengths (1, around page and piece edges), batches
 that take the split-K path and batches that do not, and bad device-side
 indices, which must be reported as AXIS_ATTN_ERR_INDEX without an access.
+Every case runs on both pool layouts: [num_pages, page_size, Hkv, D]
+(axis_attn_decode) and the head-major [num_pages, Hkv, page_size, D]
+(axis_attn_decode_hnd), the latter a transposed copy of the same pool.
 """
 import math
 
@@ -54,7 +57,14 @@ def paged(k, v, lens, page_size, seed, extra_pages=3):
     return kc, vc, table, num_pages
 
 
-def run_case(oracle_mod, B, Hq, Hkv, D, Smax, page_size, lens, seed):
+def as_layout(kc, vc, layout):
+    """The pool in the requested layout ("HND" swaps the page-row and head axes)."""
+    if layout == "HND":
+        return kc.transpose(1, 2).contiguous(), vc.transpose(1, 2).contiguous()
+    return kc, vc
+
+
+def run_case(oracle_mod, B, Hq, Hkv, D, Smax, page_size, lens, seed, layout="NHD"):
     g = torch.Generator().manual_seed(seed)
     q = torch.randn((B, Hq, D), generator=g).to(torch.bfloat16)
     k = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
@@ -62,9 +72,10 @@ def run_case(oracle_mod, B, Hq, Hkv, D, Smax, page_size, lens, seed):
     lens = np.asarray(lens, np.int32)
     sc = 1.0 / math.sqrt(D)
     kc, vc, table, num_pages = paged(k, v, lens, page_size, seed)
+    kc, vc = as_layout(kc, vc, layout)
     dev = torch.device("cuda:0")
     o, lse = aa.attention_decode(q.to(dev), kc.to(dev), vc.to(dev), table.to(dev),
-                                 torch.from_numpy(lens).to(dev), scale=sc)
+                                 torch.from_numpy(lens).to(dev), scale=sc, layout=layout)
     aa.check_status()
     ro, rl = oracle_mod.attn_decode(q, k, v, lens, sc)
     eo = float((o.cpu().double() - torch.from_numpy(ro)).abs().max())
@@ -90,10 +101,11 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("layout", ["NHD", "HND"])
 @pytest.mark.parametrize("B,Hq,Hkv,D,Smax,ps,lens", CASES)
-def test_decode_matches_oracle(oracle_mod, B, Hq, Hkv, D, Smax, ps, lens):
-    eo, el = run_case(oracle_mod, B, Hq, Hkv, D, Smax, ps, lens, seed=3000 + B + Hq + D + Smax + ps)
-    print(f"B{B} Hq{Hq} Hkv{Hkv} D{D} S{Smax} ps{ps}: O {eo:.2e} LSE {el:.2e}")
+def test_decode_matches_oracle(oracle_mod, B, Hq, Hkv, D, Smax, ps, lens, layout):
+    eo, el = run_case(oracle_mod, B, Hq, Hkv, D, Smax, ps, lens, seed=3000 + B + Hq + D + Smax + ps, layout=layout)
+    print(f"{layout} B{B} Hq{Hq} Hkv{Hkv} D{D} S{Smax} ps{ps}: O {eo:.2e} LSE {el:.2e}")
     assert eo <= TOL_O and el <= TOL_LSE
 
 
@@ -104,7 +116,8 @@ def test_decode_workspace_is_split_dependent():
     assert aa.axis_attn_decode_workspace_bytes(1, 32, 8, 96, 64, 128) == 0  # unsupported D
 
 
-def test_decode_bad_indices_are_reported_not_used(oracle_mod):
+@pytest.mark.parametrize("layout", ["NHD", "HND"])
+def test_decode_bad_indices_are_reported_not_used(oracle_mod, layout):
     B, Hq, Hkv, D, Smax, ps = 2, 4, 2, 64, 64, 16
     g = torch.Generator().manual_seed(9)
     q = torch.randn((B, Hq, D), generator=g).to(torch.bfloat16)
@@ -112,17 +125,19 @@ def test_decode_bad_indices_are_reported_not_used(oracle_mod):
     v = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
     lens = np.array([64, 40], np.int32)
     kc, vc, table, num_pages = paged(k, v, lens, ps, 9)
+    kc, vc = as_layout(kc, vc, layout)
     dev = torch.device("cuda:0")
     args = [t.to(dev) for t in (q, kc, vc)]
     bad = table.clone()
     bad[1, 1] = num_pages + 1000  # inside sequence 1's length
-    aa.attention_decode(*args, bad.to(dev), torch.from_numpy(lens).to(dev), scale=D ** -0.5)
+    aa.attention_decode(*args, bad.to(dev), torch.from_numpy(lens).to(dev), scale=D ** -0.5, layout=layout)
     assert aa.axis_attn_get_status(aa.binding._stream(None)) == 8  # AXIS_ATTN_ERR_INDEX
     bad_len = torch.tensor([64, 10 ** 6], dtype=torch.int32)
-    aa.attention_decode(*args, table.to(dev), bad_len.to(dev), scale=D ** -0.5)
+    aa.attention_decode(*args, table.to(dev), bad_len.to(dev), scale=D ** -0.5, layout=layout)
     assert aa.axis_attn_get_status(aa.binding._stream(None)) == 8
     # the same call with good indices is exact afterwards
-    o, lse = aa.attention_decode(*args, table.to(dev), torch.from_numpy(lens).to(dev), scale=D ** -0.5)
+    o, lse = aa.attention_decode(*args, table.to(dev), torch.from_numpy(lens).to(dev), scale=D ** -0.5,
+                                 layout=layout)
     aa.check_status()
     ro, rl = oracle_mod.attn_decode(q, k, v, lens, D ** -0.5)
     assert float((o.cpu().double() - torch.from_numpy(ro)).abs().max()) <= TOL_O
