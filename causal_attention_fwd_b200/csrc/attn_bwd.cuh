@@ -666,36 +666,56 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
   for (size_t k = gtid; k < dq_vec4; k += nthreads) dqacc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
+// Iterations of a grid-stride loop whose loads a thread issues together
+// before using any (one pair of 16-byte loads at a time per thread left the
+// finalize at 0.75 of HBM bandwidth).
+constexpr int BWD_STREAM_U = 4;
+
 // dq[b,i,h,:] = bf16(dqacc[b,h,i,:]); 8 features per thread.  With a RoPE
-// table the row leaves through the transposed rotation of position i.
+// table the row leaves through the transposed rotation of position i.  The
+// fp32 accumulator (twice the bytes of the output) is read in its own
+// [B, Hq, S, D] order, 32 contiguous bytes per thread; the bf16 rows go to
+// their [B, S, Hq, D] places as whole 128- or 256-byte lines.
 template <int HD>
-__global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* __restrict__ dqacc,
-                                                                  __nv_bfloat16* __restrict__ dq, int Hq,
-                                                                  int S, size_t n8,
-                                                                  const double2* __restrict__ rope_cs) {
+__global__ void __launch_bounds__(256, 4) attn_bwd_dq_convert_kernel(const float* __restrict__ dqacc,
+                                                                     __nv_bfloat16* __restrict__ dq, int Hq,
+                                                                     int S, size_t n8,
+                                                                     const double2* __restrict__ rope_cs) {
   const size_t stride = (size_t)gridDim.x * blockDim.x;
-  for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < n8; k += stride) {
-    const int c8 = (int)(k % (HD / 8));
-    const size_t row = k / (HD / 8);   // row in [B, S, Hq] order
-    const int h = (int)(row % Hq);
-    const size_t bi = row / Hq;        // b * S + i
-    const int i = (int)(bi % S);
-    const size_t b = bi / S;
-    const float4* src = reinterpret_cast<const float4*>(dqacc + (((b * Hq + h) * S + i) * HD) + 8 * c8);
-    float4 x = src[0], y = src[1];
-    if (rope_cs != nullptr) {  // pairs 4 c8 .. 4 c8 + 3 at position i, transposed rotation
-      const double2* t = rope_cs + (size_t)i * (HD / 2) + 4 * c8;
-      rope_back(x.x, x.y, t[0]);
-      rope_back(x.z, x.w, t[1]);
-      rope_back(y.x, y.y, t[2]);
-      rope_back(y.z, y.w, t[3]);
+  const float4* src = reinterpret_cast<const float4*>(dqacc);
+  for (size_t k0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k0 < n8; k0 += BWD_STREAM_U * stride) {
+    float4 x[BWD_STREAM_U], y[BWD_STREAM_U];
+#pragma unroll
+    for (int u = 0; u < BWD_STREAM_U; ++u) {
+      const size_t k = k0 + u * stride;
+      if (k < n8) {
+        x[u] = src[2 * k];
+        y[u] = src[2 * k + 1];
+      }
     }
-    uint4 out;
-    out.x = pack_bf16x2(x.x, x.y);
-    out.y = pack_bf16x2(x.z, x.w);
-    out.z = pack_bf16x2(y.x, y.y);
-    out.w = pack_bf16x2(y.z, y.w);
-    reinterpret_cast<uint4*>(dq + row * HD)[c8] = out;
+#pragma unroll
+    for (int u = 0; u < BWD_STREAM_U; ++u) {
+      const size_t k = k0 + u * stride;
+      if (k >= n8) continue;
+      const int c8 = (int)(k % (HD / 8));
+      const size_t r = k / (HD / 8);  // (b * Hq + h) * S + i
+      const int i = (int)(r % S);
+      const size_t bh = r / S;
+      const size_t row = (bh / Hq * S + i) * Hq + bh % Hq;  // (b * S + i) * Hq + h
+      if (rope_cs != nullptr) {  // pairs 4 c8 .. 4 c8 + 3 at position i, transposed rotation
+        const double2* t = rope_cs + (size_t)i * (HD / 2) + 4 * c8;
+        rope_back(x[u].x, x[u].y, t[0]);
+        rope_back(x[u].z, x[u].w, t[1]);
+        rope_back(y[u].x, y[u].y, t[2]);
+        rope_back(y[u].z, y[u].w, t[3]);
+      }
+      uint4 out;
+      out.x = pack_bf16x2(x[u].x, x[u].y);
+      out.y = pack_bf16x2(x[u].z, x[u].w);
+      out.z = pack_bf16x2(y[u].x, y[u].y);
+      out.w = pack_bf16x2(y[u].z, y[u].w);
+      reinterpret_cast<uint4*>(dq + row * HD)[c8] = out;
+    }
   }
 }
 

@@ -359,7 +359,7 @@ int run_main(const void* q, const void* k, const void* v, const void* dO, void* 
 int run_finalize(void* dq, int B, int Hq, int S, int D, const WsPtrs& p, cudaStream_t st,
                  const double* rope_cs = nullptr) {
   const size_t n8 = (size_t)B * S * Hq * D / 8;
-  const unsigned grid = (unsigned)((n8 + 255) / 256 < 4096 ? (n8 + 255) / 256 : 4096);
+  const unsigned grid = (unsigned)((n8 + 255) / 256 < 148 * 16 ? (n8 + 255) / 256 : 148 * 16);
   auto* out = static_cast<__nv_bfloat16*>(dq);
   const double2* cs = reinterpret_cast<const double2*>(rope_cs);
   if (D == 64) {
