@@ -57,13 +57,16 @@ struct DecArgs {
   float scale_log2;        // scale * log2(e)
 };
 
-// Compute warps per CTA and ring stages at head dim 64 / 128 (warp 0 is the
-// producer).  Small CTAs, many per SM: each CTA's producer and compute warps
-// form one dependent chain per piece, so the SM's throughput grows with the
-// number of chains.  Measured at page size 16 to 64 (HBM fraction): D = 64,
-// 4 warps x 4 stages (5 CTAs / SM) 0.79-0.91 against 0.70-0.72 with 8 stages
-// (3 CTAs / SM); D = 128, 1 warp x 2 stages (6 CTAs / SM) 0.94-0.98 against
-// 0.90-0.96 with 4 x 4 (2 CTAs / SM).
+// Compute warps per CTA and ring stages (warp 0 is the producer).  Each CTA's
+// producer and compute warps form one dependent chain per piece, and an SM's
+// bytes in flight are its CTAs x stages x piece bytes.  Two configurations per
+// head dim, chosen per call by the host:
+//   * wide (many small CTAs per SM) when the items fill them: measured at page
+//     size 16 to 64 (HBM fraction), D = 64 4 warps x 4 stages (5 CTAs / SM)
+//     0.79-0.91 against 0.70-0.72 with 8 stages (3 CTAs / SM); D = 128 1 warp
+//     x 2 stages (5 CTAs / SM) 0.94-0.98 against 0.90-0.96 with 4 x 4;
+//   * deep (fewer CTAs, more stages each) when a small batch leaves most of
+//     the wide configuration's CTAs without an item.
 #ifndef AXIS_ATTN_DEC_CW64
 #define AXIS_ATTN_DEC_CW64 4
 #endif
@@ -76,15 +79,29 @@ struct DecArgs {
 #ifndef AXIS_ATTN_DEC_NST128
 #define AXIS_ATTN_DEC_NST128 2
 #endif
+#ifndef AXIS_ATTN_DEC_DEEP_CW64
+#define AXIS_ATTN_DEC_DEEP_CW64 4
+#endif
+#ifndef AXIS_ATTN_DEC_DEEP_NST64
+#define AXIS_ATTN_DEC_DEEP_NST64 8
+#endif
+#ifndef AXIS_ATTN_DEC_DEEP_CW128
+#define AXIS_ATTN_DEC_DEEP_CW128 4
+#endif
+#ifndef AXIS_ATTN_DEC_DEEP_NST128
+#define AXIS_ATTN_DEC_DEEP_NST128 4
+#endif
 
-template <int HD>
+template <int HD, bool DEEP>
 struct DecCfg {
   static constexpr int NSLAB = HD / 64;
   static constexpr uint32_t SLAB = 32 * 128;            // 32 rows x 128 bytes
   static constexpr uint32_t PIECE = NSLAB * SLAB;       // 32 keys x HD bf16
-  static constexpr int CW = HD == 64 ? AXIS_ATTN_DEC_CW64 : AXIS_ATTN_DEC_CW128;  // compute warps
+  static constexpr int CW = DEEP ? (HD == 64 ? AXIS_ATTN_DEC_DEEP_CW64 : AXIS_ATTN_DEC_DEEP_CW128)
+                                 : (HD == 64 ? AXIS_ATTN_DEC_CW64 : AXIS_ATTN_DEC_CW128);  // compute warps
   static constexpr int THREADS = 32 * (1 + CW);
-  static constexpr int NST = HD == 64 ? AXIS_ATTN_DEC_NST64 : AXIS_ATTN_DEC_NST128;  // ring stages
+  static constexpr int NST = DEEP ? (HD == 64 ? AXIS_ATTN_DEC_DEEP_NST64 : AXIS_ATTN_DEC_DEEP_NST128)
+                                  : (HD == 64 ? AXIS_ATTN_DEC_NST64 : AXIS_ATTN_DEC_NST128);  // ring stages
   // A compute warp waits on the phase of a stage only after the stage's
   // previous phase has completed (a parity wait cannot tell phase k from
   // phase k - 2): the previous piece in a stage must be the same warp's,
@@ -128,11 +145,11 @@ __device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report
 // ...; the ring positions count pieces over all of its items, so the producer
 // streams the next item's pieces while the compute warps finish this one.
 // Compute warp (g mod CW) takes the CTA's g-th piece.
-template <int HD>
-__global__ void __launch_bounds__(DecCfg<HD>::THREADS)
+template <int HD, bool DEEP>
+__global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const DecArgs a) {
-  using C = DecCfg<HD>;
+  using C = DecCfg<HD, DEEP>;
   constexpr int NST = C::NST, CW = C::CW;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -407,34 +424,84 @@ __global__ void __launch_bounds__(DecCfg<HD>::THREADS)
   }
 }
 
-// Merge the splits of every (b, h): one warp per row, lanes over features.
+// Merge the splits of every (b, h): one 256-thread CTA per row.  The maximum
+// over the splits comes from all threads at once (one split each); then warp w
+// takes splits w, w + 8, ... (lanes over features, DEC_COMBINE_U splits'
+// loads in flight at a time) and the 8 warps' sums meet in shared memory.
+// The few round trips to L2 this leaves per row matter: with one warp walking
+// tens of splits the merge took as long as the decode kernel itself.
+constexpr int DEC_COMBINE_U = 4;
 template <int HD>
 __global__ void __launch_bounds__(256) attn_decode_combine_kernel(const float* __restrict__ part,
                                                                   __nv_bfloat16* __restrict__ o,
                                                                   float* __restrict__ lse, int rows, int n_splits) {
-  constexpr int FPL = HD / 32;
-  const int lane = threadIdx.x & 31;
-  for (int bh = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); bh < rows;
-       bh += (int)((gridDim.x * blockDim.x) >> 5)) {
+  constexpr int FPL = HD / 32, NW = 8;
+  __shared__ float s_red[NW];
+  __shared__ float s_o[NW][HD];
+  const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
+  for (int bh = (int)blockIdx.x; bh < rows; bh += (int)gridDim.x) {
     const float* p = part + (size_t)bh * n_splits * (HD + 2);
+    // the maximum over the splits that saw keys (l > 0; a split past the end of the sequence has none)
     float mm = -INFINITY;
-    for (int s = 0; s < n_splits; ++s)
-      if (p[s * (HD + 2) + 1] > 0.f) mm = fmaxf(mm, p[s * (HD + 2)]);
+    for (int s = (int)threadIdx.x; s < n_splits; s += 32 * NW) {
+      const float2 ml = *reinterpret_cast<const float2*>(p + (size_t)s * (HD + 2));
+      if (ml.y > 0.f) mm = fmaxf(mm, ml.x);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, off));
+    if (lane == 0) s_red[warp] = mm;
+    __syncthreads();
+    mm = s_red[0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) mm = fmaxf(mm, s_red[w]);
+    // this warp's splits, weighted by 2^(m_s - mm)
     float l = 0.f, ov[FPL];
 #pragma unroll
     for (int f = 0; f < FPL; ++f) ov[f] = 0.f;
-    for (int s = 0; s < n_splits; ++s) {
-      const float* ps = p + s * (HD + 2);
-      if (!(ps[1] > 0.f)) continue;  // a split past the end of the sequence
-      const float e = ex2_approx(ps[0] - mm);
-      l += ps[1] * e;
+    for (int s0 = warp; s0 < n_splits; s0 += NW * DEC_COMBINE_U) {
+      float2 ml[DEC_COMBINE_U];
+      float v[DEC_COMBINE_U][FPL];
 #pragma unroll
-      for (int f = 0; f < FPL; ++f) ov[f] += ps[2 + lane * FPL + f] * e;
+      for (int u = 0; u < DEC_COMBINE_U; ++u) {
+        const int sp = s0 + NW * u;
+        ml[u] = make_float2(0.f, 0.f);
+        if (sp < n_splits) {
+          const float* ps = p + (size_t)sp * (HD + 2);
+          ml[u] = *reinterpret_cast<const float2*>(ps);
+#pragma unroll
+          for (int f = 0; f < FPL; ++f) v[u][f] = ps[2 + lane * FPL + f];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < DEC_COMBINE_U; ++u) {
+        if (!(ml[u].y > 0.f)) continue;
+        const float e = ex2_approx(ml[u].x - mm);
+        l += ml[u].y * e;
+#pragma unroll
+        for (int f = 0; f < FPL; ++f) ov[f] += v[u][f] * e;
+      }
     }
-    const float inv = l > 0.f ? 1.f / l : 0.f;
+    __syncthreads();  // every warp has read s_red
 #pragma unroll
-    for (int f = 0; f < FPL; ++f) o[(size_t)bh * HD + lane * FPL + f] = __float2bfloat16_rn(ov[f] * inv);
-    if (lane == 0) lse[bh] = (mm + __log2f(l)) * 0.69314718055994531f;
+    for (int f = 0; f < FPL; ++f) s_o[warp][lane * FPL + f] = ov[f];
+    if (lane == 0) s_red[warp] = l;
+    __syncthreads();
+    if (warp == 0) {
+      float lt = 0.f, ot[FPL];
+#pragma unroll
+      for (int f = 0; f < FPL; ++f) ot[f] = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        lt += s_red[w];
+#pragma unroll
+        for (int f = 0; f < FPL; ++f) ot[f] += s_o[w][lane * FPL + f];
+      }
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+#pragma unroll
+      for (int f = 0; f < FPL; ++f) o[(size_t)bh * HD + lane * FPL + f] = __float2bfloat16_rn(ot[f] * inv);
+      if (lane == 0) lse[bh] = (mm + __log2f(lt)) * 0.69314718055994531f;
+    }
+    __syncthreads();  // warp 0 has read s_red and s_o before the next row writes them
   }
 }
 

@@ -604,8 +604,12 @@ int check_decode_shape(int B, int Hq, int Hkv, int D, int page_size, int max_pag
   return AXIS_ATTN_OK;
 }
 
-// Splits of each sequence: at least one full wave of CTAs (two per SM) when the
-// batch is small, at least 256 keys (8 pieces, 2 per compute warp) per split.
+// Splits of each sequence: at least 296 items (two per SM) when the batch is
+// small, at least 256 keys (8 pieces) per split.  Measured against filling
+// every CTA that fits at once (740 items): that rule was slower at batch 1-4
+// (more partial results and per-item start-up for the same bytes) and faster
+// only around batch 8 at D = 128.  A pure function of the shape, so that the
+// workspace query needs no device.
 struct DecSplit {
   int n_splits, keys_per_split;
 };
@@ -659,23 +663,44 @@ bool make_cache_map_hnd(CUtensorMap* map, const void* ptr, int num_pages, int pa
 }
 
 // Persistent decode: as many CTAs as fit on the SMs at once (or one per item).
-template <int HD>
-int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev) {
-  auto kern = attn_decode_kernel<HD>;
+template <int HD, bool DEEP>
+int launch_decode_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev,
+                      long long items) {
+  using C = DecCfg<HD, DEEP>;
+  auto kern = attn_decode_kernel<HD, DEEP>;
   static bool done[64];
   static int per_sm[64];
-  if (int rc = set_smem(kern, DecCfg<HD>::SMEM, dev, done)) return rc;
+  if (int rc = set_smem(kern, C::SMEM, dev, done)) return rc;
   if (per_sm[dev] == 0) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, DecCfg<HD>::THREADS, DecCfg<HD>::SMEM) != cudaSuccess || n < 1)
-      n = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, C::THREADS, C::SMEM) != cudaSuccess || n < 1) n = 1;
     per_sm[dev] = n;
   }
-  const long long items = (long long)a.B * a.Hkv * a.n_splits;
   const long long cap = (long long)per_sm[dev] * sm_count(dev);
   const unsigned grid = (unsigned)(items < cap ? items : cap);
-  kern<<<grid, DecCfg<HD>::THREADS, DecCfg<HD>::SMEM, st>>>(mk, mv, a);
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(mk, mv, a);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+}
+
+// Resident CTAs per SM of a configuration, from its shared memory and threads
+// (228 KB per SM, 1 KB reserved per CTA; 2048 threads).
+template <int HD, bool DEEP>
+constexpr int dec_per_sm() {
+  using C = DecCfg<HD, DEEP>;
+  constexpr int by_smem = 233472 / (int)(C::SMEM + 1024), by_threads = 2048 / C::THREADS;
+  return by_smem < by_threads ? by_smem : by_threads;
+}
+
+// The deep configuration when all items fit its CTAs in one wave (a small
+// batch: the wide configuration's extra CTAs would have no item), else the
+// wide one.  Measured (HBM fraction): 296-304 items, deep 0.43-0.56 against
+// wide 0.39-0.51; 512 items, wide 0.80 against deep 0.59.
+template <int HD>
+int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev) {
+  const long long items = (long long)a.B * a.Hkv * a.n_splits;
+  const bool deep = items <= (long long)dec_per_sm<HD, true>() * sm_count(dev);
+  return deep ? launch_decode_cfg<HD, true>(mk, mv, a, st, dev, items)
+              : launch_decode_cfg<HD, false>(mk, mv, a, st, dev, items);
 }
 
 }  // namespace
@@ -732,7 +757,7 @@ int run_decode(const void* q, const void* k_cache, const void* v_cache, const in
   int rc = D == 64 ? launch_decode<64>(mk, mv, a, st, dev) : launch_decode<128>(mk, mv, a, st, dev);
   if (rc || sp.n_splits == 1) return rc;
   const int rows = B * Hq;
-  const unsigned grid = (unsigned)((rows + 7) / 8 < 4096 ? (rows + 7) / 8 : 4096);
+  const unsigned grid = (unsigned)(rows < 148 * 8 ? rows : 148 * 8);  // one CTA per (b, h) row
   if (D == 64)
     attn_decode_combine_kernel<64><<<grid, 256, 0, st>>>(a.part, a.o, lse, rows, sp.n_splits);
   else

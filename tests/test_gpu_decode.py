@@ -6,7 +6,8 @@ sequence's last page hold -1, which the kernel must never touch) and compares
 O and LSE with the tolerances of the other tests (O max abs <= 1e-2, LSE max
 abs <= 1e-4).  Cases cover both head dims, GQA groups 1..8 (including 3),
 page sizes 8..256, ragged lengths (1, around page and piece edges), batches
-that take the split-K path and batches that do not, and bad device-side
+that take the split-K path and batches that do not, both kernel
+configurations (deep for few items, wide for many), and bad device-side
 indices, which must be reported as AXIS_ATTN_ERR_INDEX without an access.
 Every case runs on both pool layouts: [num_pages, page_size, Hkv, D]
 (axis_attn_decode) and the head-major [num_pages, Hkv, page_size, D]
@@ -98,6 +99,10 @@ CASES = [
     # table in several blocks of 32 pieces (3 at 2100 keys, 2 at 1500)
     (40, 8, 8, 64, 2100, 8, [2100, 1, 1024, 1025, 2047, 2048, 2049, 33] * 5),
     (40, 16, 8, 128, 1500, 16, [1500, 1023, 1056, 17, 1499] * 8),
+    # more items than the wide D = 64 configuration's resident CTAs (800 > 740):
+    # the wide kernel, some CTAs walking two items (the cases above with at most
+    # 444 items at D = 64 / 296 at D = 128 run the deep configuration)
+    (200, 8, 4, 64, 300, 16, [300, 1, 17, 256, 299] * 40),
 ]
 
 
