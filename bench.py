@@ -474,13 +474,15 @@ def time_rope(aa, w, seed, dev, steps, flush, p_meas):
 
 # Decode workloads: one new token per sequence against a paged KV cache of
 # `ctx` tokens (the axiomlm model's heads and block size; an 8B-class model),
-# each on both pool layouts: NHD [num_pages, page_size, Hkv, D] and the
-# head-major HND [num_pages, Hkv, page_size, D].
+# each batched one on both pool layouts: NHD [num_pages, page_size, Hkv, D] and
+# the head-major HND [num_pages, Hkv, page_size, D]; and one sequence of 32K
+# tokens (batch 1: the split-K path and the merge kernel, latency-bound).
 DECODE = {
     "decode_gpt2s_gqa": dict(B=256, Hq=12, Hkv=4, D=64, ctx=1024, page=16, layout="NHD"),
     "decode_gpt2s_gqa_hnd": dict(B=256, Hq=12, Hkv=4, D=64, ctx=1024, page=16, layout="HND"),
     "decode_llm8b_gqa": dict(B=32, Hq=32, Hkv=8, D=128, ctx=8192, page=64, layout="NHD"),
     "decode_llm8b_gqa_hnd": dict(B=32, Hq=32, Hkv=8, D=128, ctx=8192, page=64, layout="HND"),
+    "decode_llm8b_b1_32k": dict(B=1, Hq=32, Hkv=8, D=128, ctx=32768, page=64, layout="NHD"),
 }
 
 
@@ -534,6 +536,7 @@ def time_decode(aa, name, dev, steps, flush, hbm_gbs):
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"config": f"B={B} Hq={Hq} Hkv={Hkv} D={D} context={ctx} page_size={page} (bf16 paged cache, "
                       f"{c['layout']} pages, random page order)", "ms": ms, "steps": steps, "algorithmic_bytes": nbytes,
+            "launches_per_call": 2 if need > 0 else 1,  # the decode kernel, and the split merge when it splits
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs}}
 
 
