@@ -335,8 +335,8 @@ class Problem:
                                              Hkv, S, D, w.scale, c, ws, wsb, sp), "bwd_det")
             rec(4)
             return
-        self._check(aa.axis_attn_bwd_prepare(self.o.data_ptr(), do, self.lse.data_ptr(), B, Hq, Hkv, S, D, ws,
-                                             wsb, sp), "bwd_prepare")
+        self._check(aa.axis_attn_bwd_prepare(self.o.data_ptr(), do, self.lse.data_ptr(), B, Hq, Hkv, S, D, w.scale,
+                                             ws, wsb, sp), "bwd_prepare")
         rec(2)
         self._check(aa.axis_attn_bwd_main(q, k, v, do, self.dk.data_ptr(), self.dv.data_ptr(), B, Hq, Hkv, S, D,
                                           w.scale, c, ws, wsb, sp), "bwd_main")

@@ -86,7 +86,7 @@ def load():
             lib.axis_attn_bwd_head_split.restype = i
             lib.axis_attn_bwd.argtypes = [vp] * 9 + [i] * 5 + [f, i, vp, sz, vp]
             lib.axis_attn_bwd.restype = i
-            lib.axis_attn_bwd_prepare.argtypes = [vp] * 3 + [i] * 5 + [vp, sz, vp]
+            lib.axis_attn_bwd_prepare.argtypes = [vp] * 3 + [i] * 5 + [f, vp, sz, vp]
             lib.axis_attn_bwd_prepare.restype = i
             lib.axis_attn_bwd_main.argtypes = [vp] * 6 + [i] * 5 + [f, i, vp, sz, vp]
             lib.axis_attn_bwd_main.restype = i
@@ -141,8 +141,8 @@ def axis_attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, Hq, Hkv, S, D, scale, caus
                                 workspace, workspace_bytes, stream)
 
 
-def axis_attn_bwd_prepare(o, dO, lse, B, Hq, Hkv, S, D, workspace, workspace_bytes, stream) -> int:
-    return load().axis_attn_bwd_prepare(o, dO, lse, B, Hq, Hkv, S, D, workspace, workspace_bytes, stream)
+def axis_attn_bwd_prepare(o, dO, lse, B, Hq, Hkv, S, D, scale, workspace, workspace_bytes, stream) -> int:
+    return load().axis_attn_bwd_prepare(o, dO, lse, B, Hq, Hkv, S, D, scale, workspace, workspace_bytes, stream)
 
 
 def axis_attn_bwd_main(q, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, workspace,

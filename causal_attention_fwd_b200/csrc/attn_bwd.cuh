@@ -8,7 +8,7 @@
 //   dS_ij = P_ij (dP_ij - Dr_i),  dQ_i = scale sum_j dS_ij K_j,
 //   dK_j = scale sum_{h in group} sum_i dS_ij Q_i,  dV_j = sum_{h, i} P_ij dO_i.
 // Design on sm_100a:
-//   * preprocess (HBM-bound): Dr and log2-scaled LSE per row, padded to a
+//   * preprocess (HBM-bound): scale Dr and log2-scaled LSE per row, padded to a
 //     multiple of 128 rows (padding rows get Dr = 0, LSE = +inf, so their P is
 //     exactly 0); zero the fp32 dQ accumulator;
 //   * main kernel: one CTA per (b, kv head, 128-key tile); K_j, V_j stay in
@@ -17,6 +17,8 @@
 //     MMAs, one the score products, one the gradient products):
 //       S^T = K Q^T and dP^T = V dO^T into TMEM (thread = key row),
 //       P^T = 2^(S^T c - LSE2), dS^T = P^T (dP^T - Dr) by 8 warps from TMEM,
+//       formed as scale dS^T = P^T (scale dP^T - scale Dr) (the preprocess
+//       stores -scale Dr), so dQ and dK leave their products scaled,
 //       P^T back to TMEM (bf16), dS^T to shared memory (bf16, 128B swizzle),
 //       dV += P^T dO (A from TMEM), dK += dS^T Q, and dQ of the tile,
 //     the compute warps copy each dQ tile from TMEM into a swizzled
@@ -409,7 +411,6 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
       const int wq = warp & 3;
       const int kr = wq * 32 + lane;
       const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-      const float sc = a.scale;
       for (int t = 0; t < n_it; ++t) {
         if (!wait_warp(bar_dqfull, t & 1, abort, B_DQFULL)) break;
         if (t > 0 && !wait_warp(bar_stgfree, (t - 1) & 1, abort, B_STGFREE)) break;
@@ -427,12 +428,12 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
           }
           if (C::QLANE) {
             // lane = query row kr, columns = features [32 ch, 32 ch + 32): one 128-byte box row
+            // (dQ is already scaled: dS was formed scaled)
             const uint32_t row = sSTG + ((kr >> 6) * 2 + ch) * C::DQ_BOX + (kr & 63) * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-              asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(row + ((c ^ (kr & 7)) << 4)),
-                           "f"(__uint_as_float(v[4 * c]) * sc), "f"(__uint_as_float(v[4 * c + 1]) * sc),
-                           "f"(__uint_as_float(v[4 * c + 2]) * sc), "f"(__uint_as_float(v[4 * c + 3]) * sc)
+              asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(row + ((c ^ (kr & 7)) << 4)),
+                           "r"(v[4 * c]), "r"(v[4 * c + 1]), "r"(v[4 * c + 2]), "r"(v[4 * c + 3])
                            : "memory");
           } else {
             // lane = feature kr (box kr / 32, column kr % 32), columns = query rows 32 ch + e
@@ -440,8 +441,8 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const int q = 32 * ch + e;
-              asm volatile("st.shared.f32 [%0], %1;" ::"r"(boxb + q * 128 + (((lane >> 2) ^ (q & 7)) << 4)),
-                           "f"(__uint_as_float(v[e]) * sc)
+              asm volatile("st.shared.b32 [%0], %1;" ::"r"(boxb + q * 128 + (((lane >> 2) ^ (q & 7)) << 4)),
+                           "r"(v[e])
                            : "memory");
             }
           }
@@ -459,6 +460,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int c0 = ch * COLS;
     const uint64_t cc2 = f2_pack(a.scale_log2, a.scale_log2);
+    const uint64_t sc2 = f2_pack(a.scale, a.scale);  // dS is formed scaled: P (scale dP - scale Dr)
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int s = it % ST;
@@ -517,7 +519,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
             }
             const uint64_t pp = f2_pack(p0, p1);
             const uint64_t dd =
-                f2_mul(pp, f2_add(f2_pack(__uint_as_float(dpv[ee]), __uint_as_float(dpv[ee + 1])), nd));
+                f2_mul(pp, f2_fma(f2_pack(__uint_as_float(dpv[ee]), __uint_as_float(dpv[ee + 1])), sc2, nd));
             pk[ee / 2] = pack_bf16x2(pp);
             dk[ee / 2] = pack_bf16x2(dd);
           }
@@ -547,14 +549,14 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
       if (lane == 0 && !(AXIS_ATTN_TEST_DROP_ARRIVE == 2 && it == 0)) mbar_arrive(bar_pdsfull);
     }
     // epilogue: the first half of the column groups writes dV, the second dK
-    // (x scale); with 16 warps each group takes half of the features
+    // (already scaled: dS was formed scaled); with 16 warps each group takes
+    // half of the features
     constexpr int NG = BWD_CW / 4, GPT = NG / 2;  // column groups, groups per tensor
     if (ok && wait_warp(bar_fin, 0, abort, B_FIN)) {
       tc_fence_after();
       const bool is_dv = ch < GPT;
       const int f0 = (ch % GPT) * (HD / GPT);  // first feature of this group
       const uint32_t tcol = (is_dv ? C::T_DV : C::T_DK) + f0;
-      const float mul = is_dv ? 1.f : a.scale;
       const size_t row_off = (((size_t)b * a.S + key) * a.Hkv + kvh) * HD + f0;
       __nv_bfloat16* dst_row = (is_dv ? a.dv : a.dk) + row_off;
       float* part_row = a.hsplit > 1 ? (is_dv ? a.dv_part : a.dk_part) + (size_t)hs * a.B * a.S * a.Hkv * HD + row_off
@@ -569,8 +571,8 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
             float4* dst = reinterpret_cast<float4*>(part_row + cc * 32);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(v[4 * i]) * mul, __uint_as_float(v[4 * i + 1]) * mul,
-                                   __uint_as_float(v[4 * i + 2]) * mul, __uint_as_float(v[4 * i + 3]) * mul);
+              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
           }
           continue;
         }
@@ -580,14 +582,14 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
           const double2* t = a.rope_cs + (size_t)key * (HD / 2) + (f0 + 32 * cc) / 2;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            float g0 = __uint_as_float(v[2 * i]) * mul, g1 = __uint_as_float(v[2 * i + 1]) * mul;
+            float g0 = __uint_as_float(v[2 * i]), g1 = __uint_as_float(v[2 * i + 1]);
             rope_back(g0, g1, t[i]);
             pk2[i] = pack_bf16x2(g0, g1);
           }
         } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            pk2[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+            pk2[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
         }
         if (key < a.S) {
           uint4* dst = reinterpret_cast<uint4*>(dst_row + cc * 32);
@@ -606,7 +608,8 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
   }
 }
 
-// -Dr = -rowsum(dO * O) (fp32) and -LSE2 = -LSE * log2(e) per (b, h, i); rows
+// -scale Dr = -scale rowsum(dO * O) (fp32) and -LSE2 = -LSE * log2(e) per
+// (b, h, i) (the backward forms dS scaled: P (scale dP - scale Dr)); rows
 // S..S_pad-1 of each (b, h) get 0 and -inf (so their P is exactly 0).  Also
 // zeroes the dQ accumulator.  HBM-bound: D/8 threads per row with one 16-byte
 // load each of O and dO (every row a whole 128- or 256-byte line) and a shuffle
@@ -619,7 +622,7 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
                                                             const __nv_bfloat16* __restrict__ dout,
                                                             const float* __restrict__ lse, float* nlse2,
                                                             float* ndr, float4* dqacc, size_t dq_vec4,
-                                                            int Hq, int S, int S_pad, int rows) {
+                                                            int Hq, int S, int S_pad, int rows, float scale) {
   constexpr int TPR = HD / 8;  // threads per row
   const size_t gtid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t nthreads = (size_t)gridDim.x * blockDim.x;
@@ -650,7 +653,7 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off, TPR);
     if (act && part == 0) {
-      ndr[bh * S_pad + i] = -d;
+      ndr[bh * S_pad + i] = -d * scale;
       nlse2[bh * S_pad + i] = -lse[bh * S + i] * 1.4426950408889634f;
     }
   }

@@ -1,7 +1,8 @@
 // attn_bwd_dq.cuh -- deterministic dQ pass of the backward: one CTA per
 // (b, query head, 128-row query tile) recomputes, for every key tile the rows
-// see, S = Q K^T, P = 2^(S c - LSE2) and dS = P (dP - Dr) with dP = dO V^T,
-// and accumulates dQ = scale * sum_j dS_j K_j in tensor memory, in the fixed
+// see, S = Q K^T, P = 2^(S c - LSE2) and scale dS = P (scale dP - scale Dr)
+// with dP = dO V^T, and accumulates dQ = sum_j (scale dS_j) K_j in tensor
+// memory, in the fixed
 // order of the key tiles.  No cross-CTA additions: the result is bitwise the
 // same from run to run, and the only scratch is the per-row LSE2 and Dr of
 // the preprocess (O(B Hq S) floats), so memory stays flat as S grows.
@@ -27,7 +28,7 @@ namespace axis_attn {
 struct DqArgs {
   __nv_bfloat16* dq;   // [B, S, Hq, HD]
   const float* nlse2;  // [B*Hq][S_pad]  -LSE * log2(e); -inf on padding rows
-  const float* ndr;    // [B*Hq][S_pad]  -rowsum(dO * O); 0 on padding rows
+  const float* ndr;    // [B*Hq][S_pad]  -scale rowsum(dO * O); 0 on padding rows
   int B, Hq, Hkv, S, S_pad;
   float scale, scale_log2;
   const double2* rope_cs;  // RoPE: (cos, sin) table [S][HD/2], fp64; dQ leaves through the transposed rotation
@@ -215,6 +216,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
     const float ndr = a.ndr[(size_t)bh * a.S_pad + row_g];
     const uint64_t cc2 = f2_pack(a.scale_log2, a.scale_log2);
     const uint64_t nl2_2 = f2_pack(nl2, nl2), ndr2 = f2_pack(ndr, ndr);
+    const uint64_t sc2 = f2_pack(a.scale, a.scale);  // dS formed scaled: P (scale dP - scale Dr)
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       if (!wait_warp<true>(bar_sfull, j & 1, abort, Q_SFULL)) { ok = false; break; }
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
           if (2 * e + 1 >= limit) p1 = 0.f;
         }
         const uint64_t ds =
-            f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1])), ndr2));
+            f2_mul(f2_pack(p0, p1), f2_fma(f2_pack(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1])), sc2, ndr2));
         pk[e] = pack_bf16x2(ds);
       }
       // dS into its buffer (the dQ MMA of j - NDS must be done with it)
@@ -263,7 +265,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_dsfull(x));
     }
-    // epilogue: dQ * scale -> bf16, this thread's HD / 4 columns of its row
+    // epilogue: dQ (already scaled) -> bf16, this thread's HD / 4 columns of its row
     if (ok && wait_warp<true>(bar_fin, 0, abort, Q_FIN)) {
       tc_fence_after();
       constexpr int NC = HD / 4;  // 16 or 32 columns
@@ -292,10 +294,10 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         uint4* dst = reinterpret_cast<uint4*>(a.dq + (((size_t)b * a.S + row_g) * a.Hq + h) * HD + NC * qc);
 #pragma unroll
         for (int i = 0; i < NC / 8; ++i)
-          dst[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]) * a.scale, __uint_as_float(v[8 * i + 1]) * a.scale),
-                              pack_bf16x2(__uint_as_float(v[8 * i + 2]) * a.scale, __uint_as_float(v[8 * i + 3]) * a.scale),
-                              pack_bf16x2(__uint_as_float(v[8 * i + 4]) * a.scale, __uint_as_float(v[8 * i + 5]) * a.scale),
-                              pack_bf16x2(__uint_as_float(v[8 * i + 6]) * a.scale, __uint_as_float(v[8 * i + 7]) * a.scale));
+          dst[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                              pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                              pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                              pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
       }
     }
   }

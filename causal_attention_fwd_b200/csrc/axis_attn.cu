@@ -285,10 +285,10 @@ WsPtrs ws_ptrs(void* workspace, const WsLayout& w) {
 
 namespace {
 
-// Stage 1: -Dr and -LSE*log2(e) rows (padding rows 0 / -inf); zero the dQ
-// accumulator unless the deterministic mode's slices are used.
-int run_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, int S, int D, const WsLayout& w,
-                const WsPtrs& p, bool zero_dq, cudaStream_t st) {
+// Stage 1: -scale*Dr and -LSE*log2(e) rows (padding rows 0 / -inf); zero the
+// dQ accumulator unless the deterministic mode's slices are used.
+int run_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, int S, int D, float scale,
+                const WsLayout& w, const WsPtrs& p, bool zero_dq, cudaStream_t st) {
   const int rows = B * Hq * w.S_pad;
   const size_t dq_vec4 = zero_dq ? (size_t)B * Hq * S * D / 4 : 0;
   // grid-stride kernel: a few waves of 256-thread blocks over the 148 SMs
@@ -298,10 +298,10 @@ int run_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, 
   const auto* db = static_cast<const __nv_bfloat16*>(dO);
   if (D == 64)
     attn_bwd_prep_kernel<64><<<grid, 256, 0, st>>>(ob, db, lse, p.lse2, p.dr, reinterpret_cast<float4*>(p.dqacc),
-                                                   dq_vec4, Hq, S, w.S_pad, rows);
+                                                   dq_vec4, Hq, S, w.S_pad, rows, scale);
   else
     attn_bwd_prep_kernel<128><<<grid, 256, 0, st>>>(ob, db, lse, p.lse2, p.dr, reinterpret_cast<float4*>(p.dqacc),
-                                                    dq_vec4, Hq, S, w.S_pad, rows);
+                                                    dq_vec4, Hq, S, w.S_pad, rows, scale);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 
@@ -373,15 +373,17 @@ int run_finalize(void* dq, int B, int Hq, int S, int D, const WsPtrs& p, cudaStr
 }  // namespace
 
 extern "C" int axis_attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, int Hkv,
-                                     int S, int D, void* workspace, size_t workspace_bytes, void* stream) {
+                                     int S, int D, float scale, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
   if (!o || !dO || !lse) return AXIS_ATTN_ERR_NULL;
   if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return AXIS_ATTN_ERR_ALIGN;
-  if (int rc = check_shape(B, Hq, Hkv, S, D, 1.f)) return rc;
+  if (int rc = check_shape(B, Hq, Hkv, S, D, scale)) return rc;
   const WsLayout w = ws_layout(B, Hq, Hkv, S, D);
   if (int rc = check_ws(workspace, workspace_bytes, w)) return rc;
   int dev = 0;
   if (int rc = check_device(&dev)) return rc;
-  return run_prepare(o, dO, lse, B, Hq, S, D, w, ws_ptrs(workspace, w), true, static_cast<cudaStream_t>(stream));
+  return run_prepare(o, dO, lse, B, Hq, S, D, scale, w, ws_ptrs(workspace, w), true,
+                     static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int axis_attn_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
@@ -457,7 +459,7 @@ int run_bwd(const void* q, const void* k, const void* v, const void* o, const vo
   if (int rc = check_device(&dev)) return rc;
   const WsPtrs p = ws_ptrs(workspace, w);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (int rc = run_prepare(o, dO, lse, B, Hq, S, D, w, p, !det, st)) return rc;
+  if (int rc = run_prepare(o, dO, lse, B, Hq, S, D, scale, w, p, !det, st)) return rc;
   if (int rc = run_main(q, k, v, dO, dk, dv, B, Hq, Hkv, S, D, scale, causal, w, p, det, st, dev, rope_cs))
     return rc;
   if (det) return run_dq_pass(q, k, v, dO, dq, B, Hq, Hkv, S, D, scale, causal, w, p, st, dev, rope_cs);

@@ -116,15 +116,18 @@ int axis_attn_bwd(const void* q, const void* k, const void* v, const void* o,
  * for axis_attn_bwd() and are validated the same way; the workspace carries the
  * state from one stage to the next, so all three must get the same workspace
  * and sizes, in this order, with nothing writing the workspace in between.
- *   prepare:  Dr = rowsum(dO * O) and LSE * log2(e) into the workspace; zeroes
- *             the fp32 dQ accumulator.  Reads o, dO, lse.
+ *   prepare:  scale * Dr = scale * rowsum(dO * O) and LSE * log2(e) into the
+ *             workspace (the main stage forms dS already multiplied by scale,
+ *             so prepare and main must get the same scale); zeroes the fp32 dQ
+ *             accumulator.  Reads o, dO, lse.
  *   main:     dk, dv (written) and the dQ accumulator (added into).  Reads q, k,
  *             v, dO and the workspace.  (With a head split, a second kernel
  *             adds up the partial dK, dV.)
  *   finalize: dq = bf16(dQ accumulator).
  */
 int axis_attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, int Hkv,
-                          int S, int D, void* workspace, size_t workspace_bytes, void* stream);
+                          int S, int D, float scale, void* workspace, size_t workspace_bytes,
+                          void* stream);
 int axis_attn_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk,
                        void* dv, int B, int Hq, int Hkv, int S, int D, float scale, int causal,
                        void* workspace, size_t workspace_bytes, void* stream);
