@@ -291,9 +291,11 @@ int run_prepare(const void* o, const void* dO, const float* lse, int B, int Hq, 
                 const WsLayout& w, const WsPtrs& p, bool zero_dq, cudaStream_t st) {
   const int rows = B * Hq * w.S_pad;
   const size_t dq_vec4 = zero_dq ? (size_t)B * Hq * S * D / 4 : 0;
-  // grid-stride kernel: a few waves of 256-thread blocks over the 148 SMs
+  // grid-stride kernel: a few waves of 256-thread blocks over the 148 SMs, twice
+  // as many when half of them zero the accumulator
   const size_t work = (size_t)B * Hq * S * (D / 8);
-  const unsigned grid = (unsigned)((work + 255) / 256 < 148 * 16 ? (work + 255) / 256 : 148 * 16);
+  unsigned grid = (unsigned)((work + 255) / 256 < 148 * 16 ? (work + 255) / 256 : 148 * 16);
+  if (dq_vec4 > 0) grid *= 2;
   const auto* ob = static_cast<const __nv_bfloat16*>(o);
   const auto* db = static_cast<const __nv_bfloat16*>(dO);
   if (D == 64)

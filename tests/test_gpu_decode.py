@@ -103,6 +103,9 @@ CASES = [
     # the wide kernel, some CTAs walking two items (the cases above with at most
     # 444 items at D = 64 / 296 at D = 128 run the deep configuration)
     (200, 8, 4, 64, 300, 16, [300, 1, 17, 256, 299] * 40),
+    # 128 splits of 256 keys (more than the merge kernel's 32 splits per pass of
+    # its warps), the last 10 past the end of the sequence (weight 0)
+    (1, 4, 2, 64, 32768, 16, [30001]),
 ]
 
 
