@@ -43,6 +43,17 @@ namespace axis_attn {
 // latencies of a step; measured 11% faster than 8 at D = 64) or 8 (two per
 // sub-partition, half of the columns in 32-column chunks: at D = 128 a step
 // has only 64 query columns, and 16 columns a thread measured 5% slower).
+// Q / dO ring depth and dS^T buffers at D = 64 (D = 128: 3 and 1).  Two dS^T
+// buffers let the compute warps write a step's dS^T while the dK and dQ
+// products of the previous step still read theirs; they fit shared memory only
+// with a 2-deep ring.  Measured (llm1b main kernel, same box): 3 / 1 251.5 us,
+// 2 / 1 264.2 us, 2 / 2 270.0 us: the ring depth matters more than that wait.
+#ifndef AXIS_ATTN_BWD_ST64
+#define AXIS_ATTN_BWD_ST64 3
+#endif
+#ifndef AXIS_ATTN_BWD_NDS64
+#define AXIS_ATTN_BWD_NDS64 1
+#endif
 #ifndef AXIS_ATTN_BWD_CW64
 #define AXIS_ATTN_BWD_CW64 16
 #endif
@@ -83,7 +94,8 @@ struct BwdCfg {
   static constexpr uint32_t QSLAB = BM * 128;      // BM query rows x 128 bytes
   static constexpr uint32_t QTILE = NSLAB * QSLAB;
   static constexpr uint32_t PS_BYTES = (BM / 64) * 128 * 128;  // dS^T: 128 keys x BM bf16
-  static constexpr int ST = 3;                     // Q / dO / LSE / Dr ring depth
+  static constexpr int ST = HD == 64 ? AXIS_ATTN_BWD_ST64 : 3;    // Q / dO / LSE / Dr ring depth
+  static constexpr int NDS = HD == 64 ? AXIS_ATTN_BWD_NDS64 : 1;  // dS^T buffers
   // warps: 0 .. CW-1 compute; CW loads; CW+1 score MMAs (and TMEM owner);
   // CW+2 TMA reduce-adds; CW+3 gradient MMAs; CW+4 .. CW+7 dQ read-out
   static constexpr int CW = HD == 64 ? AXIS_ATTN_BWD_CW64 : AXIS_ATTN_BWD_CW128;
@@ -104,11 +116,11 @@ struct BwdCfg {
   static constexpr uint32_t OFF_Q = 2 * KTILE;
   static constexpr uint32_t OFF_DO = OFF_Q + ST * QTILE;
   static constexpr uint32_t OFF_DST = OFF_DO + ST * QTILE;
-  static constexpr uint32_t OFF_STG = OFF_DST + PS_BYTES;
+  static constexpr uint32_t OFF_STG = OFF_DST + NDS * PS_BYTES;
   static constexpr uint32_t OFF_LSE = OFF_STG + STAGE_BYTES;
   static constexpr uint32_t OFF_DR = OFF_LSE + ST * BM * 4;
   static constexpr uint32_t OFF_BAR = OFF_DR + ST * BM * 4;
-  static constexpr int NBAR = 20;
+  static constexpr int NBAR = 13 + 2 * ST;
   static constexpr uint32_t SMEM = OFF_BAR + 8 * NBAR + 16 + 1024;
   static_assert(SMEM <= 232448, "shared memory budget");
   // TMEM columns: S^T, dP^T, dV, dK, dQ tile, P^T (bf16 pairs)
@@ -204,7 +216,9 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
   const uint32_t bar_dqfull = bars + 8u * (5 + 2 * ST);   // dQ tile of a step is in TMEM
   const uint32_t bar_dqfree = bars + 8u * (6 + 2 * ST);   // ... and has been read (8 warps)
   const uint32_t bar_fin = bars + 8u * (7 + 2 * ST);
-  const uint32_t bar_dstfree = bars + 8u * (8 + 2 * ST);  // dK, dQ of a step are done with dS^T
+  // dK, dQ of a step are done with dS^T buffer x
+  auto bar_dstfree = [&](int x) { return bars + 8u * (x == 0 ? 8 + 2 * ST : 11 + 2 * ST); };
+  auto sDSB = [&](int it) { return sDST + (uint32_t)(it % C::NDS) * C::PS_BYTES; };  // dS^T buffer of step it
   const uint32_t bar_stgfull = bars + 8u * (9 + 2 * ST);  // dQ tile staged (8 warps)
   const uint32_t bar_stgfree = bars + 8u * (10 + 2 * ST); // staged tile read by the TMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 8 * C::NBAR);
@@ -240,7 +254,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
     mbar_init(bar_dqfull, 1);
     mbar_init(bar_dqfree, 4);
     mbar_init(bar_fin, 2);
-    mbar_init(bar_dstfree, 1);
+    for (int x = 0; x < C::NDS; ++x) mbar_init(bar_dstfree(x), 1);
     mbar_init(bar_stgfull, 4);
     mbar_init(bar_stgfree, 1);
     wait_ctl_init(abort);
@@ -352,12 +366,12 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t po = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss_w(tmem + C::T_DK, sw128_desc(sDST + po, 16, 1024), sw128_desc(sQ(s) + kk * 2048, C::QSLAB, 1024),
+          mma_ss_w(tmem + C::T_DK, sw128_desc(sDSB(it) + po, 16, 1024), sw128_desc(sQ(s) + kk * 2048, C::QSLAB, 1024),
                    ID_GV, (it > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit_w(bar_qempty(s));  // this warp is done with Q, dO of the step
         if (a.no_dq) {  // dQ comes from the separate deterministic pass
-          mma_commit_w(bar_dstfree);
+          mma_commit_w(bar_dstfree(it % C::NDS));
           continue;
         }
         // dQ tile (reduction over the 128 keys) once the previous one has been read
@@ -365,7 +379,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ds_mn = sw128_desc(sDST + kk * 2048, 128 * 128, 1024);
+          const uint64_t ds_mn = sw128_desc(sDSB(it) + kk * 2048, 128 * 128, 1024);
           const uint64_t k_mn = sw128_desc(sK + kk * 2048, C::KSLAB, 1024);
           if (C::QLANE)
             mma_ss_w(tmem + C::T_DQ, ds_mn, k_mn, ID_Q, kk > 0);   // dQ = dS K
@@ -373,7 +387,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
             mma_ss_w(tmem + C::T_DQ, k_mn, ds_mn, ID_Q, kk > 0);   // dQ^T = K^T dS^T
         }
         mma_commit_w(bar_dqfull);
-        mma_commit_w(bar_dstfree);
+        mma_commit_w(bar_dstfree(it % C::NDS));
       }
     }
     // Drain: all MMAs issued by this warp complete before TMEM is freed.
@@ -534,12 +548,14 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
         else
           tmem_st8(tmem + lane_off + C::T_P + (c0 >> 1) + (SUBW / 2) * cc, pk);
         // ... and the previous step's dK, dQ with dS^T
-        if (cc == 0 && it > 0 && !wait_warp(bar_dstfree, (it - 1) & 1, abort, B_PDSFREE)) {
+        // (with two buffers: the step before the previous one's)
+        if (cc == 0 && it >= C::NDS &&
+            !wait_warp(bar_dstfree(it % C::NDS), ((it - C::NDS) / C::NDS) & 1, abort, B_PDSFREE)) {
           ok = false;
           break;
         }
 #pragma unroll
-        for (int x = 0; x < SUBW / 16; ++x) store_row16(sDST, kr, c0 + SUBW * cc + 16 * x, &dk[8 * x]);
+        for (int x = 0; x < SUBW / 16; ++x) store_row16(sDSB(it), kr, c0 + SUBW * cc + 16 * x, &dk[8 * x]);
       }
       if (!ok) break;
       tmem_wait_st();
