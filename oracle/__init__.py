@@ -6,6 +6,7 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 from .oracle import (  # noqa: F401
     attn_bwd,
     attn_decode,
+    attn_decode_q,
     attn_bwd_dkdv_rows,
     attn_bwd_dq_rows,
     attn_fwd,

@@ -457,6 +457,59 @@ int oracle_attn_decode(const double* q, const double* k, const double* v, const 
     return 0;
 }
 
+/*
+ * Decode step with q_len new tokens per sequence at once (q_len = 1 is
+ * oracle_attn_decode): the decode engine of the axiomlm page (Key Features,
+ * "State-cached Key-Value (KV) decode engine"; Quick Start section 4) advancing
+ * several positions in one step -- a chunk of a prompt appended to the cache,
+ * or several proposed tokens checked together.  The new tokens are the last
+ * q_len positions of their sequence, so new token t of sequence b sits at
+ * position p = lens[b] - q_len + t and, under the causal mask, sees the cached
+ * keys j <= p (the earlier new tokens and itself included, the later ones
+ * not):
+ *   s_j = scale * sum_d q[b,t,h,d] K[b,j,kv,d]   for j <= p, kv = h / G
+ *   o[b,t,h,:] = sum_j softmax(s)_j V[b,j,kv,:]   lse[b,h,t] = ln sum_j exp(s_j)
+ * q, o: [B, q_len, Hq, D]; k, v: [B, Smax, Hkv, D], of which sequence b uses its
+ * first lens[b] rows (q_len <= lens[b] <= Smax); lse: [B, Hq, q_len].  Returns
+ * 0, or -1 for bad sizes.
+ */
+int oracle_attn_decode_q(const double* q, const double* k, const double* v, const int* lens,
+                         double* o, double* lse, int B, int q_len, int Hq, int Hkv, int Smax, int D,
+                         double scale) {
+    if (B < 1 || q_len < 1 || Hq < 1 || Hkv < 1 || Smax < 1 || D < 1 || Hq % Hkv) return -1;
+    for (int b = 0; b < B; ++b)
+        if (lens[b] < q_len || lens[b] > Smax) return -1;
+    const int G = Hq / Hkv;
+#pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)Smax);
+#pragma omp for collapse(3) schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b)
+            for (int t = 0; t < q_len; ++t)
+                for (int h = 0; h < Hq; ++h) {
+                    const int kv = h / G, p = lens[b] - q_len + t;  /* this token's position */
+                    const double* qh = q + (((size_t)b * q_len + t) * Hq + h) * D;
+                    double m = -INFINITY;
+                    for (int j = 0; j <= p; ++j) {
+                        s[j] = scale * dot(qh, k + (((size_t)b * Smax + j) * Hkv + kv) * D, D);
+                        if (s[j] > m) m = s[j];
+                    }
+                    double l = 0.0;
+                    for (int j = 0; j <= p; ++j) l += exp(s[j] - m);
+                    double* oh = o + (((size_t)b * q_len + t) * Hq + h) * D;
+                    for (int d = 0; d < D; ++d) oh[d] = 0.0;
+                    for (int j = 0; j <= p; ++j) {
+                        const double pj = exp(s[j] - m) / l;
+                        const double* vj = v + (((size_t)b * Smax + j) * Hkv + kv) * D;
+                        for (int d = 0; d < D; ++d) oh[d] += pj * vj[d];
+                    }
+                    lse[((size_t)b * Hq + h) * q_len + t] = m + log(l);
+                }
+        free(s);
+    }
+    return 0;
+}
+
 /* Threads OpenMP will use (1 when built without OpenMP). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

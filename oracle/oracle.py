@@ -85,9 +85,10 @@ class Oracle:
         lib.oracle_attn_bwd_dkdv_rows.argtypes = [_dp] * 4 + dims + [i, _ip, _dp, _dp]
         lib.oracle_rope.argtypes = [_dp, i, i, i, i, d, i]
         lib.oracle_attn_decode.argtypes = [_dp] * 3 + [_ip] + [_dp] * 2 + [i] * 5 + [d]
+        lib.oracle_attn_decode_q.argtypes = [_dp] * 3 + [_ip] + [_dp] * 2 + [i] * 6 + [d]
         for f in ("oracle_attn_fwd", "oracle_attn_fwd_rows", "oracle_attn_probs_row",
                   "oracle_attn_bwd", "oracle_attn_bwd_dq_rows", "oracle_attn_bwd_dkdv_rows",
-                  "oracle_rope", "oracle_attn_decode", "oracle_max_threads"):
+                  "oracle_rope", "oracle_attn_decode", "oracle_attn_decode_q", "oracle_max_threads"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
 
@@ -119,6 +120,25 @@ class Oracle:
                                          B, Hq, Hkv, Smax, D, float(scale))
         if rc:
             raise ValueError("oracle_attn_decode rejected the arguments")
+        return o, lse
+
+    def attn_decode_q(self, q, k, v, lens, scale: float):
+        """Decode step with several new tokens per sequence: q [B, q_len, Hq, D]
+        (the last q_len positions of each sequence), cache k, v [B, Smax, Hkv,
+        D] of which sequence b uses its first lens[b] rows (the new tokens'
+        included).  Returns (O [B, q_len, Hq, D], LSE [B, Hq, q_len]), float64."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, q_len, Hq, D = q.shape
+        Bk, Smax, Hkv, Dk = k.shape
+        if (B, D) != (Bk, Dk) or v.shape != k.shape:
+            raise ValueError(f"incompatible shapes q{q.shape} k{k.shape} v{v.shape}")
+        ln = np.ascontiguousarray(np.asarray(lens, dtype=np.int32).reshape(-1))
+        o = np.empty((B, q_len, Hq, D))
+        lse = np.empty((B, Hq, q_len))
+        rc = self.lib.oracle_attn_decode_q(_ptr(q), _ptr(k), _ptr(v), ln.ctypes.data_as(_ip), _ptr(o), _ptr(lse),
+                                           B, q_len, Hq, Hkv, Smax, D, float(scale))
+        if rc:
+            raise ValueError("oracle_attn_decode_q rejected the arguments")
         return o, lse
 
     def attn_fwd(self, q, k, v, scale: float, causal: bool = True):
@@ -226,3 +246,4 @@ attn_bwd_dq_rows = _forward("attn_bwd_dq_rows")
 attn_bwd_dkdv_rows = _forward("attn_bwd_dkdv_rows")
 rope = _forward("rope")
 attn_decode = _forward("attn_decode")
+attn_decode_q = _forward("attn_decode_q")
