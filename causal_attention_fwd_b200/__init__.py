@@ -25,6 +25,8 @@ from .binding import (  # noqa: F401
     axis_attn_bwd_head_split,
     axis_attn_decode,
     axis_attn_decode_hnd,
+    axis_attn_decode_q,
+    axis_attn_decode_q_workspace_bytes,
     axis_attn_decode_workspace_bytes,
     axis_attn_fwd,
     axis_attn_fwd_rope,

@@ -36,6 +36,8 @@ EXPORTS = (
     "axis_attn_decode_workspace_bytes",
     "axis_attn_decode",
     "axis_attn_decode_hnd",
+    "axis_attn_decode_q",
+    "axis_attn_decode_q_workspace_bytes",
     "axis_attn_get_status",
     "axis_attn_last_status_word",
     "axis_attn_strerror",
@@ -112,6 +114,10 @@ def load():
             lib.axis_attn_decode.restype = i
             lib.axis_attn_decode_hnd.argtypes = [vp] * 7 + [i] * 7 + [f, vp, sz, vp]
             lib.axis_attn_decode_hnd.restype = i
+            lib.axis_attn_decode_q.argtypes = [vp] * 7 + [i] * 8 + [f, i, vp, sz, vp]
+            lib.axis_attn_decode_q.restype = i
+            lib.axis_attn_decode_q_workspace_bytes.argtypes = [i] * 7
+            lib.axis_attn_decode_q_workspace_bytes.restype = sz
             lib.axis_attn_get_status.argtypes = [vp]
             lib.axis_attn_get_status.restype = i
             lib.axis_attn_last_status_word.argtypes = []
@@ -209,6 +215,18 @@ def axis_attn_decode_hnd(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, 
     """Decode step against a head-major paged KV cache (see include/axis_attn.h)."""
     return load().axis_attn_decode_hnd(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
                                        max_pages, num_pages, scale, workspace, workspace_bytes, stream)
+
+
+def axis_attn_decode_q_workspace_bytes(B, q_len, Hq, Hkv, D, page_size, max_pages) -> int:
+    return int(load().axis_attn_decode_q_workspace_bytes(B, q_len, Hq, Hkv, D, page_size, max_pages))
+
+
+def axis_attn_decode_q(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, q_len, Hq, Hkv, D, page_size,
+                       max_pages, num_pages, scale, head_major, workspace, workspace_bytes, stream) -> int:
+    """Decode step with q_len new tokens per sequence (see include/axis_attn.h)."""
+    return load().axis_attn_decode_q(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, q_len, Hq, Hkv, D,
+                                     page_size, max_pages, num_pages, scale, head_major, workspace, workspace_bytes,
+                                     stream)
 
 
 def axis_attn_get_status(stream) -> int:
@@ -425,27 +443,35 @@ def attention_backward_rope(q_rot, k_rot, v, cs, o, lse, dout, causal: bool = Tr
 
 def attention_decode(q, k_cache, v_cache, block_table, seq_lens, scale: float | None = None, out=None,
                      lse=None, workspace=None, stream=None, layout: str = "NHD"):
-    """Decode step: q [B, Hq, D] bf16, k_cache / v_cache [num_pages, page_size,
-    Hkv, D] bf16 (layout "NHD") or [num_pages, Hkv, page_size, D] (layout
-    "HND"), block_table [B, max_pages] int32, seq_lens [B] int32, all on one
-    CUDA device.  Returns (o [B, Hq, D] bf16, lse [B, Hq] fp32)."""
+    """Decode step: q [B, Hq, D] bf16 (one new token per sequence) or
+    [B, q_len, Hq, D] (the last q_len positions of each sequence),
+    k_cache / v_cache [num_pages, page_size, Hkv, D] bf16 (layout "NHD") or
+    [num_pages, Hkv, page_size, D] (layout "HND"), block_table [B, max_pages]
+    int32, seq_lens [B] int32 (the new tokens included), all on one CUDA
+    device.  Returns (o shaped like q, bf16; lse [B, Hq] or [B, Hq, q_len],
+    fp32)."""
     import torch
 
     where = "attention_decode"
     _require(layout in ("NHD", "HND"), ERR_SHAPE, where, "layout must be 'NHD' or 'HND'")
     hnd = layout == "HND"
     dims = "[num_pages, Hkv, page_size, D]" if hnd else "[num_pages, page_size, Hkv, D]"
-    _require(isinstance(q, torch.Tensor) and q.dim() == 3, ERR_SHAPE, where, "q must be a 3-D tensor [B, Hq, D]")
+    _require(isinstance(q, torch.Tensor) and q.dim() in (3, 4), ERR_SHAPE, where,
+             "q must be a 3-D tensor [B, Hq, D] or a 4-D tensor [B, q_len, Hq, D]")
     _require(isinstance(k_cache, torch.Tensor) and k_cache.dim() == 4, ERR_SHAPE, where,
              f"k_cache must be a 4-D tensor {dims}")
-    B, Hq, D = q.shape
+    multi = q.dim() == 4
+    if multi:
+        B, q_len, Hq, D = q.shape
+    else:
+        (B, Hq, D), q_len = q.shape, 1
     if hnd:
         num_pages, Hkv, page_size, _ = k_cache.shape
         cache_shape = (num_pages, Hkv, page_size, D)
     else:
         num_pages, page_size, Hkv, _ = k_cache.shape
         cache_shape = (num_pages, page_size, Hkv, D)
-    _check_tensor(q, "q", (B, Hq, D), torch.bfloat16, where)
+    _check_tensor(q, "q", tuple(q.shape), torch.bfloat16, where)
     _check_tensor(k_cache, "k_cache", cache_shape, torch.bfloat16, where)
     _check_tensor(v_cache, "v_cache", cache_shape, torch.bfloat16, where)
     _require(isinstance(block_table, torch.Tensor) and block_table.dim() == 2, ERR_SHAPE, where,
@@ -454,26 +480,33 @@ def attention_decode(q, k_cache, v_cache, block_table, seq_lens, scale: float | 
     _check_tensor(block_table, "block_table", (B, max_pages), torch.int32, where)
     _check_tensor(seq_lens, "seq_lens", (B,), torch.int32, where)
     named = {"q": q, "k_cache": k_cache, "v_cache": v_cache, "block_table": block_table, "seq_lens": seq_lens}
+    lse_shape = (B, Hq, q_len) if multi else (B, Hq)
     if out is not None:
-        _check_tensor(out, "out", (B, Hq, D), torch.bfloat16, where)
+        _check_tensor(out, "out", tuple(q.shape), torch.bfloat16, where)
         named["out"] = out
     if lse is not None:
-        _check_tensor(lse, "lse", (B, Hq), torch.float32, where)
+        _check_tensor(lse, "lse", lse_shape, torch.float32, where)
         named["lse"] = lse
     dev = _check_device(named, where)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    need = axis_attn_decode_workspace_bytes(B, Hq, Hkv, D, page_size, max_pages)
+    need = (axis_attn_decode_q_workspace_bytes(B, q_len, Hq, Hkv, D, page_size, max_pages) if multi
+            else axis_attn_decode_workspace_bytes(B, Hq, Hkv, D, page_size, max_pages))
     with torch.cuda.device(dev):
         o = torch.empty_like(q) if out is None else out
-        l = torch.empty((B, Hq), device=dev, dtype=torch.float32) if lse is None else lse
+        l = torch.empty(lse_shape, device=dev, dtype=torch.float32) if lse is None else lse
         if workspace is None and need > 0:
             workspace = torch.empty(need, device=dev, dtype=torch.uint8)
         wp = workspace.data_ptr() if workspace is not None else None
         wb = workspace.numel() * workspace.element_size() if workspace is not None else 0
-        call = axis_attn_decode_hnd if hnd else axis_attn_decode
-        rc = call(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
-                  o.data_ptr(), l.data_ptr(), B, Hq, Hkv, D, page_size, max_pages, num_pages, scale, wp, wb,
-                  _stream(stream, dev))
+        ptrs = (q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
+                o.data_ptr(), l.data_ptr())
+        if multi:
+            call = axis_attn_decode_q
+            rc = call(*ptrs, B, q_len, Hq, Hkv, D, page_size, max_pages, num_pages, scale, int(hnd), wp, wb,
+                      _stream(stream, dev))
+        else:
+            call = axis_attn_decode_hnd if hnd else axis_attn_decode
+            rc = call(*ptrs, B, Hq, Hkv, D, page_size, max_pages, num_pages, scale, wp, wb, _stream(stream, dev))
     if rc:
         raise AxisAttnError(rc, call.__name__)
     return o, l

@@ -44,13 +44,15 @@
 namespace axis_attn {
 
 struct DecArgs {
-  const __nv_bfloat16* q;  // [B, Hq, D]
+  const __nv_bfloat16* q;  // [B, q_len, Hq, D]
   const int* block_table;  // [B, max_pages]
   const int* seq_lens;     // [B]
-  __nv_bfloat16* o;        // [B, Hq, D]
-  float* lse;              // [B, Hq]
-  float* part;             // [B * Hq][n_splits][D + 2]: m, l, O (n_splits > 1)
+  __nv_bfloat16* o;        // [B, q_len, Hq, D]
+  float* lse;              // [B, Hq, q_len]
+  float* part;             // [B * q_len * Hq][n_splits][D + 2]: m, l, O (n_splits > 1)
   int B, Hq, Hkv, G, page_size, max_pages, num_pages;
+  int q_len;               // new tokens per sequence: the last q_len positions
+  int n_rt;                // row tiles per (b, kv head): ceil(G * q_len / 8) of 8 (token, head) rows
   int hnd;                 // cache layout: 0 [pages, page_size, Hkv, D]; 1 [pages, Hkv, page_size, D]
   int keys_per_split;      // a multiple of 32
   int n_splits;
@@ -107,6 +109,11 @@ struct DecCfg {
   // phase k - 2): the previous piece in a stage must be the same warp's,
   // which holds when the ring depth is a multiple of the warp count.
   static_assert(NST % CW == 0, "ring depth must be a multiple of the compute warps");
+  // Resident CTAs per SM the registers must allow (0: no bound).  The wide
+  // D = 64 configuration (160 threads) fits 4 per SM only at <= 102 registers
+  // a thread; left alone ptxas takes 125 and 3 fit (page size 16: 58.6 us
+  // against 52.8 us with the bound, at a few dozen bytes of spills).
+  static constexpr int MIN_CTAS = (HD == 64 && !DEEP) ? 4 : 0;
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = NST * PIECE;
   static constexpr uint32_t OFF_C = 2 * NST * PIECE;              // fp32 [CW][8][HD + 2]
@@ -119,22 +126,30 @@ struct DecCfg {
 
 enum DecSite { D_EMPTY = 41, D_FULL };
 
-// One work item: (b, kv head, split of the sequence), its key range and pieces.
+// One work item: (b, kv head, split of the sequence, row tile), its key
+// range and pieces.  The row tiles of a (b, kv head, split) are adjacent in
+// the item order, so the CTAs that read the same pieces run at the same time
+// (the second reader finds them in L2).  len: the sequence's length (its
+// q_len new tokens included).
 struct DecItem {
-  int b, kv, split, k0, k1, n_pieces;
+  int b, kv, split, rt, k0, k1, n_pieces, len;
 };
-__device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report) {
+// q_len, n_rt: the launch's (compile-time 1, 1 in the one-token instantiation)
+__device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report, int q_len, int n_rt) {
   DecItem it;
+  it.rt = w % n_rt;
+  w /= n_rt;
   it.split = w % a.n_splits;
   const int bkv = w / a.n_splits;
   it.b = bkv / a.Hkv;
   it.kv = bkv % a.Hkv;
   int len = a.seq_lens[it.b];
   const int cap = a.max_pages * a.page_size;
-  if (len < 1 || len > cap) {  // clamped; reported once (by the producer)
+  if (len < q_len || len > cap) {  // clamped (cap >= q_len); reported once (by the producer)
     if (report) atomicOr(&g_status, 2u);
-    len = len < 1 ? 1 : cap;
+    len = len < q_len ? q_len : cap;
   }
+  it.len = len;
   it.k0 = it.split * a.keys_per_split;
   it.k1 = min(len, it.k0 + a.keys_per_split);
   it.n_pieces = it.k1 > it.k0 ? (it.k1 - it.k0 + 31) / 32 : 0;
@@ -145,8 +160,8 @@ __device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report
 // ...; the ring positions count pieces over all of its items, so the producer
 // streams the next item's pieces while the compute warps finish this one.
 // Compute warp (g mod CW) takes the CTA's g-th piece.
-template <int HD, bool DEEP>
-__global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
+template <int HD, bool DEEP, bool MULTI>
+__global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS, DecCfg<HD, DEEP>::MIN_CTAS)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const DecArgs a) {
   using C = DecCfg<HD, DEEP>;
@@ -164,7 +179,10 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
   volatile WaitCtl* ctl = reinterpret_cast<volatile WaitCtl*>(gbase + C::OFF_BAR + 16 * NST + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_items = a.B * a.Hkv * a.n_splits;
+  // several new tokens per sequence, or one (MULTI = false: q_len = 1 and one
+  // row tile at compile time, the code of the one-token step)
+  const int q_len = MULTI ? a.q_len : 1, n_rt = MULTI ? a.n_rt : 1;
+  const int n_items = a.B * a.Hkv * a.n_splits * n_rt;
   const int G = a.G;
 
   if (threadIdx.x == 0) {
@@ -198,7 +216,7 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
     int g = 0;  // pieces issued (over all items); the same in every lane
     bool ok = true;
     for (int w = (int)blockIdx.x; ok && w < n_items; w += (int)gridDim.x) {
-      const DecItem I = dec_item(a, w, lane == 0);
+      const DecItem I = dec_item(a, w, lane == 0, q_len, n_rt);
       const int* row_tbl = a.block_table + (size_t)I.b * a.max_pages;
       for (int t0 = 0; ok && t0 < I.n_pieces; t0 += 32) {
         const int kt = I.k0 + 32 * (t0 + lane);  // this lane's piece
@@ -256,9 +274,11 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
   } else {
     // ============================================================ compute warps
     // Per 32-key piece: S (16 x 32) = Q K^T and O (16 x D) += P V on the
-    // warp-level MMA, the G <= 8 query heads as rows 0..G-1 of a 16-row tile
-    // (rows G..15 zero).  Lane l holds, in the accumulator layout, row
-    // g0 = l / 4 and the columns 2 (l % 4) + {0, 1} of every 8-column tile.
+    // warp-level MMA, the item's 8 (token, head) rows as rows 0..7 of a
+    // 16-row tile (rows 8..15 zero): row r = 8 rt + g0 of the unit is new
+    // token r / G and head r % G (rows past G q_len unused).  Lane l holds, in
+    // the accumulator layout, row g0 = l / 4 and the columns 2 (l % 4) + {0, 1}
+    // of every 8-column tile.
     const int cw = warp - 1;
     const float c = a.scale_log2;
     constexpr int KS = HD / 16;  // k-steps of the score product (features)
@@ -271,15 +291,22 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
     // (its later waits then return at once: the CTA's abort flag is set), so
     // that all of them reach each of the named barriers below.
     for (int w = (int)blockIdx.x; w < n_items; w += (int)gridDim.x) {
-      const DecItem I = dec_item(a, w, false);
+      const DecItem I = dec_item(a, w, false, q_len, n_rt);
+      const int row = 8 * I.rt + g0;
+      const bool row_ok = row < G * q_len;
+      const int tok = row / G, gh = row % G;  // new token, head in the group
+      // this row's keys end after its own position len - q_len + tok (the
+      // later new tokens are masked): keys of piece t below row_end - 32 t - k0
+      const int row_end = I.len - q_len + tok + 1;
       // Q as A fragments: (row g0, columns 16 ks + q2 + {0,1}) and (+8); the
       // fragments of rows 8..15 are zero
       uint32_t qa[KS][2];
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         qa[ks][0] = qa[ks][1] = 0u;
-        if (g0 < G) {
-          const __nv_bfloat16* qrow = a.q + ((size_t)I.b * a.Hq + I.kv * G + g0) * HD + 16 * ks + q2;
+        if (row_ok) {
+          const __nv_bfloat16* qrow =
+              a.q + (((size_t)I.b * q_len + tok) * a.Hq + I.kv * G + gh) * HD + 16 * ks + q2;
           qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow);
           qa[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 8);
         }
@@ -321,13 +348,15 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
               mma_16816(sc[nt], qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u, bk[2], bk[3]);
             }
           }
-          // ---- online softmax of row g0 (the 4 lanes of a quad hold its 32 keys)
+          // ---- online softmax of row g0 (the 4 lanes of a quad hold its 32 keys);
+          // the row sees this piece's keys below lim (its own position included)
+          const int lim = min(n_valid, row_end - (I.k0 + 32 * t));
           float mx = -INFINITY;
 #pragma unroll
           for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              if (8 * nt + q2 + e >= n_valid) sc[nt][e] = -INFINITY;
+              if (8 * nt + q2 + e >= lim) sc[nt][e] = -INFINITY;
               mx = fmaxf(mx, sc[nt][e]);
             }
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -344,12 +373,16 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
             }
           }
           // p = 2^(s c - m); bf16 P as the A fragments of P V: k-step k2 takes the
-          // key tiles 2 k2 (columns 0..7) and 2 k2 + 1 (columns 8..15)
+          // key tiles 2 k2 (columns 0..7) and 2 k2 + 1 (columns 8..15).  A row
+          // that has seen no key of its own yet (m = -inf: this piece and the
+          // warp's earlier ones all lie past its position) gets p = 0, not
+          // 2^(-inf + inf).
+          const float nm = m_run == -INFINITY ? 0.f : -m_run;
           uint32_t pa[4];
 #pragma unroll
           for (int nt = 0; nt < 4; ++nt) {
-            const float p0 = ex2_approx(fmaf(sc[nt][0], c, -m_run));
-            const float p1 = ex2_approx(fmaf(sc[nt][1], c, -m_run));
+            const float p0 = ex2_approx(fmaf(sc[nt][0], c, nm));
+            const float p1 = ex2_approx(fmaf(sc[nt][1], c, nm));
             l_part += p0 + p1;
             pa[nt] = pack_bf16x2(p0, p1);
           }
@@ -370,11 +403,11 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
         if (lane == 0) mbar_arrive(bar_empty(s));
       }
       gbase_item += I.n_pieces;
-      // ---- this warp's (m, l, O) of each head, then the merge of the CW warps
+      // ---- this warp's (m, l, O) of each row, then the merge of the CW warps
       float l = l_part;
       l += __shfl_xor_sync(0xffffffffu, l, 1);
       l += __shfl_xor_sync(0xffffffffu, l, 2);
-      if (g0 < G) {
+      if (row_ok) {
         float* cs = c_s + (cw * 8 + g0) * (HD + 2);
 #pragma unroll
         for (int nd = 0; nd < ND; ++nd) {
@@ -387,7 +420,7 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
         }
       }
       named_bar_sync(1, 32 * CW);
-      for (int g = cw; g < G; g += CW) {
+      for (int g = cw; g < 8 && 8 * I.rt + g < G * q_len; g += CW) {
         float mm = -INFINITY;
 #pragma unroll
         for (int x = 0; x < CW; ++x) mm = fmaxf(mm, c_s[(x * 8 + g) * (HD + 2)]);
@@ -402,14 +435,17 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
 #pragma unroll
           for (int f = 0; f < FPL; ++f) ov[f] += cs[2 + lane * FPL + f] * e;
         }
-        const int bh = I.b * a.Hq + I.kv * G + g;
+        // output row (b, new token, head) of o [B, q_len, Hq, D]; lse is [B, Hq, q_len]
+        const int r = 8 * I.rt + g, h = I.kv * G + r % G, tk = r / G;
+        const size_t orow = ((size_t)I.b * q_len + tk) * a.Hq + h;
         if (a.n_splits == 1) {
           const float inv = lt > 0.f ? 1.f / lt : 0.f;
 #pragma unroll
-          for (int f = 0; f < FPL; ++f) a.o[(size_t)bh * HD + lane * FPL + f] = __float2bfloat16_rn(ov[f] * inv);
-          if (lane == 0) a.lse[bh] = (mm + __log2f(lt)) * 0.69314718055994531f;
+          for (int f = 0; f < FPL; ++f) a.o[orow * HD + lane * FPL + f] = __float2bfloat16_rn(ov[f] * inv);
+          if (lane == 0)
+            a.lse[((size_t)I.b * a.Hq + h) * q_len + tk] = (mm + __log2f(lt)) * 0.69314718055994531f;
         } else {
-          float* dst = a.part + ((size_t)bh * a.n_splits + I.split) * (HD + 2);
+          float* dst = a.part + (orow * a.n_splits + I.split) * (HD + 2);
 #pragma unroll
           for (int f = 0; f < FPL; ++f) dst[2 + lane * FPL + f] = ov[f];
           if (lane == 0) {
@@ -424,7 +460,7 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS)
   }
 }
 
-// Merge the splits of every (b, h): one 256-thread CTA per row.  The maximum
+// Merge the splits of every (b, new token, h): one 256-thread CTA per row.  The maximum
 // over the splits comes from all threads at once (one split each); then warp w
 // takes splits w, w + 8, ... (lanes over features, DEC_COMBINE_U splits'
 // loads in flight at a time) and the 8 warps' sums meet in shared memory.
@@ -434,7 +470,8 @@ constexpr int DEC_COMBINE_U = 4;
 template <int HD>
 __global__ void __launch_bounds__(256) attn_decode_combine_kernel(const float* __restrict__ part,
                                                                   __nv_bfloat16* __restrict__ o,
-                                                                  float* __restrict__ lse, int rows, int n_splits) {
+                                                                  float* __restrict__ lse, int rows, int n_splits,
+                                                                  int Hq, int q_len) {
   constexpr int FPL = HD / 32, NW = 8;
   __shared__ float s_red[NW];
   __shared__ float s_o[NW][HD];
@@ -499,7 +536,10 @@ __global__ void __launch_bounds__(256) attn_decode_combine_kernel(const float* _
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
 #pragma unroll
       for (int f = 0; f < FPL; ++f) o[(size_t)bh * HD + lane * FPL + f] = __float2bfloat16_rn(ot[f] * inv);
-      if (lane == 0) lse[bh] = (mm + __log2f(lt)) * 0.69314718055994531f;
+      // row bh = (b q_len + token) Hq + h of o; lse is [B, Hq, q_len]
+      if (lane == 0)
+        lse[((size_t)(bh / (q_len * Hq)) * Hq + bh % Hq) * q_len + (bh / Hq) % q_len] =
+            (mm + __log2f(lt)) * 0.69314718055994531f;
     }
     __syncthreads();  // warp 0 has read s_red and s_o before the next row writes them
   }

@@ -597,13 +597,17 @@ namespace {
 
 bool pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
 
-int check_decode_shape(int B, int Hq, int Hkv, int D, int page_size, int max_pages, int num_pages, float scale) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_pages < 1 || num_pages < 1) return AXIS_ATTN_ERR_SHAPE;
+// q_len: new tokens per sequence (1 .. 64; a sequence must have room for them).
+int check_decode_shape(int B, int Hq, int Hkv, int D, int page_size, int max_pages, int num_pages, float scale,
+                       int q_len = 1) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || max_pages < 1 || num_pages < 1 || q_len < 1)
+    return AXIS_ATTN_ERR_SHAPE;
   if (!(std::isfinite(scale) && scale > 0.f)) return AXIS_ATTN_ERR_SHAPE;
   if (D != 64 && D != 128) return AXIS_ATTN_ERR_UNSUPPORTED;
-  if (Hq / Hkv > 8 || !pow2_in(page_size, 8, 256)) return AXIS_ATTN_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 8 || !pow2_in(page_size, 8, 256) || q_len > 64) return AXIS_ATTN_ERR_UNSUPPORTED;
   if ((long long)max_pages * page_size >= (1LL << 30) || (long long)num_pages * page_size >= (1LL << 31) ||
-      (long long)B * max_pages >= (1LL << 31))
+      (long long)B * max_pages >= (1LL << 31) || (long long)B * q_len * Hq * D >= (1LL << 31) ||
+      (long long)max_pages * page_size < q_len)
     return AXIS_ATTN_ERR_SHAPE;
   return AXIS_ATTN_OK;
 }
@@ -620,9 +624,11 @@ struct DecSplit {
 #ifndef AXIS_ATTN_DEC_SPLIT_ITEMS
 #define AXIS_ATTN_DEC_SPLIT_ITEMS 296
 #endif
-DecSplit decode_split(int B, int Hkv, int page_size, int max_pages) {
+// (b, kv head) units, each n_rt row tiles of 8 (new token, head) rows
+int decode_row_tiles(int Hq, int Hkv, int q_len) { return (Hq / Hkv * q_len + 7) / 8; }
+DecSplit decode_split(int B, int Hkv, int page_size, int max_pages, int n_rt = 1) {
   const long long keys = (long long)max_pages * page_size;
-  const long long units = (long long)B * Hkv;
+  const long long units = (long long)B * Hkv * n_rt;
   long long n = (AXIS_ATTN_DEC_SPLIT_ITEMS + units - 1) / units;
   const long long n_max = (keys + 255) / 256;
   if (n > n_max) n = n_max;
@@ -632,8 +638,9 @@ DecSplit decode_split(int B, int Hkv, int page_size, int max_pages) {
   return {(int)n, (int)kps};
 }
 
-size_t decode_ws_bytes(int B, int Hq, int D, const DecSplit& sp) {
-  return sp.n_splits > 1 ? (size_t)B * Hq * sp.n_splits * (D + 2) * 4 : 0;
+// partial (m, l, O) of every (b, new token, head) row and split
+size_t decode_ws_bytes(int B, int Hq, int D, const DecSplit& sp, int q_len = 1) {
+  return sp.n_splits > 1 ? (size_t)B * q_len * Hq * sp.n_splits * (D + 2) * 4 : 0;
 }
 
 // 3-D map over a paged cache [num_pages * page_size rows][Hkv][D] (bf16):
@@ -667,11 +674,11 @@ bool make_cache_map_hnd(CUtensorMap* map, const void* ptr, int num_pages, int pa
 }
 
 // Persistent decode: as many CTAs as fit on the SMs at once (or one per item).
-template <int HD, bool DEEP>
+template <int HD, bool DEEP, bool MULTI>
 int launch_decode_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev,
                       long long items) {
   using C = DecCfg<HD, DEEP>;
-  auto kern = attn_decode_kernel<HD, DEEP>;
+  auto kern = attn_decode_kernel<HD, DEEP, MULTI>;
   static bool done[64];
   static int per_sm[64];
   if (int rc = set_smem(kern, C::SMEM, dev, done)) return rc;
@@ -701,10 +708,13 @@ constexpr int dec_per_sm() {
 // wide 0.39-0.51; 512 items, wide 0.80 against deep 0.59.
 template <int HD>
 int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev) {
-  const long long items = (long long)a.B * a.Hkv * a.n_splits;
+  const long long items = (long long)a.B * a.Hkv * a.n_splits * a.n_rt;
   const bool deep = items <= (long long)dec_per_sm<HD, true>() * sm_count(dev);
-  return deep ? launch_decode_cfg<HD, true>(mk, mv, a, st, dev, items)
-              : launch_decode_cfg<HD, false>(mk, mv, a, st, dev, items);
+  if (a.q_len > 1)
+    return deep ? launch_decode_cfg<HD, true, true>(mk, mv, a, st, dev, items)
+                : launch_decode_cfg<HD, false, true>(mk, mv, a, st, dev, items);
+  return deep ? launch_decode_cfg<HD, true, false>(mk, mv, a, st, dev, items)
+              : launch_decode_cfg<HD, false, false>(mk, mv, a, st, dev, items);
 }
 
 }  // namespace
@@ -715,18 +725,26 @@ extern "C" size_t axis_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D
   return decode_ws_bytes(B, Hq, D, decode_split(B, Hkv, page_size, max_pages));
 }
 
+extern "C" size_t axis_attn_decode_q_workspace_bytes(int B, int q_len, int Hq, int Hkv, int D, int page_size,
+                                                     int max_pages) {
+  if (check_decode_shape(B, Hq, Hkv, D, page_size, max_pages, 1, 1.f, q_len) != AXIS_ATTN_OK) return 0;
+  const int n_rt = decode_row_tiles(Hq, Hkv, q_len);
+  return decode_ws_bytes(B, Hq, D, decode_split(B, Hkv, page_size, max_pages, n_rt), q_len);
+}
+
 namespace axis_attn {
 namespace {
 int run_decode(const void* q, const void* k_cache, const void* v_cache, const int* block_table, const int* seq_lens,
                void* o, float* lse, int B, int Hq, int Hkv, int D, int page_size, int max_pages, int num_pages,
-               float scale, void* workspace, size_t workspace_bytes, void* stream, bool hnd) {
+               float scale, void* workspace, size_t workspace_bytes, void* stream, bool hnd, int q_len) {
   if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !o || !lse) return AXIS_ATTN_ERR_NULL;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse) ||
       (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
     return AXIS_ATTN_ERR_ALIGN;
-  if (int rc = check_decode_shape(B, Hq, Hkv, D, page_size, max_pages, num_pages, scale)) return rc;
-  const DecSplit sp = decode_split(B, Hkv, page_size, max_pages);
-  const size_t need = decode_ws_bytes(B, Hq, D, sp);
+  if (int rc = check_decode_shape(B, Hq, Hkv, D, page_size, max_pages, num_pages, scale, q_len)) return rc;
+  const int n_rt = decode_row_tiles(Hq, Hkv, q_len);
+  const DecSplit sp = decode_split(B, Hkv, page_size, max_pages, n_rt);
+  const size_t need = decode_ws_bytes(B, Hq, D, sp, q_len);
   if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need))
     return AXIS_ATTN_ERR_WORKSPACE;
   int dev = 0;
@@ -754,18 +772,20 @@ int run_decode(const void* q, const void* k_cache, const void* v_cache, const in
   a.max_pages = max_pages;
   a.num_pages = num_pages;
   a.hnd = hnd ? 1 : 0;
+  a.q_len = q_len;
+  a.n_rt = n_rt;
   a.keys_per_split = sp.keys_per_split;
   a.n_splits = sp.n_splits;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int rc = D == 64 ? launch_decode<64>(mk, mv, a, st, dev) : launch_decode<128>(mk, mv, a, st, dev);
   if (rc || sp.n_splits == 1) return rc;
-  const int rows = B * Hq;
-  const unsigned grid = (unsigned)(rows < 148 * 8 ? rows : 148 * 8);  // one CTA per (b, h) row
+  const int rows = B * q_len * Hq;
+  const unsigned grid = (unsigned)(rows < 148 * 8 ? rows : 148 * 8);  // one CTA per (b, new token, h) row
   if (D == 64)
-    attn_decode_combine_kernel<64><<<grid, 256, 0, st>>>(a.part, a.o, lse, rows, sp.n_splits);
+    attn_decode_combine_kernel<64><<<grid, 256, 0, st>>>(a.part, a.o, lse, rows, sp.n_splits, Hq, q_len);
   else
-    attn_decode_combine_kernel<128><<<grid, 256, 0, st>>>(a.part, a.o, lse, rows, sp.n_splits);
+    attn_decode_combine_kernel<128><<<grid, 256, 0, st>>>(a.part, a.o, lse, rows, sp.n_splits, Hq, q_len);
   return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 }  // namespace
@@ -776,7 +796,7 @@ extern "C" int axis_attn_decode(const void* q, const void* k_cache, const void* 
                                 int page_size, int max_pages, int num_pages, float scale, void* workspace,
                                 size_t workspace_bytes, void* stream) {
   return axis_attn::run_decode(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
-                               max_pages, num_pages, scale, workspace, workspace_bytes, stream, false);
+                               max_pages, num_pages, scale, workspace, workspace_bytes, stream, false, 1);
 }
 
 extern "C" int axis_attn_decode_hnd(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
@@ -784,7 +804,16 @@ extern "C" int axis_attn_decode_hnd(const void* q, const void* k_cache, const vo
                                     int page_size, int max_pages, int num_pages, float scale, void* workspace,
                                     size_t workspace_bytes, void* stream) {
   return axis_attn::run_decode(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
-                               max_pages, num_pages, scale, workspace, workspace_bytes, stream, true);
+                               max_pages, num_pages, scale, workspace, workspace_bytes, stream, true, 1);
+}
+
+extern "C" int axis_attn_decode_q(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                                  const int* seq_lens, void* o, float* lse, int B, int q_len, int Hq, int Hkv, int D,
+                                  int page_size, int max_pages, int num_pages, float scale, int head_major,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  return axis_attn::run_decode(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, D, page_size,
+                               max_pages, num_pages, scale, workspace, workspace_bytes, stream, head_major != 0,
+                               q_len);
 }
 
 static unsigned int g_last_status_word;

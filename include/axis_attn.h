@@ -297,6 +297,40 @@ int axis_attn_decode_hnd(const void* q, const void* k_cache, const void* v_cache
                          size_t workspace_bytes, void* stream);
 
 /*
+ * Decode step with q_len new tokens per sequence at once: the engine above
+ * advancing several positions in one step (a chunk of a prompt appended to
+ * the cache, or several proposed tokens checked together).  The new tokens are
+ * the last q_len positions of their sequence, already in the cache: new token
+ * t of sequence b sits at position p = seq_lens[b] - q_len + t and, under the
+ * causal mask, attends to the cached keys j <= p (the earlier new tokens and
+ * itself, not the later ones).  For query head h (kv head h / (Hq / Hkv)):
+ *   o[b,t,h,:] = sum_{j<=p} P_j V_j,  P = softmax_j(scale * <q[b,t,h,:], K_j>)
+ *   lse[b,h,t] = ln sum_{j<=p} exp(scale * <q[b,t,h,:], K_j>)
+ *
+ *  - q, o: [B, q_len, Hq, D] bf16; lse: [B, Hq, q_len] fp32.  q_len = 1 is
+ *    axis_attn_decode (head_major = 0) / axis_attn_decode_hnd (head_major = 1).
+ *  - k_cache, v_cache: [num_pages, page_size, Hkv, D] (head_major = 0) or
+ *    [num_pages, Hkv, page_size, D] (head_major = 1) bf16, read through
+ *    block_table as for axis_attn_decode.
+ *  - seq_lens[b]: cached tokens of sequence b, the q_len new ones included; a
+ *    length outside [q_len, max_pages*page_size] is clamped and reported as
+ *    AXIS_ATTN_ERR_INDEX (as are out-of-range page indices).
+ *  - Requirements: those of axis_attn_decode, and 1 <= q_len <= 64,
+ *    q_len <= max_pages * page_size, B * q_len * Hq * D < 2^31.  The kernel
+ *    takes the G * q_len (token, head) rows of a kv head in tiles of 8, each
+ *    tile streaming the kv head's keys (the tiles of a head run side by side,
+ *    so the second and later reads come from L2).
+ *  - workspace: axis_attn_decode_q_workspace_bytes() bytes (0 is possible),
+ *    256-byte aligned, caller-owned; calls that overlap must not share it.
+ */
+size_t axis_attn_decode_q_workspace_bytes(int B, int q_len, int Hq, int Hkv, int D, int page_size,
+                                          int max_pages);
+int axis_attn_decode_q(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                       const int* seq_lens, void* o, float* lse, int B, int q_len, int Hq, int Hkv, int D,
+                       int page_size, int max_pages, int num_pages, float scale, int head_major,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then returns AXIS_ATTN_ERR_TIMEOUT if any kernel of
  * this library on the current device has reported a timed-out device wait since
  * the last call, else AXIS_ATTN_ERR_INDEX if a decode step met an out-of-range

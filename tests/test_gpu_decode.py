@@ -149,3 +149,85 @@ def test_decode_bad_indices_are_reported_not_used(oracle_mod, layout):
     aa.check_status()
     ro, rl = oracle_mod.attn_decode(q, k, v, lens, D ** -0.5)
     assert float((o.cpu().double() - torch.from_numpy(ro)).abs().max()) <= TOL_O
+
+
+# ---- several new tokens per sequence (axis_attn_decode_q)
+
+def run_case_q(oracle_mod, B, q_len, Hq, Hkv, D, Smax, page_size, lens, seed, layout="NHD"):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((B, q_len, Hq, D), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
+    lens = np.asarray(lens, np.int32)
+    sc = 1.0 / math.sqrt(D)
+    kc, vc, table, num_pages = paged(k, v, lens, page_size, seed)
+    kc, vc = as_layout(kc, vc, layout)
+    dev = torch.device("cuda:0")
+    o, lse = aa.attention_decode(q.to(dev), kc.to(dev), vc.to(dev), table.to(dev),
+                                 torch.from_numpy(lens).to(dev), scale=sc, layout=layout)
+    aa.check_status()
+    assert o.shape == (B, q_len, Hq, D) and lse.shape == (B, Hq, q_len)
+    ro, rl = oracle_mod.attn_decode_q(q, k, v, lens, sc)
+    eo = float((o.cpu().double() - torch.from_numpy(ro)).abs().max())
+    el = float((lse.cpu().double() - torch.from_numpy(rl)).abs().max())
+    return eo, el
+
+
+CASES_Q = [
+    # B, q_len, Hq, Hkv, D, Smax, page_size, lens
+    (2, 2, 8, 8, 64, 100, 16, [2, 100]),               # G = 1: 2 rows per tile
+    (3, 4, 12, 4, 64, 300, 16, [4, 33, 300]),          # G = 3: 12 rows -> 2 tiles; len = q_len
+    (2, 3, 32, 4, 128, 700, 64, [700, 35]),            # G = 8: 24 rows -> 3 tiles
+    (1, 16, 2, 2, 64, 8192, 32, [8190]),               # one long sequence: split-K, 16 new tokens
+    (1, 5, 24, 8, 64, 5000, 8, [4999]),                # G = 3, q_len 5: tiles ragged; split-K
+    (48, 2, 16, 8, 128, 600, 16, [600, 2, 37, 599] * 12),  # many sequences, no split
+    (40, 8, 8, 8, 64, 2100, 8, [2100, 8, 1024, 1025, 2047, 2048, 2049, 33] * 5),
+    # a split boundary (8192) among the new tokens: the first 8 of them see no
+    # key of the last split, whose partial result must weigh nothing
+    (1, 16, 2, 2, 64, 8320, 32, [8200]),
+]
+
+
+@pytest.mark.parametrize("layout", ["NHD", "HND"])
+@pytest.mark.parametrize("B,q_len,Hq,Hkv,D,Smax,ps,lens", CASES_Q)
+def test_decode_q_matches_oracle(oracle_mod, B, q_len, Hq, Hkv, D, Smax, ps, lens, layout):
+    eo, el = run_case_q(oracle_mod, B, q_len, Hq, Hkv, D, Smax, ps, lens,
+                        seed=7000 + B + q_len + Hq + D + Smax + ps, layout=layout)
+    print(f"{layout} B{B} q{q_len} Hq{Hq} Hkv{Hkv} D{D} S{Smax} ps{ps}: O {eo:.2e} LSE {el:.2e}")
+    assert eo <= TOL_O and el <= TOL_LSE
+
+
+def test_decode_q_one_token_is_the_decode_step():
+    B, Hq, Hkv, D, Smax, ps = 4, 8, 2, 64, 300, 16
+    g = torch.Generator().manual_seed(71)
+    q = torch.randn((B, Hq, D), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
+    lens = np.array([300, 1, 17, 256], np.int32)
+    kc, vc, table, _ = paged(k, v, lens, ps, 71)
+    dev = torch.device("cuda:0")
+    args = [t.to(dev) for t in (kc, vc, table)] + [torch.from_numpy(lens).to(dev)]
+    o1, l1 = aa.attention_decode(q.to(dev), *args, scale=0.125)
+    oq, lq = aa.attention_decode(q.to(dev)[:, None], *args, scale=0.125)
+    aa.check_status()
+    assert torch.equal(o1, oq[:, 0]) and torch.equal(l1, lq[:, :, 0])
+
+
+def test_decode_q_short_length_is_reported(oracle_mod):
+    B, q_len, Hq, Hkv, D, Smax, ps = 2, 4, 4, 2, 64, 64, 16
+    g = torch.Generator().manual_seed(72)
+    q = torch.randn((B, q_len, Hq, D), generator=g).to(torch.bfloat16)
+    k = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Smax, Hkv, D), generator=g).to(torch.bfloat16)
+    lens = np.array([64, 40], np.int32)
+    kc, vc, table, _ = paged(k, v, lens, ps, 72)
+    dev = torch.device("cuda:0")
+    args = [t.to(dev) for t in (q, kc, vc, table)]
+    aa.attention_decode(*args, torch.tensor([64, 3], dtype=torch.int32, device=dev), scale=0.125)
+    assert aa.axis_attn_get_status(aa.binding._stream(None)) == 8  # a sequence shorter than its new tokens
+    # the same call with good lengths is exact afterwards
+    o, lse = aa.attention_decode(*args, torch.from_numpy(lens).to(dev), scale=0.125)
+    aa.check_status()
+    ro, rl = oracle_mod.attn_decode_q(q, k, v, lens, 0.125)
+    assert float((o.cpu().double() - torch.from_numpy(ro)).abs().max()) <= TOL_O
+    assert float((lse.cpu().double() - torch.from_numpy(rl)).abs().max()) <= TOL_LSE
