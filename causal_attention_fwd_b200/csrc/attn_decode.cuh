@@ -33,6 +33,11 @@
 //     memory; a split writes its unnormalised (m, l, O) to the workspace,
 //     which a second kernel merges (split-K over long sequences keeps every
 //     SM busy at small batch); with one split the CTA writes O and LSE itself.
+// Several new tokens per sequence (q_len > 1: a prompt chunk appended to the
+// cache, or proposed tokens checked together) are the last q_len positions;
+// a work item then takes a tile of 8 or 16 (token, head) rows of a kv head,
+// every row masked at its own position, and the tiles of a kv head, adjacent
+// in the item order, stream the same pieces (the later reads hit L2).
 // Page indices and sequence lengths are device data: a page index outside
 // [0, num_pages) or a length outside [1, max_pages * page_size] is never used
 // for an access; it sets bit 1 of the device status word (reported by
@@ -94,8 +99,12 @@ struct DecArgs {
 #define AXIS_ATTN_DEC_DEEP_NST128 4
 #endif
 
-template <int HD, bool DEEP>
+// MODE: 0 one new token per sequence (q_len = 1 at compile time); 1 several,
+// at most 8 (token, head) rows per kv head (8-row tiles); 2 several, more rows
+// (16-row tiles: both halves of the MMA's 16 rows carry rows).
+template <int HD, bool DEEP, int MODE = 0>
 struct DecCfg {
+  static constexpr int RT = MODE == 2 ? 16 : 8;  // (token, head) rows per work item
   static constexpr int NSLAB = HD / 64;
   static constexpr uint32_t SLAB = 32 * 128;            // 32 rows x 128 bytes
   static constexpr uint32_t PIECE = NSLAB * SLAB;       // 32 keys x HD bf16
@@ -113,11 +122,11 @@ struct DecCfg {
   // D = 64 configuration (160 threads) fits 4 per SM only at <= 102 registers
   // a thread; left alone ptxas takes 125 and 3 fit (page size 16: 58.6 us
   // against 52.8 us with the bound, at a few dozen bytes of spills).
-  static constexpr int MIN_CTAS = (HD == 64 && !DEEP) ? 4 : 0;
+  static constexpr int MIN_CTAS = (HD == 64 && !DEEP && MODE != 2) ? 4 : 0;
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = NST * PIECE;
-  static constexpr uint32_t OFF_C = 2 * NST * PIECE;              // fp32 [CW][8][HD + 2]
-  static constexpr uint32_t OFF_FLAG = OFF_C + CW * 8 * (HD + 2) * 4;  // int [NST]: piece usable
+  static constexpr uint32_t OFF_C = 2 * NST * PIECE;              // fp32 [CW][RT][HD + 2]
+  static constexpr uint32_t OFF_FLAG = OFF_C + CW * RT * (HD + 2) * 4;  // int [NST]: piece usable
   static constexpr uint32_t OFF_TBL = OFF_FLAG + NST * 4;                  // int [32][4]: pages of 32 pieces
   static constexpr uint32_t OFF_BAR = (OFF_TBL + 32 * 4 * 4 + 7) & ~7u;
   static constexpr uint32_t SMEM = OFF_BAR + 8 * 2 * NST + 16 + 1024;
@@ -160,12 +169,13 @@ __device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report
 // ...; the ring positions count pieces over all of its items, so the producer
 // streams the next item's pieces while the compute warps finish this one.
 // Compute warp (g mod CW) takes the CTA's g-th piece.
-template <int HD, bool DEEP, bool MULTI>
-__global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS, DecCfg<HD, DEEP>::MIN_CTAS)
+template <int HD, bool DEEP, int MODE>
+__global__ void __launch_bounds__(DecCfg<HD, DEEP, MODE>::THREADS, DecCfg<HD, DEEP, MODE>::MIN_CTAS)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const DecArgs a) {
-  using C = DecCfg<HD, DEEP>;
+  using C = DecCfg<HD, DEEP, MODE>;
   constexpr int NST = C::NST, CW = C::CW;
+  constexpr bool MULTI = MODE > 0;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -179,8 +189,8 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS, DecCfg<HD, DEEP>::M
   volatile WaitCtl* ctl = reinterpret_cast<volatile WaitCtl*>(gbase + C::OFF_BAR + 16 * NST + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // several new tokens per sequence, or one (MULTI = false: q_len = 1 and one
-  // row tile at compile time, the code of the one-token step)
+  // several new tokens per sequence, or one (MODE 0: q_len = 1 and one row
+  // tile at compile time, the code of the one-token step)
   const int q_len = MULTI ? a.q_len : 1, n_rt = MULTI ? a.n_rt : 1;
   const int n_items = a.B * a.Hkv * a.n_splits * n_rt;
   const int G = a.G;
@@ -274,11 +284,14 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS, DecCfg<HD, DEEP>::M
   } else {
     // ============================================================ compute warps
     // Per 32-key piece: S (16 x 32) = Q K^T and O (16 x D) += P V on the
-    // warp-level MMA, the item's 8 (token, head) rows as rows 0..7 of a
-    // 16-row tile (rows 8..15 zero): row r = 8 rt + g0 of the unit is new
-    // token r / G and head r % G (rows past G q_len unused).  Lane l holds, in
-    // the accumulator layout, row g0 = l / 4 and the columns 2 (l % 4) + {0, 1}
-    // of every 8-column tile.
+    // warp-level MMA, the item's RT (token, head) rows as rows of a 16-row
+    // tile: row r = RT rt + i of the unit is new token r / G and head r % G
+    // (rows past G q_len unused).  RT = 8 (MODE 0, 1): rows 0..7 of the MMA
+    // tile, rows 8..15 zero; RT = 16 (MODE 2): all 16 rows.  Lane l
+    // holds, in the accumulator layout, rows g0 = l / 4 (half 0) and g0 + 8
+    // (half 1) and the columns 2 (l % 4) + {0, 1} of every 8-column tile.
+    constexpr int NR = MODE == 2 ? 2 : 1;  // row halves this lane works on
+    constexpr int RT = C::RT;          // rows per tile: 8 NR
     const int cw = warp - 1;
     const float c = a.scale_log2;
     constexpr int KS = HD / 16;  // k-steps of the score product (features)
@@ -292,29 +305,36 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS, DecCfg<HD, DEEP>::M
     // that all of them reach each of the named barriers below.
     for (int w = (int)blockIdx.x; w < n_items; w += (int)gridDim.x) {
       const DecItem I = dec_item(a, w, false, q_len, n_rt);
-      const int row = 8 * I.rt + g0;
-      const bool row_ok = row < G * q_len;
-      const int tok = row / G, gh = row % G;  // new token, head in the group
-      // this row's keys end after its own position len - q_len + tok (the
-      // later new tokens are masked): keys of piece t below row_end - 32 t - k0
-      const int row_end = I.len - q_len + tok + 1;
-      // Q as A fragments: (row g0, columns 16 ks + q2 + {0,1}) and (+8); the
-      // fragments of rows 8..15 are zero
-      uint32_t qa[KS][2];
+      bool row_ok[NR];
+      int row_end[NR];
+      // Q as A fragments: (row, columns 16 ks + q2 + {0,1}) and (+8) of each half
+      uint32_t qf[NR][KS][2];
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        qa[ks][0] = qa[ks][1] = 0u;
-        if (row_ok) {
-          const __nv_bfloat16* qrow =
-              a.q + (((size_t)I.b * q_len + tok) * a.Hq + I.kv * G + gh) * HD + 16 * ks + q2;
-          qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow);
-          qa[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 8);
+      for (int hb = 0; hb < NR; ++hb) {
+        const int row = RT * I.rt + g0 + 8 * hb;
+        row_ok[hb] = row < G * q_len;
+        const int tok = row / G, gh = row % G;  // new token, head in the group
+        // this row's keys end after its own position len - q_len + tok (the
+        // later new tokens are masked): keys of piece t below row_end - 32 t - k0
+        row_end[hb] = I.len - q_len + tok + 1;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          qf[hb][ks][0] = qf[hb][ks][1] = 0u;
+          if (row_ok[hb]) {
+            const __nv_bfloat16* qrow =
+                a.q + (((size_t)I.b * q_len + tok) * a.Hq + I.kv * G + gh) * HD + 16 * ks + q2;
+            qf[hb][ks][0] = *reinterpret_cast<const uint32_t*>(qrow);
+            qf[hb][ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 8);
+          }
         }
       }
       float o_acc[ND][4];
 #pragma unroll
       for (int nd = 0; nd < ND; ++nd) o_acc[nd][0] = o_acc[nd][1] = o_acc[nd][2] = o_acc[nd][3] = 0.f;
-      float m_run = -INFINITY, l_part = 0.f;  // row g0: running max (log2 units), this lane's share of the sum
+      // per half: running max (log2 units), this lane's share of the row sum
+      float m_run[NR], l_part[NR];
+#pragma unroll
+      for (int hb = 0; hb < NR; ++hb) m_run[hb] = -INFINITY, l_part[hb] = 0.f;
       // this warp's pieces of the item: the CTA's piece gbase_item + t goes to warp (gbase_item + t) % CW
       for (int t = (cw - gbase_item % CW + CW) % CW; ok && t < I.n_pieces; t += CW) {
         const int gp = gbase_item + t;
@@ -344,47 +364,52 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS, DecCfg<HD, DEEP>::M
               const int key = 8 * nt + (lane & 7), f0 = 32 * k2 + 8 * (lane >> 3);
               uint32_t bk[4];
               ldsm_x4(kb + (f0 >> 6) * C::SLAB + key * 128 + ((((f0 & 63) >> 3) ^ (key & 7)) << 4), bk);
-              mma_16816(sc[nt], qa[2 * k2][0], 0u, qa[2 * k2][1], 0u, bk[0], bk[1]);
-              mma_16816(sc[nt], qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u, bk[2], bk[3]);
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk)
+                mma_16816(sc[nt], qf[0][2 * k2 + kk][0], NR > 1 ? qf[NR - 1][2 * k2 + kk][0] : 0u,
+                          qf[0][2 * k2 + kk][1], NR > 1 ? qf[NR - 1][2 * k2 + kk][1] : 0u, bk[2 * kk],
+                          bk[2 * kk + 1]);
             }
           }
-          // ---- online softmax of row g0 (the 4 lanes of a quad hold its 32 keys);
-          // the row sees this piece's keys below lim (its own position included)
-          const int lim = min(n_valid, row_end - (I.k0 + 32 * t));
-          float mx = -INFINITY;
+          // ---- online softmax of each row (the 4 lanes of a quad hold its 32 keys);
+          // a row sees this piece's keys below lim (its own position included).
+          // p = 2^(s c - m), bf16 P as the A fragments of P V (k-step k2: key
+          // tiles 2 k2 and 2 k2 + 1).  A row that has seen no key of its own yet
+          // (m = -inf: this piece and the warp's earlier ones all lie past its
+          // position) gets p = 0, not 2^(-inf + inf).
+          uint32_t pf[NR][4];
 #pragma unroll
-          for (int nt = 0; nt < 4; ++nt)
+          for (int hb = 0; hb < NR; ++hb) {
+            const int lim = min(n_valid, row_end[hb] - (I.k0 + 32 * t));
+            float mx = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              if (8 * nt + q2 + e >= lim) sc[nt][e] = -INFINITY;
-              mx = fmaxf(mx, sc[nt][e]);
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                if (8 * nt + q2 + e >= lim) sc[nt][2 * hb + e] = -INFINITY;
+                mx = fmaxf(mx, sc[nt][2 * hb + e]);
+              }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run[hb], mx * c);
+            if (m_new > m_run[hb] + 8.0f) {  // the running max moves only by more than 8 (a factor 256)
+              const float alpha = ex2_approx(m_run[hb] - m_new);  // 0 on the first piece
+              m_run[hb] = m_new;
+              l_part[hb] *= alpha;
+#pragma unroll
+              for (int nd = 0; nd < ND; ++nd) {
+                o_acc[nd][2 * hb] *= alpha;
+                o_acc[nd][2 * hb + 1] *= alpha;
+              }
             }
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          const float m_new = fmaxf(m_run, mx * c);
-          if (m_new > m_run + 8.0f) {  // the running max moves only by more than 8 (a factor 256)
-            const float alpha = ex2_approx(m_run - m_new);  // 0 on the first piece
-            m_run = m_new;
-            l_part *= alpha;
+            const float nm = m_run[hb] == -INFINITY ? 0.f : -m_run[hb];
 #pragma unroll
-            for (int nd = 0; nd < ND; ++nd) {
-              o_acc[nd][0] *= alpha;
-              o_acc[nd][1] *= alpha;
+            for (int nt = 0; nt < 4; ++nt) {
+              const float p0 = ex2_approx(fmaf(sc[nt][2 * hb], c, nm));
+              const float p1 = ex2_approx(fmaf(sc[nt][2 * hb + 1], c, nm));
+              l_part[hb] += p0 + p1;
+              pf[hb][nt] = pack_bf16x2(p0, p1);
             }
-          }
-          // p = 2^(s c - m); bf16 P as the A fragments of P V: k-step k2 takes the
-          // key tiles 2 k2 (columns 0..7) and 2 k2 + 1 (columns 8..15).  A row
-          // that has seen no key of its own yet (m = -inf: this piece and the
-          // warp's earlier ones all lie past its position) gets p = 0, not
-          // 2^(-inf + inf).
-          const float nm = m_run == -INFINITY ? 0.f : -m_run;
-          uint32_t pa[4];
-#pragma unroll
-          for (int nt = 0; nt < 4; ++nt) {
-            const float p0 = ex2_approx(fmaf(sc[nt][0], c, nm));
-            const float p1 = ex2_approx(fmaf(sc[nt][1], c, nm));
-            l_part += p0 + p1;
-            pa[nt] = pack_bf16x2(p0, p1);
           }
           // ---- O += P V: B fragments of V (rows = keys) through the transposing load
 #pragma unroll
@@ -395,8 +420,10 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS, DecCfg<HD, DEEP>::M
               const int key = 16 * k2 + 8 * ((lane >> 3) & 1) + (lane & 7), f0 = 16 * n2 + 8 * (lane >> 4);
               uint32_t bv[4];
               ldsm_x4_t(vb + (f0 >> 6) * C::SLAB + key * 128 + ((((f0 & 63) >> 3) ^ (key & 7)) << 4), bv);
-              mma_16816(o_acc[2 * n2], pa[2 * k2], 0u, pa[2 * k2 + 1], 0u, bv[0], bv[1]);
-              mma_16816(o_acc[2 * n2 + 1], pa[2 * k2], 0u, pa[2 * k2 + 1], 0u, bv[2], bv[3]);
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk)
+                mma_16816(o_acc[2 * n2 + kk], pf[0][2 * k2], NR > 1 ? pf[NR - 1][2 * k2] : 0u, pf[0][2 * k2 + 1],
+                          NR > 1 ? pf[NR - 1][2 * k2 + 1] : 0u, bv[2 * kk], bv[2 * kk + 1]);
             }
         }
         __syncwarp();
@@ -404,39 +431,42 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP>::THREADS, DecCfg<HD, DEEP>::M
       }
       gbase_item += I.n_pieces;
       // ---- this warp's (m, l, O) of each row, then the merge of the CW warps
-      float l = l_part;
-      l += __shfl_xor_sync(0xffffffffu, l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      if (row_ok) {
-        float* cs = c_s + (cw * 8 + g0) * (HD + 2);
 #pragma unroll
-        for (int nd = 0; nd < ND; ++nd) {
-          cs[2 + 8 * nd + q2] = o_acc[nd][0];
-          cs[3 + 8 * nd + q2] = o_acc[nd][1];
-        }
-        if ((lane & 3) == 0) {
-          cs[0] = m_run;
-          cs[1] = l;
+      for (int hb = 0; hb < NR; ++hb) {
+        float l = l_part[hb];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        if (row_ok[hb]) {
+          float* cs = c_s + (cw * RT + g0 + 8 * hb) * (HD + 2);
+#pragma unroll
+          for (int nd = 0; nd < ND; ++nd) {
+            cs[2 + 8 * nd + q2] = o_acc[nd][2 * hb];
+            cs[3 + 8 * nd + q2] = o_acc[nd][2 * hb + 1];
+          }
+          if ((lane & 3) == 0) {
+            cs[0] = m_run[hb];
+            cs[1] = l;
+          }
         }
       }
       named_bar_sync(1, 32 * CW);
-      for (int g = cw; g < 8 && 8 * I.rt + g < G * q_len; g += CW) {
+      for (int g = cw; g < RT && RT * I.rt + g < G * q_len; g += CW) {
         float mm = -INFINITY;
 #pragma unroll
-        for (int x = 0; x < CW; ++x) mm = fmaxf(mm, c_s[(x * 8 + g) * (HD + 2)]);
+        for (int x = 0; x < CW; ++x) mm = fmaxf(mm, c_s[(x * RT + g) * (HD + 2)]);
         float lt = 0.f, ov[FPL];
 #pragma unroll
         for (int f = 0; f < FPL; ++f) ov[f] = 0.f;
 #pragma unroll
         for (int x = 0; x < CW; ++x) {
-          const float* cs = c_s + (x * 8 + g) * (HD + 2);
+          const float* cs = c_s + (x * RT + g) * (HD + 2);
           const float e = cs[1] > 0.f ? ex2_approx(cs[0] - mm) : 0.f;  // warps without keys weigh 0
           lt += cs[1] * e;
 #pragma unroll
           for (int f = 0; f < FPL; ++f) ov[f] += cs[2 + lane * FPL + f] * e;
         }
         // output row (b, new token, head) of o [B, q_len, Hq, D]; lse is [B, Hq, q_len]
-        const int r = 8 * I.rt + g, h = I.kv * G + r % G, tk = r / G;
+        const int r = RT * I.rt + g, h = I.kv * G + r % G, tk = r / G;
         const size_t orow = ((size_t)I.b * q_len + tk) * a.Hq + h;
         if (a.n_splits == 1) {
           const float inv = lt > 0.f ? 1.f / lt : 0.f;

@@ -624,8 +624,13 @@ struct DecSplit {
 #ifndef AXIS_ATTN_DEC_SPLIT_ITEMS
 #define AXIS_ATTN_DEC_SPLIT_ITEMS 296
 #endif
-// (b, kv head) units, each n_rt row tiles of 8 (new token, head) rows
-int decode_row_tiles(int Hq, int Hkv, int q_len) { return (Hq / Hkv * q_len + 7) / 8; }
+// The kernel's mode: 0 one new token; 1 several, at most 8 (token, head) rows
+// per kv head (one 8-row tile); 2 more rows (tiles of 16).  A (b, kv head)
+// unit is n_rt tiles.
+int decode_mode(int Hq, int Hkv, int q_len) { return q_len == 1 ? 0 : Hq / Hkv * q_len <= 8 ? 1 : 2; }
+int decode_row_tiles(int Hq, int Hkv, int q_len) {
+  return decode_mode(Hq, Hkv, q_len) == 2 ? (Hq / Hkv * q_len + 15) / 16 : 1;
+}
 DecSplit decode_split(int B, int Hkv, int page_size, int max_pages, int n_rt = 1) {
   const long long keys = (long long)max_pages * page_size;
   const long long units = (long long)B * Hkv * n_rt;
@@ -674,11 +679,11 @@ bool make_cache_map_hnd(CUtensorMap* map, const void* ptr, int num_pages, int pa
 }
 
 // Persistent decode: as many CTAs as fit on the SMs at once (or one per item).
-template <int HD, bool DEEP, bool MULTI>
+template <int HD, bool DEEP, int MODE>
 int launch_decode_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev,
                       long long items) {
-  using C = DecCfg<HD, DEEP>;
-  auto kern = attn_decode_kernel<HD, DEEP, MULTI>;
+  using C = DecCfg<HD, DEEP, MODE>;
+  auto kern = attn_decode_kernel<HD, DEEP, MODE>;
   static bool done[64];
   static int per_sm[64];
   if (int rc = set_smem(kern, C::SMEM, dev, done)) return rc;
@@ -695,9 +700,9 @@ int launch_decode_cfg(const CUtensorMap& mk, const CUtensorMap& mv, const DecArg
 
 // Resident CTAs per SM of a configuration, from its shared memory and threads
 // (228 KB per SM, 1 KB reserved per CTA; 2048 threads).
-template <int HD, bool DEEP>
+template <int HD, bool DEEP, int MODE>
 constexpr int dec_per_sm() {
-  using C = DecCfg<HD, DEEP>;
+  using C = DecCfg<HD, DEEP, MODE>;
   constexpr int by_smem = 233472 / (int)(C::SMEM + 1024), by_threads = 2048 / C::THREADS;
   return by_smem < by_threads ? by_smem : by_threads;
 }
@@ -709,12 +714,17 @@ constexpr int dec_per_sm() {
 template <int HD>
 int launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, const DecArgs& a, cudaStream_t st, int dev) {
   const long long items = (long long)a.B * a.Hkv * a.n_splits * a.n_rt;
-  const bool deep = items <= (long long)dec_per_sm<HD, true>() * sm_count(dev);
-  if (a.q_len > 1)
-    return deep ? launch_decode_cfg<HD, true, true>(mk, mv, a, st, dev, items)
-                : launch_decode_cfg<HD, false, true>(mk, mv, a, st, dev, items);
-  return deep ? launch_decode_cfg<HD, true, false>(mk, mv, a, st, dev, items)
-              : launch_decode_cfg<HD, false, false>(mk, mv, a, st, dev, items);
+  const int mode = decode_mode(a.Hq, a.Hkv, a.q_len);
+  const int deep_per_sm = mode == 2 ? dec_per_sm<HD, true, 2>() : dec_per_sm<HD, true, 0>();
+  const bool deep = items <= (long long)deep_per_sm * sm_count(dev);
+  if (mode == 2)
+    return deep ? launch_decode_cfg<HD, true, 2>(mk, mv, a, st, dev, items)
+                : launch_decode_cfg<HD, false, 2>(mk, mv, a, st, dev, items);
+  if (mode == 1)
+    return deep ? launch_decode_cfg<HD, true, 1>(mk, mv, a, st, dev, items)
+                : launch_decode_cfg<HD, false, 1>(mk, mv, a, st, dev, items);
+  return deep ? launch_decode_cfg<HD, true, 0>(mk, mv, a, st, dev, items)
+              : launch_decode_cfg<HD, false, 0>(mk, mv, a, st, dev, items);
 }
 
 }  // namespace

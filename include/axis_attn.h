@@ -317,9 +317,10 @@ int axis_attn_decode_hnd(const void* q, const void* k_cache, const void* v_cache
  *    AXIS_ATTN_ERR_INDEX (as are out-of-range page indices).
  *  - Requirements: those of axis_attn_decode, and 1 <= q_len <= 64,
  *    q_len <= max_pages * page_size, B * q_len * Hq * D < 2^31.  The kernel
- *    takes the G * q_len (token, head) rows of a kv head in tiles of 8, each
- *    tile streaming the kv head's keys (the tiles of a head run side by side,
- *    so the second and later reads come from L2).
+ *    takes the G * q_len (token, head) rows of a kv head in tiles of 8 (when
+ *    there are at most 8) or 16, each tile streaming the kv head's keys (the
+ *    tiles of a head run side by side, so the second and later reads come
+ *    from L2).
  *  - workspace: axis_attn_decode_q_workspace_bytes() bytes (0 is possible),
  *    256-byte aligned, caller-owned; calls that overlap must not share it.
  */

@@ -175,9 +175,9 @@ def run_case_q(oracle_mod, B, q_len, Hq, Hkv, D, Smax, page_size, lens, seed, la
 
 CASES_Q = [
     # B, q_len, Hq, Hkv, D, Smax, page_size, lens
-    (2, 2, 8, 8, 64, 100, 16, [2, 100]),               # G = 1: 2 rows per tile
-    (3, 4, 12, 4, 64, 300, 16, [4, 33, 300]),          # G = 3: 12 rows -> 2 tiles; len = q_len
-    (2, 3, 32, 4, 128, 700, 64, [700, 35]),            # G = 8: 24 rows -> 3 tiles
+    (2, 2, 8, 8, 64, 100, 16, [2, 100]),               # G = 1: 2 of a tile's 16 rows
+    (3, 4, 12, 4, 64, 300, 16, [4, 33, 300]),          # G = 3: 12 rows; len = q_len
+    (2, 3, 32, 4, 128, 700, 64, [700, 35]),            # G = 8: 24 rows -> 2 tiles, the second ragged
     (1, 16, 2, 2, 64, 8192, 32, [8190]),               # one long sequence: split-K, 16 new tokens
     (1, 5, 24, 8, 64, 5000, 8, [4999]),                # G = 3, q_len 5: tiles ragged; split-K
     (48, 2, 16, 8, 128, 600, 16, [600, 2, 37, 599] * 12),  # many sequences, no split
@@ -185,6 +185,7 @@ CASES_Q = [
     # a split boundary (8192) among the new tokens: the first 8 of them see no
     # key of the last split, whose partial result must weigh nothing
     (1, 16, 2, 2, 64, 8320, 32, [8200]),
+    (2, 8, 32, 4, 64, 500, 16, [500, 9]),              # G = 8: 64 rows -> 4 tiles of 16
 ]
 
 
