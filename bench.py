@@ -483,6 +483,8 @@ DECODE = {
     "decode_llm8b_gqa": dict(B=32, Hq=32, Hkv=8, D=128, ctx=8192, page=64, layout="NHD"),
     "decode_llm8b_gqa_hnd": dict(B=32, Hq=32, Hkv=8, D=128, ctx=8192, page=64, layout="HND"),
     "decode_llm8b_b1_32k": dict(B=1, Hq=32, Hkv=8, D=128, ctx=32768, page=64, layout="NHD"),
+    # 4 new tokens per sequence in one step (proposed tokens checked together)
+    "decode_llm8b_gqa_q4": dict(B=32, Hq=32, Hkv=8, D=128, ctx=8192, page=64, layout="NHD", q_len=4),
 }
 
 
@@ -494,20 +496,24 @@ def time_decode(aa, name, dev, steps, flush, hbm_gbs):
 
     c = DECODE[name]
     B, Hq, Hkv, D, ctx, page = c["B"], c["Hq"], c["Hkv"], c["D"], c["ctx"], c["page"]
+    T = c.get("q_len", 1)  # new tokens per sequence
     g = torch.Generator().manual_seed(4000)
     max_pages = ctx // page
     num_pages = B * max_pages
-    q = torch.randn((B, Hq, D), generator=g).to(torch.bfloat16).to(dev)
+    q = torch.randn((B, Hq, D) if T == 1 else (B, T, Hq, D), generator=g).to(torch.bfloat16).to(dev)
     kc = torch.randn((num_pages, page, Hkv, D), generator=g).to(torch.bfloat16).to(dev)
     vc = torch.randn((num_pages, page, Hkv, D), generator=g).to(torch.bfloat16).to(dev)
     hnd = c["layout"] == "HND"
     if hnd:
         kc, vc = kc.transpose(1, 2).contiguous(), vc.transpose(1, 2).contiguous()
     call = aa.axis_attn_decode_hnd if hnd else aa.axis_attn_decode
+    if T > 1:
+        call = aa.axis_attn_decode_q
     table = torch.randperm(num_pages, generator=g).to(torch.int32).reshape(B, max_pages).to(dev)
     lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
-    o, lse = torch.empty_like(q), torch.empty((B, Hq), device=dev, dtype=torch.float32)
-    need = aa.axis_attn_decode_workspace_bytes(B, Hq, Hkv, D, page, max_pages)
+    o, lse = torch.empty_like(q), torch.empty((B, Hq, T), device=dev, dtype=torch.float32)
+    need = (aa.axis_attn_decode_workspace_bytes(B, Hq, Hkv, D, page, max_pages) if T == 1
+            else aa.axis_attn_decode_q_workspace_bytes(B, T, Hq, Hkv, D, page, max_pages))
     ws = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
     st = torch.cuda.current_stream(dev)
     import ctypes
@@ -515,9 +521,13 @@ def time_decode(aa, name, dev, steps, flush, hbm_gbs):
     sp = ctypes.c_void_p(st.cuda_stream)
     # the C ABI straight (as the main step does): the torch helper's checks would run on the host
     # between the events while the GPU waits, and count as device time
-    args = (q.data_ptr(), kc.data_ptr(), vc.data_ptr(), table.data_ptr(), lens.data_ptr(), o.data_ptr(),
-            lse.data_ptr(), B, Hq, Hkv, D, page, max_pages, num_pages, 1.0 / math.sqrt(D), ws.data_ptr(),
-            ws.numel(), sp)
+    ptrs = (q.data_ptr(), kc.data_ptr(), vc.data_ptr(), table.data_ptr(), lens.data_ptr(), o.data_ptr(),
+            lse.data_ptr())
+    if T == 1:
+        args = ptrs + (B, Hq, Hkv, D, page, max_pages, num_pages, 1.0 / math.sqrt(D), ws.data_ptr(), ws.numel(), sp)
+    else:
+        args = ptrs + (B, T, Hq, Hkv, D, page, max_pages, num_pages, 1.0 / math.sqrt(D), int(hnd), ws.data_ptr(),
+                       ws.numel(), sp)
     ev = []
     for n in range(3 + steps):
         flush.fill_(n & 0xFF)
@@ -532,10 +542,10 @@ def time_decode(aa, name, dev, steps, flush, hbm_gbs):
     torch.cuda.synchronize()
     aa.check_status(st)
     ms = sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev)
-    nbytes = B * ctx * Hkv * D * 2 * 2 + 2 * B * Hq * D * 2
+    nbytes = B * ctx * Hkv * D * 2 * 2 + 2 * B * T * Hq * D * 2
     gbs = nbytes / (ms * 1e-3) / 1e9
-    return {"config": f"B={B} Hq={Hq} Hkv={Hkv} D={D} context={ctx} page_size={page} (bf16 paged cache, "
-                      f"{c['layout']} pages, random page order)", "ms": ms, "steps": steps, "algorithmic_bytes": nbytes,
+    return {"config": f"B={B} Hq={Hq} Hkv={Hkv} D={D} context={ctx} page_size={page} new_tokens={T} (bf16 paged "
+                      f"cache, {c['layout']} pages, random page order)", "ms": ms, "steps": steps, "algorithmic_bytes": nbytes,
             "launches_per_call": 2 if need > 0 else 1,  # the decode kernel, and the split merge when it splits
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs}}
 
