@@ -186,6 +186,10 @@ CASES_Q = [
     # key of the last split, whose partial result must weigh nothing
     (1, 16, 2, 2, 64, 8320, 32, [8200]),
     (2, 8, 32, 4, 64, 500, 16, [500, 9]),              # G = 8: 64 rows -> 4 tiles of 16
+    # 16-row tiles with more items than the deep configuration takes in one wave
+    # (the wide kernel): 320 items at D = 64, 384 at D = 128
+    (80, 4, 16, 4, 64, 200, 16, [200, 4, 63, 150] * 20),
+    (48, 8, 16, 8, 128, 300, 32, [300, 8, 100, 257] * 12),
 ]
 
 
