@@ -16,12 +16,13 @@
 //     query tile that can see the keys.  Per tile (two threads issue the
 //     MMAs, one the score products, one the gradient products):
 //       S^T = K Q^T and dP^T = V dO^T into TMEM (thread = key row),
-//       P^T = 2^(S^T c - LSE2), dS^T = P^T (dP^T - Dr) by 8 warps from TMEM,
+//       P^T = 2^(S^T c - LSE2), dS^T = P^T (dP^T - Dr) by the compute warps
+//       (16 at D = 64, 8 at D = 128) from TMEM,
 //       formed as scale dS^T = P^T (scale dP^T - scale Dr) (the preprocess
 //       stores -scale Dr), so dQ and dK leave their products scaled,
 //       P^T back to TMEM (bf16), dS^T to shared memory (bf16, 128B swizzle),
 //       dV += P^T dO (A from TMEM), dK += dS^T Q, and dQ of the tile,
-//     the compute warps copy each dQ tile from TMEM into a swizzled
+//     four read-out warps copy each dQ tile from TMEM into a swizzled
 //     shared-memory staging tile, which one thread adds into the fp32
 //     accumulator with TMA reduce-add copies; dK, dV stay in TMEM until the
 //     end.  In the deterministic mode the kernel skips dQ altogether (the
@@ -210,16 +211,16 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
   auto bar_qfull = [&](int s) { return bars + 8u * (1 + s); };
   auto bar_qempty = [&](int s) { return bars + 8u * (1 + ST + s); };
   const uint32_t bar_spfull = bars + 8u * (1 + 2 * ST);   // S^T, dP^T of a step are in TMEM
-  const uint32_t bar_spfree = bars + 8u * (2 + 2 * ST);   // ... and have been read (8 warps)
-  const uint32_t bar_pdsfull = bars + 8u * (3 + 2 * ST);  // P^T (TMEM), dS^T (smem) written (8 warps)
+  const uint32_t bar_spfree = bars + 8u * (2 + 2 * ST);   // ... and have been read (the compute warps)
+  const uint32_t bar_pdsfull = bars + 8u * (3 + 2 * ST);  // P^T (TMEM), dS^T (smem) written (the compute warps)
   const uint32_t bar_ptfree = bars + 8u * (4 + 2 * ST);   // dV of a step is done with P^T
   const uint32_t bar_dqfull = bars + 8u * (5 + 2 * ST);   // dQ tile of a step is in TMEM
-  const uint32_t bar_dqfree = bars + 8u * (6 + 2 * ST);   // ... and has been read (8 warps)
+  const uint32_t bar_dqfree = bars + 8u * (6 + 2 * ST);   // ... and has been read (4 read-out warps)
   const uint32_t bar_fin = bars + 8u * (7 + 2 * ST);
   // dK, dQ of a step are done with dS^T buffer x
   auto bar_dstfree = [&](int x) { return bars + 8u * (x == 0 ? 8 + 2 * ST : 11 + 2 * ST); };
   auto sDSB = [&](int it) { return sDST + (uint32_t)(it % C::NDS) * C::PS_BYTES; };  // dS^T buffer of step it
-  const uint32_t bar_stgfull = bars + 8u * (9 + 2 * ST);  // dQ tile staged (8 warps)
+  const uint32_t bar_stgfull = bars + 8u * (9 + 2 * ST);  // dQ tile staged (4 read-out warps)
   const uint32_t bar_stgfree = bars + 8u * (10 + 2 * ST); // staged tile read by the TMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 8 * C::NBAR);
   volatile WaitCtl* abort = reinterpret_cast<volatile WaitCtl*>(gbase + C::OFF_BAR + 8 * C::NBAR + 4);
