@@ -143,8 +143,9 @@ enum DecSite { D_EMPTY = 41, D_FULL };
 struct DecItem {
   int b, kv, split, rt, k0, k1, n_pieces, len;
 };
-// q_len, n_rt: the launch's (compile-time 1, 1 in the one-token instantiation)
-__device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report, int q_len, int n_rt) {
+// The item's indices (no memory access).  q_len, n_rt: the launch's
+// (compile-time 1, 1 in the one-token instantiation).
+__device__ __forceinline__ DecItem dec_index(const DecArgs& a, int w, int n_rt) {
   DecItem it;
   it.rt = w % n_rt;
   w /= n_rt;
@@ -152,6 +153,11 @@ __device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report
   const int bkv = w / a.n_splits;
   it.b = bkv / a.Hkv;
   it.kv = bkv % a.Hkv;
+  it.k0 = it.split * a.keys_per_split;
+  return it;
+}
+// ... and its length (one load), key range and pieces.
+__device__ __forceinline__ void dec_length(const DecArgs& a, DecItem& it, bool report, int q_len) {
   int len = a.seq_lens[it.b];
   const int cap = a.max_pages * a.page_size;
   if (len < q_len || len > cap) {  // clamped (cap >= q_len); reported once (by the producer)
@@ -159,9 +165,12 @@ __device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report
     len = len < q_len ? q_len : cap;
   }
   it.len = len;
-  it.k0 = it.split * a.keys_per_split;
   it.k1 = min(len, it.k0 + a.keys_per_split);
   it.n_pieces = it.k1 > it.k0 ? (it.k1 - it.k0 + 31) / 32 : 0;
+}
+__device__ __forceinline__ DecItem dec_item(const DecArgs& a, int w, bool report, int q_len, int n_rt) {
+  DecItem it = dec_index(a, w, n_rt);
+  dec_length(a, it, report, q_len);
   return it;
 }
 
@@ -225,9 +234,19 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP, MODE>::THREADS, DecCfg<HD, DE
     const int ps_mask = a.page_size - 1;
     int g = 0;  // pieces issued (over all items); the same in every lane
     bool ok = true;
+    const int cap = a.max_pages * a.page_size;
     for (int w = (int)blockIdx.x; ok && w < n_items; w += (int)gridDim.x) {
-      const DecItem I = dec_item(a, w, lane == 0, q_len, n_rt);
+      DecItem I = dec_index(a, w, n_rt);
       const int* row_tbl = a.block_table + (size_t)I.b * a.max_pages;
+      // the block-table entries of the item's first 32 pieces, loaded together
+      // with its length (they do not depend on it; which of them are used does)
+      int page0[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int key = I.k0 + 32 * lane + x * rows;
+        page0[x] = x < nbox && key < cap ? row_tbl[key >> ps_shift] : 0;
+      }
+      dec_length(a, I, lane == 0, q_len);
       for (int t0 = 0; ok && t0 < I.n_pieces; t0 += 32) {
         const int kt = I.k0 + 32 * (t0 + lane);  // this lane's piece
         // boxes x < nload of this lane's piece: cache coordinates (c1[x], c2[x]) of box row 0
@@ -237,7 +256,7 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP, MODE>::THREADS, DecCfg<HD, DE
           const int key = kt + x * rows;
           c1[x] = c2[x] = 0;
           if (t0 + lane < I.n_pieces && x < nbox && key < I.k1) {
-            const int page = row_tbl[key >> ps_shift];
+            const int page = t0 == 0 ? page0[x] : row_tbl[key >> ps_shift];
             if (page < 0 || page >= a.num_pages) usable = 0;
             c1[x] = a.hnd ? (key & ps_mask) : I.kv;
             c2[x] = a.hnd ? page * a.Hkv + I.kv : page * a.page_size + (key & ps_mask);
