@@ -236,3 +236,28 @@ def test_decode_workspace_bytes(lib):
 ])
 def test_rope_rejects(lib, fn, args, code):
     assert getattr(aa, fn)(*args) == code
+
+
+def _decq(**over):
+    args = dict(q=A, k_cache=A, v_cache=A, block_table=A, seq_lens=A, o=A, lse=A, B=1, q_len=4, Hq=32, Hkv=8, D=128,
+                page_size=64, max_pages=128, num_pages=128, scale=0.088, head_major=0, workspace=A,
+                workspace_bytes=1 << 30, stream=None)
+    args.update(over)
+    return aa.axis_attn_decode_q(*args.values())
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), 1), (dict(seq_lens=A + 2), 2), (dict(q_len=0), 3), (dict(q_len=65), 4),
+    (dict(max_pages=1, page_size=8, q_len=9), 3), (dict(Hq=72, Hkv=8), 4), (dict(workspace=None), 5),
+])
+def test_decode_q_rejects(lib, over, code):
+    assert _decq(**over) == code
+
+
+def test_decode_q_workspace_bytes(lib):
+    # q_len = 1 is the one-token query; 4 tokens x G = 4 heads = 16 rows: one tile per kv head,
+    # so the same splits (B=1, 8 kv heads, 8192 keys: 32), and 4x the partial rows
+    one = aa.axis_attn_decode_workspace_bytes(1, 32, 8, 128, 64, 128)
+    assert aa.axis_attn_decode_q_workspace_bytes(1, 1, 32, 8, 128, 64, 128) == one
+    assert aa.axis_attn_decode_q_workspace_bytes(1, 4, 32, 8, 128, 64, 128) == 4 * one
+    assert aa.axis_attn_decode_q_workspace_bytes(1, 65, 32, 8, 128, 64, 128) == 0  # unsupported q_len

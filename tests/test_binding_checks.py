@@ -111,3 +111,21 @@ def test_decode_layouts_read_the_cache_shape_their_own_way():
     assert "v_cache" in str(e)
     e = dec_error("BHSD")
     assert "layout" in str(e)
+
+
+def test_decode_several_tokens_checks_shapes():
+    # q [B, q_len, Hq, D]: correct shapes stop at the device check, a wrong lse shape earlier
+    base = dict(q=bf(2, 3, 8, D), k_cache=bf(5, 16, 4, D), v_cache=bf(5, 16, 4, D),
+                block_table=torch.zeros(2, 3, dtype=torch.int32), seq_lens=torch.full((2,), 3, dtype=torch.int32))
+    with pytest.raises(aa.AxisAttnError) as e:
+        aa.attention_decode(*base.values())
+    assert e.value.code == 4 and "CUDA device" in str(e.value)
+    with pytest.raises(aa.AxisAttnError) as e:  # lse of a 4-D q is [B, Hq, q_len]
+        aa.attention_decode(*base.values(), lse=torch.zeros(2, 8))
+    assert "lse" in str(e.value)
+    with pytest.raises(aa.AxisAttnError) as e:  # out must be shaped like q
+        aa.attention_decode(*base.values(), out=bf(2, 8, D))
+    assert "out" in str(e.value)
+    with pytest.raises(aa.AxisAttnError) as e:  # a 5-D q is neither form
+        aa.attention_decode(bf(2, 3, 1, 8, D), *list(base.values())[1:])
+    assert "q must be" in str(e.value)
