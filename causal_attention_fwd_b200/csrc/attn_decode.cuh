@@ -198,6 +198,11 @@ __global__ void __launch_bounds__(DecCfg<HD, DEEP, MODE>::THREADS, DecCfg<HD, DE
   volatile WaitCtl* ctl = reinterpret_cast<volatile WaitCtl*>(gbase + C::OFF_BAR + 16 * NST + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The split merge (launched as this grid's programmatic dependent) may be
+  // scheduled now: its CTAs wait for this grid's completion and memory
+  // (griddepcontrol.wait) before reading a partial result, so only its launch
+  // latency overlaps this kernel.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // several new tokens per sequence, or one (MODE 0: q_len = 1 and one row
   // tile at compile time, the code of the one-token step)
   const int q_len = MULTI ? a.q_len : 1, n_rt = MULTI ? a.n_rt : 1;
@@ -525,6 +530,10 @@ __global__ void __launch_bounds__(256) attn_decode_combine_kernel(const float* _
   __shared__ float s_red[NW];
   __shared__ float s_o[NW][HD];
   const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
+  // launched as the decode kernel's programmatic dependent: wait until that
+  // grid has completed and its partial results are visible (a no-op when
+  // launched in the ordinary way)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   for (int bh = (int)blockIdx.x; bh < rows; bh += (int)gridDim.x) {
     const float* p = part + (size_t)bh * n_splits * (HD + 2);
     // the maximum over the splits that saw keys (l > 0; a split past the end of the sequence has none)

@@ -792,11 +792,26 @@ int run_decode(const void* q, const void* k_cache, const void* v_cache, const in
   if (rc || sp.n_splits == 1) return rc;
   const int rows = B * q_len * Hq;
   const unsigned grid = (unsigned)(rows < 148 * 8 ? rows : 148 * 8);  // one CTA per (b, new token, h) row
-  if (D == 64)
-    attn_decode_combine_kernel<64><<<grid, 256, 0, st>>>(a.part, a.o, lse, rows, sp.n_splits, Hq, q_len);
-  else
-    attn_decode_combine_kernel<128><<<grid, 256, 0, st>>>(a.part, a.o, lse, rows, sp.n_splits, Hq, q_len);
-  return cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
+  // programmatic dependent launch: the merge grid is scheduled while the decode
+  // grid runs and waits in its first instruction for that grid's results
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  float* part = a.part;
+  __nv_bfloat16* out = a.o;
+  const int ns = sp.n_splits;
+  const cudaError_t e = D == 64 ? cudaLaunchKernelEx(&cfg, attn_decode_combine_kernel<64>, (const float*)part, out,
+                                                     lse, rows, ns, Hq, q_len)
+                                : cudaLaunchKernelEx(&cfg, attn_decode_combine_kernel<128>, (const float*)part, out,
+                                                     lse, rows, ns, Hq, q_len);
+  return e == cudaSuccess && cudaPeekAtLastError() == cudaSuccess ? AXIS_ATTN_OK : AXIS_ATTN_ERR_CUDA;
 }
 }  // namespace
 }  // namespace axis_attn
