@@ -136,6 +136,50 @@ struct BwdCfg {
 #define AXIS_ATTN_BWD_POLY_MASK 0x0000
 #endif
 
+// P^T and dS^T of one chunk of a compute thread's key row (SUBW query columns
+// from q_first): p = 2^(s c - LSE2) and scale dS = p (scale dp - scale Dr),
+// each packed to bf16 pairs.  lse, dr: the staged -LSE2 and -scale Dr of those
+// columns.  MASK (the diagonal or ragged step): p = 0 where the key lies above
+// the query (causal) or past S; a template parameter, so that the other steps
+// test nothing per pair.
+template <int SUBW, bool MASK, bool CAUSAL>
+__device__ __forceinline__ void bwd_chunk_math(const uint32_t (&sv)[SUBW], const uint32_t (&dpv)[SUBW],
+                                               const float* lse, const float* dr, uint64_t cc2, uint64_t sc2,
+                                               int key, int q_first, int S, uint32_t (&pk)[SUBW / 2],
+                                               uint32_t (&dk)[SUBW / 2]) {
+#pragma unroll
+  for (int e = 0; e < SUBW; e += 4) {
+    const float4 l4 = *reinterpret_cast<const float4*>(lse + e);
+    const float4 d4 = *reinterpret_cast<const float4*>(dr + e);
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int ee = e + 2 * h2;
+      const uint64_t nl = h2 ? f2_pack(l4.z, l4.w) : f2_pack(l4.x, l4.y);
+      const uint64_t nd = h2 ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y);
+      const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[ee]), __uint_as_float(sv[ee + 1])), cc2, nl);
+      float p0, p1;
+      if ((AXIS_ATTN_BWD_POLY_MASK >> (ee / 2)) & 1) {
+        f2_unpack(f2_exp2_poly(x), p0, p1);
+      } else {
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+      }
+      if constexpr (MASK) {
+        const int q = q_first + ee;
+        if ((CAUSAL && key > q) || key >= S) p0 = 0.f;
+        if ((CAUSAL && key > q + 1) || key >= S) p1 = 0.f;
+      }
+      const uint64_t pp = f2_pack(p0, p1);
+      const uint64_t dd =
+          f2_mul(pp, f2_fma(f2_pack(__uint_as_float(dpv[ee]), __uint_as_float(dpv[ee + 1])), sc2, nd));
+      pk[ee / 2] = pack_bf16x2(pp);
+      dk[ee / 2] = pack_bf16x2(dd);
+    }
+  }
+}
+
 // Warps 0 .. CW-1: P^T / dS^T (thread = key row); CW loads; CW+1 issues the
 // score MMAs and owns TMEM; CW+2 issues the TMA reduce-adds of the dQ tiles
 // into the fp32 accumulator; CW+3 issues the gradient MMAs; CW+4 .. CW+7 copy
@@ -508,37 +552,13 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
           if (lane == 0) mbar_arrive(bar_spfree);
         }
         uint32_t pk[SUBW / 2], dk[SUBW / 2];
-#pragma unroll
-        for (int e = 0; e < SUBW; e += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse_t + SUBW * cc + e);
-          const float4 d4 = *reinterpret_cast<const float4*>(dr_t + SUBW * cc + e);
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int ee = e + 2 * h2;
-            const uint64_t nl = h2 ? f2_pack(l4.z, l4.w) : f2_pack(l4.x, l4.y);
-            const uint64_t nd = h2 ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y);
-            const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[ee]), __uint_as_float(sv[ee + 1])), cc2, nl);
-            float p0, p1;
-            if ((AXIS_ATTN_BWD_POLY_MASK >> (ee / 2)) & 1) {
-              f2_unpack(f2_exp2_poly(x), p0, p1);
-            } else {
-              float x0, x1;
-              f2_unpack(x, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
-            if (need_mask) {
-              const int q = q0 + c0 + SUBW * cc + ee;
-              if ((CAUSAL && key > q) || key >= a.S) p0 = 0.f;
-              if ((CAUSAL && key > q + 1) || key >= a.S) p1 = 0.f;
-            }
-            const uint64_t pp = f2_pack(p0, p1);
-            const uint64_t dd =
-                f2_mul(pp, f2_fma(f2_pack(__uint_as_float(dpv[ee]), __uint_as_float(dpv[ee + 1])), sc2, nd));
-            pk[ee / 2] = pack_bf16x2(pp);
-            dk[ee / 2] = pack_bf16x2(dd);
-          }
-        }
+        // the mask test once per chunk, not per pair (need_mask is the same for the whole step)
+        if (need_mask)
+          bwd_chunk_math<SUBW, true, CAUSAL>(sv, dpv, lse_t + SUBW * cc, dr_t + SUBW * cc, cc2, sc2, key,
+                                             q0 + c0 + SUBW * cc, a.S, pk, dk);
+        else
+          bwd_chunk_math<SUBW, false, CAUSAL>(sv, dpv, lse_t + SUBW * cc, dr_t + SUBW * cc, cc2, sc2, key,
+                                              q0 + c0 + SUBW * cc, a.S, pk, dk);
         // the previous step's dV must be done with P^T before it is overwritten
         if (cc == 0 && it > 0 && !wait_warp(bar_ptfree, (it - 1) & 1, abort, B_PDSFREE)) {
           ok = false;
