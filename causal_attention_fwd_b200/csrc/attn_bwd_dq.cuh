@@ -59,6 +59,29 @@ constexpr int DQ_WARP_MMA = 17;
 
 enum DqSite { Q_Q = 61, Q_KEMPTY, Q_VEMPTY, Q_KFULL, Q_VFULL, Q_SFREE, Q_DSFULL, Q_SFULL, Q_DSFREE, Q_FIN };
 
+// scale dS of one thread's 32 key columns of a tile: p = 2^(s c - LSE2),
+// ds = p (scale dp - scale Dr), packed to bf16 pairs.  MASK (the diagonal or
+// ragged tile): columns from limit on get p = 0; a template parameter, so that
+// the other tiles test nothing per pair.
+template <bool MASK>
+__device__ __forceinline__ void dq_tile_math(const uint32_t (&sv)[32], const uint32_t (&dpv)[32], uint64_t cc2,
+                                             uint64_t nl2_2, uint64_t sc2, uint64_t ndr2, int limit,
+                                             uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    float x0, x1;
+    f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), cc2, nl2_2), x0, x1);
+    float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+    if constexpr (MASK) {
+      if (2 * e >= limit) p0 = 0.f;
+      if (2 * e + 1 >= limit) p1 = 0.f;
+    }
+    const uint64_t ds =
+        f2_mul(f2_pack(p0, p1), f2_fma(f2_pack(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1])), sc2, ndr2));
+    pk[e] = pack_bf16x2(ds);
+  }
+}
+
 template <int HD, bool CAUSAL>
 __global__ void __launch_bounds__(DQ_THREADS, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -236,19 +259,11 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
         if (CAUSAL && row_g + 1 - (128 * j + 32 * qc) < limit) limit = row_g + 1 - (128 * j + 32 * qc);
       }
       uint32_t pk[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        float x0, x1;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), cc2, nl2_2), x0, x1);
-        float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-        if (masked) {
-          if (2 * e >= limit) p0 = 0.f;
-          if (2 * e + 1 >= limit) p1 = 0.f;
-        }
-        const uint64_t ds =
-            f2_mul(f2_pack(p0, p1), f2_fma(f2_pack(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1])), sc2, ndr2));
-        pk[e] = pack_bf16x2(ds);
-      }
+      // the mask test once per tile, not per pair (masked is the same for the whole tile)
+      if (masked)
+        dq_tile_math<true>(sv, dpv, cc2, nl2_2, sc2, ndr2, limit, pk);
+      else
+        dq_tile_math<false>(sv, dpv, cc2, nl2_2, sc2, ndr2, limit, pk);
       // dS into its buffer (the dQ MMA of j - NDS must be done with it)
       const int x = j % NDS;
       if (j >= NDS && !wait_warp<true>(bar_dsfree(x), ((j / NDS) - 1) & 1, abort, Q_DSFREE)) { ok = false; break; }
