@@ -1,5 +1,5 @@
-// attn_decode.cuh -- decode step: one new query row per sequence against its
-// paged KV cache, and the combine of split partial results.
+// attn_decode.cuh -- decode step: one (or a few) new query rows per sequence
+// against its paged KV cache, and the combine of split partial results.
 //
 // What it computes is the step the axiomlm inference engine repeats per
 // generated token (axiomlm page, Key Features: "State-cached Key-Value (KV)
@@ -39,7 +39,7 @@
 // every row masked at its own position, and the tiles of a kv head, adjacent
 // in the item order, stream the same pieces (the later reads hit L2).
 // Page indices and sequence lengths are device data: a page index outside
-// [0, num_pages) or a length outside [1, max_pages * page_size] is never used
+// [0, num_pages) or a length outside [q_len, max_pages * page_size] is never used
 // for an access; it sets bit 1 of the device status word (reported by
 // axis_attn_get_status as AXIS_ATTN_ERR_INDEX) and the piece is skipped.
 #pragma once
@@ -57,7 +57,8 @@ struct DecArgs {
   float* part;             // [B * q_len * Hq][n_splits][D + 2]: m, l, O (n_splits > 1)
   int B, Hq, Hkv, G, page_size, max_pages, num_pages;
   int q_len;               // new tokens per sequence: the last q_len positions
-  int n_rt;                // row tiles per (b, kv head): ceil(G * q_len / 8) of 8 (token, head) rows
+  int n_rt;                // row tiles per (b, kv head): 1 with at most 8 (token, head) rows, else
+                           // ceil(G * q_len / 16) tiles of 16
   int hnd;                 // cache layout: 0 [pages, page_size, Hkv, D]; 1 [pages, Hkv, page_size, D]
   int keys_per_split;      // a multiple of 32
   int n_splits;
@@ -69,9 +70,10 @@ struct DecArgs {
 // bytes in flight are its CTAs x stages x piece bytes.  Two configurations per
 // head dim, chosen per call by the host:
 //   * wide (many small CTAs per SM) when the items fill them: measured at page
-//     size 16 to 64 (HBM fraction), D = 64 4 warps x 4 stages (5 CTAs / SM)
-//     0.79-0.91 against 0.70-0.72 with 8 stages (3 CTAs / SM); D = 128 1 warp
-//     x 2 stages (5 CTAs / SM) 0.94-0.98 against 0.90-0.96 with 4 x 4;
+//     size 16 to 64 (HBM fraction), D = 64 4 warps x 4 stages (4 CTAs / SM, by
+//     registers) 0.79-0.91 against 0.70-0.72 with 8 stages (3 CTAs / SM);
+//     D = 128 1 warp x 2 stages (5 CTAs / SM) 0.94-0.98 against 0.90-0.96 with
+//     4 x 4;
 //   * deep (fewer CTAs, more stages each) when a small batch leaves most of
 //     the wide configuration's CTAs without an item.
 #ifndef AXIS_ATTN_DEC_CW64
