@@ -261,3 +261,30 @@ def test_decode_q_workspace_bytes(lib):
     assert aa.axis_attn_decode_q_workspace_bytes(1, 1, 32, 8, 128, 64, 128) == one
     assert aa.axis_attn_decode_q_workspace_bytes(1, 4, 32, 8, 128, 64, 128) == 4 * one
     assert aa.axis_attn_decode_q_workspace_bytes(1, 65, 32, 8, 128, 64, 128) == 0  # unsupported q_len
+
+
+def _dec_q_rule(B, q_len, Hq, Hkv, D, page_size, max_pages):
+    """The documented rule: one tile of rows when a kv head has at most 8 (token, head) rows, else
+    tiles of 16; splits give at least 296 items of at least 256 keys; partial rows are (b, token, h)."""
+    G = Hq // Hkv
+    n_rt = 1 if G * q_len <= 8 else -(-(G * q_len) // 16)
+    keys = max_pages * page_size
+    units = B * Hkv * n_rt
+    n = min(-(-296 // units), -(-keys // 256))
+    n = max(n, 1)
+    kps = -(-(-(-keys // n)) // 32) * 32
+    n = -(-keys // kps)
+    return B * q_len * Hq * n * (D + 2) * 4 if n > 1 else 0
+
+
+@pytest.mark.parametrize("B,q_len,Hq,Hkv,D,ps,mp", [
+    (1, 2, 32, 8, 128, 64, 128),    # 8 rows: one tile, as for one token
+    (1, 3, 32, 8, 128, 64, 128),    # 12 rows: one tile of 16
+    (1, 8, 64, 8, 128, 64, 128),    # 64 rows: four tiles, fewer splits
+    (2, 16, 8, 8, 64, 16, 512),     # G = 1: 16 rows
+    (64, 4, 32, 8, 128, 16, 38),    # many units: no split
+    (3, 64, 24, 8, 64, 8, 2048),    # the largest q_len
+])
+def test_decode_q_workspace_follows_the_rule(lib, B, q_len, Hq, Hkv, D, ps, mp):
+    assert aa.axis_attn_decode_q_workspace_bytes(B, q_len, Hq, Hkv, D, ps, mp) == _dec_q_rule(
+        B, q_len, Hq, Hkv, D, ps, mp)
