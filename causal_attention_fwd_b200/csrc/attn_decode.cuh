@@ -122,9 +122,10 @@ struct DecCfg {
   static_assert(NST % CW == 0, "ring depth must be a multiple of the compute warps");
   // Resident CTAs per SM the registers must allow (0: no bound).  The wide
   // D = 64 configuration (160 threads) fits 4 per SM only at <= 102 registers
-  // a thread; left alone ptxas takes 125 and 3 fit (page size 16: 58.6 us
-  // against 52.8 us with the bound, at a few dozen bytes of spills).
-  static constexpr int MIN_CTAS = (HD == 64 && !DEEP && MODE != 2) ? 4 : 0;
+  // a thread; left alone ptxas takes 125-128 and 3 fit (page size 16: 58.6 us
+  // against 52.8 us with the bound, at a few dozen bytes of spills; 4 new
+  // tokens per sequence in 16-row tiles: 63.2 against 56.3 us).
+  static constexpr int MIN_CTAS = (HD == 64 && !DEEP) ? 4 : 0;
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = NST * PIECE;
   static constexpr uint32_t OFF_C = 2 * NST * PIECE;              // fp32 [CW][RT][HD + 2]
